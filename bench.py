@@ -1,0 +1,397 @@
+"""Benchmark of the KDA forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One JSON line on rank 0.  Headline: prefill tokens/s on the long-context
+workload (1 x 131072 tokens, H=32, dk=dv=128, bf16), one kda_chunk_fwd call
+per step, inputs resident in HBM and larger than L2 (6.4 GB read per step).
+Alongside: the decode step (256 sequences x 32 heads, 512 MiB fp32 state,
+1000 consecutive in-place steps) as achieved HBM GB/s, the roofline of both
+against the measured peaks, an end-to-end figure through the same public
+call with host buffers, and the fp64 CPU oracle timed on a bounded sample.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own replica of
+the workload (sequences and heads are independent -- no data-path
+collective); value = tokens over all ranks / max-over-ranks device time.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from kda_linear_attention_fwd_b200 import kda  # noqa: E402
+from kda_linear_attention_fwd_b200 import workloads as W  # noqa: E402
+
+METRIC = "KDA prefill tokens/s (H=32,d=128) & decode-step state GB/s vs B200 roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def prefill_bytes(w, T, N):
+    """Algorithmic HBM bytes of one prefill call: read q, k, g, v, gate, beta,
+    write y (dtype), read the initial and write the final state (fp32)."""
+    e = 2 if w.dtype == "bf16" else 4
+    per_tok_head = (3 * w.dk + 3 * w.dv + 1) * e
+    states = N * w.H * w.dk * w.dv * 4 * ((1 if w.init_state else 0) + 1)
+    return T * w.H * per_tok_head + states
+
+
+def prefill_flops(w, T):
+    """Chunk-form FLOPs per token-head: the three state contractions
+    (W S, Qd S, Kb^T U: 6 dk dv) and the intra-chunk products
+    (Kd Ki^T, Qd Ki^T, W, U0, P U: 2 C (3 dk + 2 dv)), C = 16."""
+    C = 16
+    return T * w.H * (6 * w.dk * w.dv + 2 * C * (3 * w.dk + 2 * w.dv))
+
+
+def decode_bytes(wd):
+    nh = wd.num_seqs * wd.H
+    e = 2
+    return nh * (2 * wd.dk * wd.dv * 4 + (3 * wd.dk + 3 * wd.dv + 1) * e)
+
+
+class Clocks:
+    """nvidia-smi sampler for the timed region."""
+
+    def __init__(self, path):
+        self.path = path
+        self.proc = None
+
+    def start(self):
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(torch.cuda.current_device()).uuid)
+            q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", uuid, f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], None, set()
+        names = ["active", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for name, val in zip(names[1:], parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(name)
+        if not sm:
+            return None
+        load = [x for x in sm if mx is None or x > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(args):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def reduce_max(x, ws):
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_baseline(w, threads=None, tokens=None):
+    """The fp64 oracle on a bounded sample of the workload: all heads of the
+    first `tokens` tokens of one sequence.  Returns (tokens/s at H, cores,
+    sample description)."""
+    import numpy as np
+
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    cores = threads or os.cpu_count() or 1
+    if tokens is None:
+        tokens = int(min(w.lengths[0], max(4096, 512 * cores)))
+    with ThreadPoolExecutor(min(32, cores)) as ex:
+        heads = list(ex.map(lambda h: W.head_inputs(w, 0, h, length=tokens), range(w.H)))
+    st = lambda key: np.stack([x[key].numpy() for x in heads], axis=1)
+    q, k, v, g, gate = st("q"), st("k"), st("v"), st("g"), st("gate")
+    beta = np.stack([x["beta"].numpy() for x in heads], axis=1)
+    t0 = time.perf_counter()
+    _, _, used = oracle.varlen(q, k, v, g, beta, gate, [0, tokens], threads=cores)
+    dt = time.perf_counter() - t0
+    return tokens / dt, used, f"{tokens} tokens x {w.H} heads of {w.name} (fp64, per token)"
+
+
+def run_reference(args, ws, rank):
+    """Reference arm: the fp64 CPU oracle, timed on the host cores, on a
+    bounded sample of the same workload each step."""
+    if rank != 0:
+        return
+    w = W.get(args.workload)
+    cores = os.cpu_count() or 1
+    tokens = int(min(w.lengths[0], max(1024, 256 * cores)))
+    for _ in range(args.warmup):
+        cpu_baseline(w, cores, tokens)
+    vals = []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        v, used, sample = cpu_baseline(w, cores, tokens)
+        vals.append(v)
+    el = time.perf_counter() - t0
+    value = args.steps * tokens / el
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "seq_len": w.lengths[0], "heads": w.H,
+                       "dk": w.dk, "dv": w.dv, "sample_tokens_per_step": tokens},
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": used, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="long_bf16")
+    ap.add_argument("--decode-steps", type=int, default=1000)
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--out-dir", default=os.path.join(ROOT, "gpurun_out"))
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
+
+    ws, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        run_reference(args, ws, rank)
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+
+    from kda_linear_attention_fwd_b200 import build
+    if rank == 0:
+        build.build()
+    barrier(ws)
+    lib = kda.load()
+    pk, pk_kind = peaks()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+
+    # ---------------- prefill ----------------
+    w = W.get(args.workload)
+    T, N = w.total_tokens, w.num_seqs
+    inp = W.fast_prefill(w, seed=w.seed + 1000 * rank, device=dev)
+    out = torch.empty(T, w.H, w.dv, dtype=w.torch_dtype, device=dev)
+    fin = torch.empty(N, w.H, w.dk, w.dv, dtype=torch.float32, device=dev)
+    plan = kda.plan(T, N, w.H)
+    ws_bytes = kda.workspace_size(T, N, w.H, w.dk, w.dv, w.torch_dtype)
+    wsp = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    cu_host = inp["cu_seqlens"].tolist()
+
+    def prefill():
+        kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["gate"],
+                      inp["cu_seqlens"], initial_state=inp["initial_state"], final_state=fin,
+                      out=out, workspace=wsp, cu_seqlens_host=cu_host, stream=stream)
+
+    for _ in range(args.warmup):
+        prefill()
+    torch.cuda.synchronize()
+    os.makedirs(args.out_dir, exist_ok=True)
+    clocks = Clocks(os.path.join(args.out_dir, f"clocks_rank{rank}.csv"))
+    clocks.start()
+    barrier(ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        prefill()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    ms_total = reduce_max(e0.elapsed_time(e1), ws)
+    clk = clocks.stop()
+    ms = ms_total / args.steps
+    value = ws * T * args.steps / (ms_total / 1e3)
+    pbytes = prefill_bytes(w, T, N)
+    pflops = prefill_flops(w, T)
+    hbm = pk["hbm_gbs"]
+    achieved = pbytes / (ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                "frac": achieved / hbm, "traffic": None,
+                "kernel": "kda_chunk_fwd call (%d launches)" % plan["launches"],
+                "peak_source": f"{pk_kind} hbm_gbs",
+                "tensor_tflops": pflops / (ms / 1e3) / 1e12,
+                "tensor_frac_of_peak": pflops / (ms / 1e3) / 1e12 / pk["bf16_tflops"],
+                "roofline_model_frac": max(pbytes / (hbm * 1e9),
+                                           pflops / (pk["bf16_tflops"] * 1e12)) / (ms / 1e3)}
+
+    # ---------------- decode ----------------
+    dec = None
+    if not args.no_decode:
+        wd = W.get("decode_bf16")
+        S = args.decode_steps
+        dd = W.fast_decode(wd, S, seed=wd.seed + 1000 * rank, device=dev)
+        state = dd["state"]
+        yout = torch.empty(wd.num_seqs, wd.H, wd.dv, dtype=torch.bfloat16, device=dev)
+        P = ctypes.c_void_p
+        ptr = lambda t: P(t.data_ptr())
+        st_ptr = P(stream.cuda_stream)
+        calls = [(ptr(dd["q"][s]), ptr(dd["k"][s]), ptr(dd["v"][s]), ptr(dd["g"][s]),
+                  ptr(dd["beta"][s]), ptr(dd["gate"][s])) for s in range(S)]
+        yp, sp = ptr(yout), ptr(state)
+
+        def dstep(s):
+            a = calls[s]
+            rc = lib.kda_decode_step(a[0], a[1], a[2], a[3], a[4], a[5], yp, sp, wd.num_seqs,
+                                     wd.H, wd.dk, wd.dv, kda.KDA_DTYPE_BF16, 1.0, 0, st_ptr)
+            if rc != 0:
+                raise RuntimeError(kda.status_string(rc))
+
+        for s in range(3):
+            dstep(s)
+        torch.cuda.synchronize()
+        barrier(ws)
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d0.record(stream)
+        for s in range(S):
+            dstep(s)
+        d1.record(stream)
+        torch.cuda.synchronize()
+        barrier(ws)
+        dms = reduce_max(d0.elapsed_time(d1), ws)
+        us = 1e3 * dms / S
+        db = decode_bytes(wd)
+        gbs = db / (us / 1e6) / 1e9
+        dec = {"value": ws * gbs, "unit": "GB/s", "us_per_step": us, "steps": S,
+               "tokens_per_s": ws * wd.num_seqs * S / (dms / 1e3),
+               "workload": "decode_bf16: 256 seqs x H=32, dk=dv=128, 512 MiB fp32 state",
+               "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                            "frac": gbs / hbm, "traffic": None,
+                            "kernel": "decode_step_kernel<128,128,bf16>",
+                            "peak_source": f"{pk_kind} hbm_gbs"},
+                "gpu_launches": S}
+        del dd, state, calls
+
+    # ---------------- end to end (host buffers) ----------------
+    e2e = None
+    if not args.no_e2e:
+        names = ("q", "k", "v", "g", "beta", "gate")
+        host = {x: torch.empty(inp[x].shape, dtype=inp[x].dtype, pin_memory=True) for x in names}
+        for x in names:
+            host[x].copy_(inp[x])
+        hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        hfin = torch.empty(fin.shape, dtype=fin.dtype, pin_memory=True)
+        h2d = sum(host[x].numel() * host[x].element_size() for x in names)
+        d2h = hout.numel() * hout.element_size() + hfin.numel() * hfin.element_size()
+
+        def e2e_step():
+            for x in names:
+                inp[x].copy_(host[x], non_blocking=True)
+            prefill()
+            hout.copy_(out, non_blocking=True)
+            hfin.copy_(fin, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(ws)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        barrier(ws)
+        ems = reduce_max(a0.elapsed_time(a1), ws)
+        e2e = {"value": ws * T * args.e2e_steps / (ems / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": ems / args.e2e_steps, "steps": args.e2e_steps}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu:
+        v, used, sample = cpu_baseline(w)
+        cpu = {"value": v, "unit": "tokens/s", "cores": used, "kind": "oracle", "sample": sample}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": w.dtype, "data": "synthetic",
+                "config": {"workload": f"{w.name}: {N} x {T} tokens, H={w.H}, dk={w.dk}, "
+                                       f"dv={w.dv}, {w.dtype}, chunk=16",
+                           "global_batch": ws * N, "seq_len": T,
+                           "parallelism": f"replicas x{ws} (sequences/heads independent)",
+                           "l2": "inputs larger than L2 (%.1f GB per step)" % (pbytes / 1e9),
+                           "piece_len": plan["piece_len"]},
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": plan["launches"] * args.steps, "clocks": clk, "decode": dec}
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,147 @@
+/*
+ * kda.h -- KDA (Kimi Delta Attention) forward on NVIDIA B200 (sm_100a).
+ *
+ * A C-ABI library (libkda_b200.so).  Plain pointers and sizes only; every
+ * pointer is a DEVICE pointer unless its name ends in _host.  The caller owns
+ * every buffer.  All work is enqueued asynchronously on `stream`; the
+ * functions never allocate device memory and never synchronise the stream.
+ *
+ * The layer (Kimi K3 report explainer, affta.cn, section
+ * "第一关：KDA 解决算得动"): per (sequence n, head h) a fixed-size state
+ * S in R^{dk x dv} (fp32 here), and for every token t, in this order:
+ *   1. forget        S <- Diag(alpha_t) S,  alpha_t = exp(g_t) per key channel
+ *                    (channel-wise forget gate: each state direction decays at
+ *                    its own rate)
+ *   2. delta write   u = beta_t (v_t - S^T k_t);  S <- S + k_t u^T
+ *                    (read the state with the key, compare with the value,
+ *                    write only the error, scaled by the update strength)
+ *   3. read          o_t = S^T (scale q_t)
+ *   4. output gate   y_t = gate_t (.) o_t   (full-rank: one gate per channel)
+ *
+ * Decay floor (same page and section): a channel keeps at least about 0.67%
+ * of its state per step, i.e. ln(0.0067) <= g <= 0.  This is a PRECONDITION
+ * of kda_chunk_fwd (it is what keeps every decay ratio inside a 16-token
+ * chunk within BF16/FP32 range -- prism.simon-ai.net, "从架构创新出发：K3的MoE
+ * 与混合注意力设计", section "数值稳定性与 Co-Design：BF16 约束下的衰减控制策略").
+ * It is not checked on the device; values below the floor may overflow to
+ * inf/NaN in the output.  g must also be finite and <= 0.
+ *
+ * Layouts ("THD", packed variable length):
+ *   q, k, g   [total_tokens][H][dk]   contiguous, element type = dtype
+ *   v, gate   [total_tokens][H][dv]   contiguous, element type = dtype
+ *   beta      [total_tokens][H]       contiguous, element type = dtype
+ *   out       [total_tokens][H][dv]   contiguous, element type = dtype
+ *   cu_seqlens[num_seqs + 1] int32, cu_seqlens[0] = 0, non-decreasing,
+ *             cu_seqlens[num_seqs] = total_tokens.  Sequence n is tokens
+ *             [cu_seqlens[n], cu_seqlens[n+1]).  Chunks never cross a
+ *             sequence boundary.
+ *   states    [num_seqs][H][dk][dv]   fp32, dv contiguous.
+ *
+ * Supported sizes: dk, dv in {64, 128}; H >= 1; dtype BF16 or F32 (all of q,
+ * k, v, g, beta, gate, out share it; states are always fp32).  Arithmetic:
+ * fp32 accumulation and an fp32 state; BF16 inputs feed the tensor cores as
+ * bf16; F32 inputs are computed in fp32 throughout.  Output is rounded to
+ * nearest-even into dtype.
+ *
+ * Alignment: q, k, v, g, gate, out, states and workspace must be 16-byte
+ * aligned; beta must be aligned to its element size.  KDA_ERR_ALIGNMENT
+ * otherwise.
+ *
+ * Errors: every function validates its arguments on the host before launching
+ * anything; on a validation error nothing is launched.  After launching, the
+ * return value also reports cudaGetLastError() (KDA_ERR_CUDA).  Errors in
+ * kernels that run later are reported by later CUDA calls on the stream.
+ */
+#ifndef KDA_B200_H
+#define KDA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *kda_stream_t; /* == cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = -1, /* null pointer, negative size, inconsistent sizes */
+    KDA_ERR_UNSUPPORTED = -2, /* dk/dv/dtype outside the supported set */
+    KDA_ERR_ALIGNMENT = -3,   /* a pointer breaks the alignment rule above */
+    KDA_ERR_WORKSPACE = -4,   /* workspace NULL or smaller than required */
+    KDA_ERR_CUDA = -5,        /* a CUDA runtime call failed (launch, attribute) */
+    KDA_ERR_TIMEOUT = -6      /* reserved: a bounded device-side wait gave up */
+} kda_status;
+
+typedef enum { KDA_DTYPE_F32 = 0, KDA_DTYPE_BF16 = 1 } kda_dtype;
+
+/* Human-readable name of a kda_status value (static string, never NULL). */
+const char *kda_status_string(int status);
+
+/* Bytes of device workspace kda_chunk_fwd needs for these sizes on the
+ * current CUDA device (the plan depends on its SM count).  0 is never
+ * returned for a valid call; returns 0 for invalid sizes. */
+size_t kda_chunk_fwd_workspace_size(int32_t total_tokens, int32_t num_seqs, int32_t H,
+                                    int32_t dk, int32_t dv, kda_dtype dtype);
+
+/* The prefill plan for these sizes on the current CUDA device: the piece
+ * length (tokens; sequences longer than this are split into pieces whose
+ * states are combined by a prefix scan), an upper bound on the number of
+ * pieces, and the number of kernel launches one kda_chunk_fwd call makes.
+ * Any output pointer may be NULL.  Returns KDA_OK or KDA_ERR_INVALID_ARG. */
+int kda_chunk_fwd_plan(int32_t total_tokens, int32_t num_seqs, int32_t H, int32_t *piece_len,
+                       int32_t *max_pieces, int32_t *launches);
+
+/*
+ * Prefill: the layer over packed variable-length sequences, computed in
+ * 16-token chunks (within a chunk by whole-block matrix products, between
+ * chunks by carrying the state -- prism.simon-ai.net page, section
+ * "计算范式演进：从递归低效到 GPU 友好的 Chunk Recurrent"), with long
+ * sequences split into pieces whose state hand-offs are combined by a prefix
+ * scan (affta.cn page, section "KDA 上下文并行，让上下文的交接变薄";
+ * prism.simon-ai.net page, section "Linear Attention 的分层 Chunking 策略").
+ *
+ *   gate            may be NULL: y = o.
+ *   cu_seqlens      device copy (required).
+ *   cu_seqlens_host optional host copy; when given it is validated
+ *                   (monotone, ends at total_tokens) -> KDA_ERR_INVALID_ARG.
+ *   scale           multiplies q (1.0 = none).
+ *   qk_l2norm       0: q, k used as given.  1: each q_t and k_t is divided
+ *                   by sqrt(sum x^2 + 1e-6) first.
+ *   initial_state   NULL = zeros.
+ *   final_state     NULL = not written.  May alias initial_state exactly
+ *                   (in-place state update); no other aliasing is allowed.
+ *   workspace       >= kda_chunk_fwd_workspace_size(...) bytes; contents on
+ *                   entry are ignored and on exit unspecified.
+ * num_seqs == 0 or total_tokens == 0 with num_seqs > 0 is valid (empty
+ * sequences copy initial_state to final_state).
+ */
+int kda_chunk_fwd(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                  const void *gate, void *out, const int32_t *cu_seqlens,
+                  const int32_t *cu_seqlens_host, int32_t num_seqs, int32_t total_tokens,
+                  int32_t H, int32_t dk, int32_t dv, kda_dtype dtype, float scale,
+                  int32_t qk_l2norm, const float *initial_state, float *final_state,
+                  void *workspace, size_t workspace_bytes, kda_stream_t stream);
+
+/*
+ * Decode: one token per sequence, the recurrence above applied once, state
+ * updated in place.  Decode cost is this per-token state update
+ * (prism.simon-ai.net page, section "推理瓶颈与Kimi K3的针对性优化").
+ *
+ *   q, k, g    [num_seqs][H][dk];  v, gate, out [num_seqs][H][dv];
+ *   beta       [num_seqs][H];  gate may be NULL.
+ *   state      [num_seqs][H][dk][dv] fp32, read and overwritten.
+ * Same dtype, alignment and decay-floor rules as kda_chunk_fwd.  No
+ * workspace.  qk_l2norm as for kda_chunk_fwd.
+ */
+int kda_decode_step(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                    const void *gate, void *out, float *state, int32_t num_seqs, int32_t H,
+                    int32_t dk, int32_t dv, kda_dtype dtype, float scale, int32_t qk_l2norm,
+                    kda_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_B200_H */

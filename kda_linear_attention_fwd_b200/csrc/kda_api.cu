@@ -1,0 +1,203 @@
+// C-ABI entry points of libkda_b200.so (declared in include/kda.h): argument
+// validation, the piece plan, and the launch sequence.  No allocation, no
+// host synchronisation, no exceptions across the boundary.
+#include <cstdlib>
+#include <cstring>
+
+#include "../../include/kda.h"
+#include "kda_common.cuh"
+#include "kda_prefill.cuh"
+
+namespace kda {
+cudaError_t launch_decode(bool bf16, int dk, int dv, const void *q, const void *k, const void *v,
+                          const void *g, const void *beta, const void *gate, void *out,
+                          float *state, long nh, float scale, int l2, cudaStream_t st);
+cudaError_t launch_plan(const int32_t *cu, int num_seqs, int total_tokens, int piece_len, int P_max,
+                        int32_t *header, int32_t *seq_first, int4 *pieces, cudaStream_t st);
+cudaError_t launch_scan(const PrefillParams &p, int dk, int dv, cudaStream_t st);
+cudaError_t launch_prefill_simt(const PrefillParams &p, bool bf16, int dk, int dv, bool summaries,
+                                cudaStream_t st);
+}  // namespace kda
+
+namespace {
+
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+bool dim_ok(int d) { return d == 64 || d == 128; }
+
+int sm_count() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+    if (dev < 0 || dev >= 64) dev = 0;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+            cudaGetLastError();
+            n = 148;
+        }
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+long env_long(const char *name, long dflt) {
+    const char *s = std::getenv(name);
+    if (!s || !*s) return dflt;
+    char *end = nullptr;
+    const long v = std::strtol(s, &end, 10);
+    return (end && *end == 0 && v > 0) ? v : dflt;
+}
+
+// Piece length (tokens, multiple of 16, >= 256): enough independent
+// (piece, head) chains to cover the GPU about twice over, and no more --
+// every extra piece boundary costs a summary pass over the piece's tokens.
+int choose_piece_len(long total_tokens, int H) {
+    const long forced = env_long("KDA_PIECE_LEN", 0);
+    if (forced > 0) return (int)(((forced + 15) / 16) * 16);
+    const long chains = env_long("KDA_TARGET_CHAINS", 2L * sm_count());
+    long work = total_tokens * (long)H;
+    long L = (work + chains - 1) / chains;
+    L = ((L + 15) / 16) * 16;
+    if (L < 256) L = 256;
+    if (L > (1L << 30)) L = 1L << 30;
+    return (int)L;
+}
+
+long max_pieces(long total_tokens, int num_seqs, int piece_len) {
+    return (long)num_seqs + (total_tokens + piece_len - 1) / piece_len;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *kda_status_string(int status) {
+    switch (status) {
+        case KDA_OK: return "KDA_OK";
+        case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG";
+        case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED";
+        case KDA_ERR_ALIGNMENT: return "KDA_ERR_ALIGNMENT";
+        case KDA_ERR_WORKSPACE: return "KDA_ERR_WORKSPACE";
+        case KDA_ERR_CUDA: return "KDA_ERR_CUDA";
+        case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT";
+        default: return "KDA_ERR_UNKNOWN";
+    }
+}
+
+size_t kda_chunk_fwd_workspace_size(int32_t total_tokens, int32_t num_seqs, int32_t H, int32_t dk,
+                                    int32_t dv, kda_dtype dtype) {
+    if (total_tokens < 0 || num_seqs < 0 || H < 1 || !dim_ok(dk) || !dim_ok(dv)) return 0;
+    if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return 0;
+    const int L = choose_piece_len(total_tokens, H);
+    const long P = max_pieces(total_tokens, num_seqs, L);
+    return kda::workspace_layout(P, num_seqs, H, dk, dv).total;
+}
+
+int kda_chunk_fwd_plan(int32_t total_tokens, int32_t num_seqs, int32_t H, int32_t *piece_len,
+                       int32_t *max_pieces_out, int32_t *launches) {
+    if (total_tokens < 0 || num_seqs < 0 || H < 1) return KDA_ERR_INVALID_ARG;
+    const int L = choose_piece_len(total_tokens, H);
+    const long P = max_pieces(total_tokens, num_seqs, L);
+    if (piece_len) *piece_len = L;
+    if (max_pieces_out) *max_pieces_out = (int32_t)(P > 0x7fffffffL ? 0x7fffffffL : P);
+    if (launches) *launches = num_seqs == 0 ? 0 : (total_tokens > L ? 4 : 2);
+    return KDA_OK;
+}
+
+int kda_chunk_fwd(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                  const void *gate, void *out, const int32_t *cu_seqlens,
+                  const int32_t *cu_seqlens_host, int32_t num_seqs, int32_t total_tokens,
+                  int32_t H, int32_t dk, int32_t dv, kda_dtype dtype, float scale,
+                  int32_t qk_l2norm, const float *initial_state, float *final_state,
+                  void *workspace, size_t workspace_bytes, kda_stream_t stream_) {
+    cudaStream_t stream = (cudaStream_t)stream_;
+    if (num_seqs < 0 || total_tokens < 0 || H < 1) return KDA_ERR_INVALID_ARG;
+    if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_UNSUPPORTED;
+    if (qk_l2norm != 0 && qk_l2norm != 1) return KDA_ERR_INVALID_ARG;
+    if (num_seqs == 0) return total_tokens == 0 ? KDA_OK : KDA_ERR_INVALID_ARG;
+    if (!cu_seqlens) return KDA_ERR_INVALID_ARG;
+    if (total_tokens > 0 && (!q || !k || !v || !g || !beta || !out)) return KDA_ERR_INVALID_ARG;
+    const size_t esz = dtype == KDA_DTYPE_BF16 ? 2 : 4;
+    const void *a16[] = {q, k, v, g, gate, out, initial_state, final_state, workspace};
+    for (const void *p : a16)
+        if (p && !aligned(p, 16)) return KDA_ERR_ALIGNMENT;
+    if (beta && !aligned(beta, esz)) return KDA_ERR_ALIGNMENT;
+    if (!aligned(cu_seqlens, 4)) return KDA_ERR_ALIGNMENT;
+    const size_t state_bytes = (size_t)num_seqs * H * dk * dv * sizeof(float);
+    if (initial_state && final_state && initial_state != final_state) {
+        const char *a = (const char *)initial_state, *b = (const char *)final_state;
+        if (a < b + state_bytes && b < a + state_bytes) return KDA_ERR_INVALID_ARG;
+    }
+    if (cu_seqlens_host) {
+        if (cu_seqlens_host[0] != 0 || cu_seqlens_host[num_seqs] != total_tokens)
+            return KDA_ERR_INVALID_ARG;
+        for (int n = 0; n < num_seqs; ++n)
+            if (cu_seqlens_host[n + 1] < cu_seqlens_host[n]) return KDA_ERR_INVALID_ARG;
+    }
+    const int L = choose_piece_len(total_tokens, H);
+    const long P_max = max_pieces(total_tokens, num_seqs, L);
+    if (P_max > (1L << 30) || (long)H * P_max > (1L << 31)) return KDA_ERR_UNSUPPORTED;
+    const kda::WorkspaceLayout WL = kda::workspace_layout(P_max, num_seqs, H, dk, dv);
+    if (!workspace || workspace_bytes < WL.total) return KDA_ERR_WORKSPACE;
+
+    char *ws = (char *)workspace;
+    kda::PrefillParams p;
+    p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.gate = gate; p.out = out;
+    p.cu_seqlens = cu_seqlens;
+    p.header = (const int32_t *)(ws + WL.off_header);
+    p.seq_first = (const int32_t *)(ws + WL.off_seq_first);
+    p.pieces = (const int4 *)(ws + WL.off_pieces);
+    p.M = (float *)(ws + WL.off_M);
+    p.Szero = (float *)(ws + WL.off_Szero);
+    p.Sin = (float *)(ws + WL.off_Sin);
+    p.initial_state = initial_state;
+    p.final_state = final_state;
+    p.num_seqs = num_seqs;
+    p.H = H;
+    p.P_max = (int)P_max;
+    p.scale = scale;
+    p.qk_l2norm = qk_l2norm;
+
+    const bool bf16 = dtype == KDA_DTYPE_BF16;
+    cudaError_t e = kda::launch_plan(cu_seqlens, num_seqs, total_tokens, L, (int)P_max,
+                                     (int32_t *)(ws + WL.off_header),
+                                     (int32_t *)(ws + WL.off_seq_first),
+                                     (int4 *)(ws + WL.off_pieces), stream);
+    if (e != cudaSuccess) return KDA_ERR_CUDA;
+    const bool multi = total_tokens > L;  // some sequence may have >1 piece
+    if (multi) {
+        e = kda::launch_prefill_simt(p, bf16, dk, dv, true, stream);
+        if (e != cudaSuccess) return KDA_ERR_CUDA;
+        e = kda::launch_scan(p, dk, dv, stream);
+        if (e != cudaSuccess) return KDA_ERR_CUDA;
+    }
+    e = kda::launch_prefill_simt(p, bf16, dk, dv, false, stream);
+    if (e != cudaSuccess) return KDA_ERR_CUDA;
+    return KDA_OK;
+}
+
+int kda_decode_step(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                    const void *gate, void *out, float *state, int32_t num_seqs, int32_t H,
+                    int32_t dk, int32_t dv, kda_dtype dtype, float scale, int32_t qk_l2norm,
+                    kda_stream_t stream) {
+    if (num_seqs < 0 || H < 1) return KDA_ERR_INVALID_ARG;
+    if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_UNSUPPORTED;
+    if (qk_l2norm != 0 && qk_l2norm != 1) return KDA_ERR_INVALID_ARG;
+    if (num_seqs == 0) return KDA_OK;
+    if (!q || !k || !v || !g || !beta || !out || !state) return KDA_ERR_INVALID_ARG;
+    const size_t esz = dtype == KDA_DTYPE_BF16 ? 2 : 4;
+    const void *a16[] = {q, k, v, g, gate, out, state};
+    for (const void *p : a16)
+        if (p && !aligned(p, 16)) return KDA_ERR_ALIGNMENT;
+    if (!aligned(beta, esz)) return KDA_ERR_ALIGNMENT;
+    const long nh = (long)num_seqs * H;
+    if (nh > 0x7fffffffL) return KDA_ERR_UNSUPPORTED;
+    const cudaError_t e = kda::launch_decode(dtype == KDA_DTYPE_BF16, dk, dv, q, k, v, g, beta,
+                                             gate, out, state, nh, scale, qk_l2norm,
+                                             (cudaStream_t)stream);
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+}  // extern "C"

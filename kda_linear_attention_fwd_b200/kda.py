@@ -1,0 +1,149 @@
+"""ctypes binding of libkda_b200.so (see include/kda.h).
+
+Argument marshalling only: PyTorch supplies device memory and the current
+stream, every step of the layer runs in the library's CUDA kernels.  There is
+no CPU fallback; if the library is missing or no CUDA device is present the
+calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkda_b200.so")
+
+KDA_DTYPE_F32 = 0
+KDA_DTYPE_BF16 = 1
+
+EXPORTS = ("kda_status_string", "kda_chunk_fwd_workspace_size", "kda_chunk_fwd_plan",
+           "kda_chunk_fwd", "kda_decode_step")
+
+_lib = None
+
+
+class KdaError(RuntimeError):
+    def __init__(self, fn, status, msg):
+        super().__init__(f"{fn} failed: {msg} ({status})")
+        self.status = status
+
+
+def load(path: str = LIB_PATH):
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} not found: build it first (python -m kda_linear_attention_fwd_b200.build)")
+    lib = ctypes.CDLL(path)
+    P, i32, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+    lib.kda_status_string.argtypes = [ctypes.c_int]
+    lib.kda_status_string.restype = ctypes.c_char_p
+    lib.kda_chunk_fwd_workspace_size.argtypes = [i32, i32, i32, i32, i32, ctypes.c_int]
+    lib.kda_chunk_fwd_workspace_size.restype = sz
+    lib.kda_chunk_fwd_plan.argtypes = [i32, i32, i32, P, P, P]
+    lib.kda_chunk_fwd_plan.restype = ctypes.c_int
+    lib.kda_chunk_fwd.argtypes = [P, P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32,
+                                  ctypes.c_int, f32, i32, P, P, P, sz, P]
+    lib.kda_chunk_fwd.restype = ctypes.c_int
+    lib.kda_decode_step.argtypes = [P, P, P, P, P, P, P, P, i32, i32, i32, i32, ctypes.c_int,
+                                    f32, i32, P]
+    lib.kda_decode_step.restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load().kda_status_string(int(status)).decode()
+
+
+def _check(fn, status):
+    if status != 0:
+        raise KdaError(fn, status, status_string(status))
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return KDA_DTYPE_BF16
+    if t.dtype == torch.float32:
+        return KDA_DTYPE_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("all tensors must be CUDA tensors")
+
+
+def workspace_size(total_tokens, num_seqs, H, dk, dv, dtype=torch.bfloat16) -> int:
+    code = KDA_DTYPE_BF16 if dtype == torch.bfloat16 else KDA_DTYPE_F32
+    return int(load().kda_chunk_fwd_workspace_size(total_tokens, num_seqs, H, dk, dv, code))
+
+
+def plan(total_tokens, num_seqs, H) -> dict:
+    """Piece length, piece bound and launch count of one kda_chunk_fwd call."""
+    L, P, n = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+    _check("kda_chunk_fwd_plan", load().kda_chunk_fwd_plan(
+        total_tokens, num_seqs, H, ctypes.byref(L), ctypes.byref(P), ctypes.byref(n)))
+    return dict(piece_len=L.value, max_pieces=P.value, launches=n.value)
+
+
+def chunk_fwd(q, k, v, g, beta, gate, cu_seqlens, *, scale=1.0, qk_l2norm=False,
+              initial_state=None, final_state=None, out=None, workspace=None,
+              cu_seqlens_host=None, output_final_state=True, stream=None):
+    """Prefill over packed sequences.  q, k, g [T, H, dk]; v, gate [T, H, dv];
+    beta [T, H]; cu_seqlens int32 [N+1] (device).  Returns (out, final_state)."""
+    lib = load()
+    _require_cuda(q, k, v, g, beta, gate, cu_seqlens, initial_state, final_state, out, workspace)
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    N = cu_seqlens.shape[0] - 1
+    code = _dtype_code(q)
+    if out is None:
+        out = torch.empty(T, H, dv, dtype=q.dtype, device=q.device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty(N, H, dk, dv, dtype=torch.float32, device=q.device)
+    need = int(lib.kda_chunk_fwd_workspace_size(T, N, H, dk, dv, code))
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    host = None
+    if cu_seqlens_host is not None:
+        host_arr = (ctypes.c_int32 * len(cu_seqlens_host))(*[int(x) for x in cu_seqlens_host])
+        host = ctypes.cast(host_arr, ctypes.c_void_p)
+    st = lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(gate), _ptr(out),
+                           _ptr(cu_seqlens), host, N, T, H, dk, dv, code, float(scale),
+                           int(bool(qk_l2norm)), _ptr(initial_state), _ptr(final_state),
+                           _ptr(workspace), workspace.numel() * workspace.element_size(),
+                           _stream(stream))
+    _check("kda_chunk_fwd", st)
+    return out, final_state
+
+
+def decode_step(q, k, v, g, beta, gate, state, *, scale=1.0, qk_l2norm=False, out=None,
+                stream=None):
+    """One token per sequence.  q, k, g [N, H, dk]; v, gate [N, H, dv]; beta
+    [N, H]; state [N, H, dk, dv] fp32, updated in place.  Returns out."""
+    lib = load()
+    _require_cuda(q, k, v, g, beta, gate, state, out)
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    if out is None:
+        out = torch.empty(N, H, dv, dtype=q.dtype, device=q.device)
+    st = lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(gate),
+                             _ptr(out), _ptr(state), N, H, dk, dv, _dtype_code(q), float(scale),
+                             int(bool(qk_l2norm)), _stream(stream))
+    _check("kda_decode_step", st)
+    return out

@@ -170,59 +170,54 @@ def _select(w: Workload, heads):
 
 
 def pack_prefill(w: Workload, heads=None, device="cpu", threads: int = 0) -> dict:
-    """Packed [T, H, d] inputs in the workload dtype.
+    """Packed [T, H, d] inputs in the workload dtype, on `device`.
 
-    heads: iterable of (n, h) generated from their seeds (None = all).  The
-    remaining heads, if any, are filled from a fast generator with the same
-    distributions (their values do not match the per-head seeds).
+    heads: iterable of (n, h) generated from their own seeds (None = all).
+    The remaining heads, if any, are filled on `device` from a fast generator
+    with the same distributions (their values do not match the per-head
+    seeds, and no check reads them).
     Returns dict(q, k, v, g, beta, gate, cu_seqlens (int32), initial_state
-    (fp32 [N, H, dk, dv] or None), exact (list of (n, h)))."""
+    (fp32 [N, H, dk, dv] or None), exact (sorted list of (n, h)))."""
     assert not w.is_decode
     cu = w.cu_seqlens()
     T, H, dk, dv, N = cu[-1], w.H, w.dk, w.dv, w.num_seqs
     sel = _select(w, heads)
-    full = len(sel) == N * H
-    f32 = torch.float32
-    if full:
-        q = torch.empty(T, H, dk, dtype=f32)
-        k = torch.empty(T, H, dk, dtype=f32)
-        g = torch.empty(T, H, dk, dtype=f32)
-        v = torch.empty(T, H, dv, dtype=f32)
-        gate = torch.empty(T, H, dv, dtype=f32)
-        beta = torch.empty(T, H, dtype=f32)
-        init = torch.zeros(N, H, dk, dv, dtype=f32) if w.init_state else None
+    dt = w.torch_dtype
+    if len(sel) == N * H:
+        out = dict(q=torch.empty(T, H, dk, dtype=dt), k=torch.empty(T, H, dk, dtype=dt),
+                   g=torch.empty(T, H, dk, dtype=dt), v=torch.empty(T, H, dv, dtype=dt),
+                   gate=torch.empty(T, H, dv, dtype=dt), beta=torch.empty(T, H, dtype=dt),
+                   initial_state=torch.zeros(N, H, dk, dv) if w.init_state else None)
+        fill_dev = "cpu"
     else:
-        fill = fast_prefill(w, seed=w.seed + 77)
-        q, k, g, v, gate, beta = (fill[x].to(f32) for x in ("q", "k", "g", "v", "gate", "beta"))
-        init = fill["initial_state"]
+        out = fast_prefill(w, seed=w.seed + 77, device=device)
+        out.pop("cu_seqlens")
+        fill_dev = device
 
     def one(nh):
         n, h = nh
         d = head_inputs(w, n, h)
         t0, t1 = cu[n], cu[n + 1]
-        q[t0:t1, h] = d["q"]
-        k[t0:t1, h] = d["k"]
-        g[t0:t1, h] = d["g"]
-        v[t0:t1, h] = d["v"]
-        gate[t0:t1, h] = d["gate"]
-        beta[t0:t1, h] = d["beta"]
-        if init is not None:
-            init[n, h] = d["init"]
+        for key in ("q", "k", "g", "v", "gate", "beta"):
+            out[key][t0:t1, h] = d[key].to(device=fill_dev, dtype=dt)
+        if out["initial_state"] is not None:
+            out["initial_state"][n, h] = d["init"].to(fill_dev)
 
-    nthreads = threads or min(32, max(1, torch.get_num_threads()))
-    if len(sel) > 1 and nthreads > 1:
-        with ThreadPoolExecutor(nthreads) as ex:
-            list(ex.map(one, sel))
-    else:
-        for nh in sel:
-            one(nh)
-    dt = w.torch_dtype
-    out = dict(q=q.to(dt), k=k.to(dt), v=v.to(dt), g=g.to(dt), beta=beta.to(dt),
-               gate=gate.to(dt), cu_seqlens=torch.tensor(cu, dtype=torch.int32),
-               initial_state=init, exact=sel)
-    if device != "cpu":
-        out = {key: (val.to(device) if torch.is_tensor(val) else val) for key, val in out.items()}
+    _run(one, sel, threads)
+    out = {key: (val.to(device) if torch.is_tensor(val) else val) for key, val in out.items()}
+    out["cu_seqlens"] = torch.tensor(cu, dtype=torch.int32, device=device)
+    out["exact"] = sel
     return out
+
+
+def _run(fn, items, threads):
+    nthreads = threads or min(32, max(1, torch.get_num_threads()))
+    if len(items) > 1 and nthreads > 1:
+        with ThreadPoolExecutor(nthreads) as ex:
+            list(ex.map(fn, items))
+    else:
+        for it in items:
+            fn(it)
 
 
 def fast_prefill(w: Workload, seed: int, device="cpu") -> dict:
@@ -246,46 +241,38 @@ def fast_prefill(w: Workload, seed: int, device="cpu") -> dict:
     return out
 
 
-def pack_decode(w: Workload, steps: int | None = None, heads=None, threads: int = 0) -> dict:
-    """Decode inputs: q, k, g [steps, N, H, dk]; v, gate [steps, N, H, dv];
-    beta [steps, N, H] (workload dtype) and the fp32 state [N, H, dk, dv].
-    heads: (n, h) drawn from their seeds (None = all); the rest come from a
-    fast generator."""
+def pack_decode(w: Workload, steps: int | None = None, heads=None, device="cpu",
+                threads: int = 0) -> dict:
+    """Decode inputs on `device`: q, k, g [steps, N, H, dk]; v, gate
+    [steps, N, H, dv]; beta [steps, N, H] (workload dtype) and the fp32 state
+    [N, H, dk, dv].  heads: (n, h) drawn from their own seeds (None = all);
+    the rest are filled on `device` from a fast generator."""
     assert w.is_decode
     S = steps if steps is not None else w.decode_steps
     N, H, dk, dv = w.num_seqs, w.H, w.dk, w.dv
     sel = _select(w, heads)
-    f32 = torch.float32
+    dt = w.torch_dtype
     if len(sel) == N * H:
-        q = torch.empty(S, N, H, dk, dtype=f32)
-        k = torch.empty_like(q)
-        g = torch.empty_like(q)
-        v = torch.empty(S, N, H, dv, dtype=f32)
-        gate = torch.empty_like(v)
-        beta = torch.empty(S, N, H, dtype=f32)
-        state = torch.empty(N, H, dk, dv, dtype=f32)
+        out = dict(q=torch.empty(S, N, H, dk, dtype=dt), k=torch.empty(S, N, H, dk, dtype=dt),
+                   g=torch.empty(S, N, H, dk, dtype=dt), v=torch.empty(S, N, H, dv, dtype=dt),
+                   gate=torch.empty(S, N, H, dv, dtype=dt), beta=torch.empty(S, N, H, dtype=dt),
+                   state=torch.empty(N, H, dk, dv))
+        fill_dev = "cpu"
     else:
-        fill = fast_decode(w, S, seed=w.seed + 77)
-        q, k, g, v, gate, beta = (fill[x].to(f32) for x in ("q", "k", "g", "v", "gate", "beta"))
-        state = fill["state"]
+        out = fast_decode(w, S, seed=w.seed + 77, device=device)
+        fill_dev = device
 
     def one(nh):
         n, h = nh
         d = head_inputs(w, n, h, length=S)
-        q[:, n, h] = d["q"]
-        k[:, n, h] = d["k"]
-        g[:, n, h] = d["g"]
-        v[:, n, h] = d["v"]
-        gate[:, n, h] = d["gate"]
-        beta[:, n, h] = d["beta"]
-        state[n, h] = d["init"]
+        for key in ("q", "k", "g", "v", "gate", "beta"):
+            out[key][:, n, h] = d[key].to(device=fill_dev, dtype=dt)
+        out["state"][n, h] = d["init"].to(fill_dev)
 
-    nthreads = threads or min(32, max(1, torch.get_num_threads()))
-    with ThreadPoolExecutor(nthreads) as ex:
-        list(ex.map(one, sel))
-    dt = w.torch_dtype
-    return dict(q=q.to(dt), k=k.to(dt), v=v.to(dt), g=g.to(dt), beta=beta.to(dt),
-                gate=gate.to(dt), state=state, exact=sel)
+    _run(one, sel, threads)
+    out = {key: val.to(device) for key, val in out.items()}
+    out["exact"] = sel
+    return out
 
 
 def fast_decode(w: Workload, steps: int, seed: int, device="cpu") -> dict:

@@ -1,0 +1,144 @@
+"""The C-ABI library builds, loads, exports what include/kda.h declares, and
+rejects bad arguments on the host (no GPU needed: nothing here launches)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from kda_linear_attention_fwd_b200 import build, kda
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kda.h")
+
+OK, INVALID, UNSUPPORTED, ALIGN, WORKSPACE, CUDA, TIMEOUT = 0, -1, -2, -3, -4, -5, -6
+BF16, F32 = 1, 0
+A = 0x100000  # a 16-byte aligned fake device address; never dereferenced on the host
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return kda.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kda_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("kda_chunk_fwd", "kda_decode_step", "kda_chunk_fwd_workspace_size",
+              "kda_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(kda.EXPORTS) <= set(declared_functions())
+
+
+def test_exports_are_c_symbols():
+    out = os.popen(f"nm -D --defined-only {kda.LIB_PATH}").read()
+    for name in declared_functions():
+        assert re.search(rf"\bT {name}$", out, flags=re.M), name
+
+
+def test_status_strings(lib):
+    for code, name in [(OK, "KDA_OK"), (INVALID, "KDA_ERR_INVALID_ARG"),
+                       (UNSUPPORTED, "KDA_ERR_UNSUPPORTED"), (ALIGN, "KDA_ERR_ALIGNMENT"),
+                       (WORKSPACE, "KDA_ERR_WORKSPACE"), (CUDA, "KDA_ERR_CUDA"),
+                       (TIMEOUT, "KDA_ERR_TIMEOUT")]:
+        assert kda.status_string(code) == name
+    assert kda.status_string(12345) == "KDA_ERR_UNKNOWN"
+
+
+def test_workspace_size(lib):
+    f = lib.kda_chunk_fwd_workspace_size
+    assert f(4096, 2, 16, 128, 128, BF16) > 0
+    assert f(0, 1, 1, 64, 64, F32) > 0
+    assert f(-1, 1, 1, 64, 64, F32) == 0
+    assert f(16, 1, 1, 96, 64, F32) == 0
+    assert f(16, 1, 0, 64, 64, F32) == 0
+    assert f(16, 1, 1, 64, 64, 7) == 0
+    # grows with the number of heads and with the state size
+    assert f(8192, 2, 32, 128, 128, BF16) > f(8192, 2, 16, 128, 128, BF16)
+    assert f(8192, 2, 16, 128, 128, BF16) > f(8192, 2, 16, 64, 64, BF16)
+
+
+def call_fwd(lib, **kw):
+    a = dict(q=A, k=A, v=A, g=A, beta=A, gate=None, out=A, cu=A, cu_host=None, N=1, T=16, H=1,
+             dk=64, dv=64, dtype=BF16, scale=1.0, l2=0, s0=None, s1=None, ws=A, ws_bytes=1 << 40,
+             stream=None)
+    a.update(kw)
+    cu_host = a["cu_host"]
+    if cu_host is not None:
+        arr = (ctypes.c_int32 * len(cu_host))(*cu_host)
+        cu_host = ctypes.cast(arr, ctypes.c_void_p)
+    return lib.kda_chunk_fwd(a["q"], a["k"], a["v"], a["g"], a["beta"], a["gate"], a["out"],
+                             a["cu"], cu_host, a["N"], a["T"], a["H"], a["dk"], a["dv"],
+                             a["dtype"], a["scale"], a["l2"], a["s0"], a["s1"], a["ws"],
+                             a["ws_bytes"], a["stream"])
+
+
+def test_chunk_fwd_validation(lib):
+    assert call_fwd(lib, N=0, T=0) == OK
+    assert call_fwd(lib, N=0, T=5) == INVALID
+    assert call_fwd(lib, N=-1) == INVALID
+    assert call_fwd(lib, H=0) == INVALID
+    assert call_fwd(lib, T=-3) == INVALID
+    assert call_fwd(lib, dk=96) == UNSUPPORTED
+    assert call_fwd(lib, dv=32) == UNSUPPORTED
+    assert call_fwd(lib, dtype=5) == UNSUPPORTED
+    assert call_fwd(lib, l2=2) == INVALID
+    assert call_fwd(lib, q=None) == INVALID
+    assert call_fwd(lib, cu=None) == INVALID
+    assert call_fwd(lib, out=None) == INVALID
+    assert call_fwd(lib, q=A + 8) == ALIGN
+    assert call_fwd(lib, gate=A + 4) == ALIGN
+    assert call_fwd(lib, s1=A + 2) == ALIGN
+    assert call_fwd(lib, beta=A + 1) == ALIGN
+    assert call_fwd(lib, ws=A + 8) == ALIGN
+    assert call_fwd(lib, ws=None) == WORKSPACE
+    assert call_fwd(lib, ws_bytes=16) == WORKSPACE
+    # host copy of cu_seqlens is checked when given
+    assert call_fwd(lib, cu_host=[0, 15]) == INVALID
+    assert call_fwd(lib, N=2, cu_host=[0, 10, 5]) == INVALID
+    assert call_fwd(lib, cu_host=[1, 16]) == INVALID
+    # final state may alias the initial state exactly, but not overlap partially
+    assert call_fwd(lib, s0=A, s1=A + 256, ws_bytes=16) == INVALID
+    assert call_fwd(lib, s0=A, s1=A, ws_bytes=16) == WORKSPACE  # aliasing accepted
+
+
+def call_dec(lib, **kw):
+    a = dict(q=A, k=A, v=A, g=A, beta=A, gate=None, out=A, state=A, N=4, H=2, dk=128, dv=128,
+             dtype=BF16, scale=1.0, l2=0, stream=None)
+    a.update(kw)
+    return lib.kda_decode_step(a["q"], a["k"], a["v"], a["g"], a["beta"], a["gate"], a["out"],
+                               a["state"], a["N"], a["H"], a["dk"], a["dv"], a["dtype"],
+                               a["scale"], a["l2"], a["stream"])
+
+
+def test_decode_validation(lib):
+    assert call_dec(lib, N=0) == OK
+    assert call_dec(lib, N=-1) == INVALID
+    assert call_dec(lib, H=0) == INVALID
+    assert call_dec(lib, dk=32) == UNSUPPORTED
+    assert call_dec(lib, dtype=3) == UNSUPPORTED
+    assert call_dec(lib, state=None) == INVALID
+    assert call_dec(lib, beta=None) == INVALID
+    assert call_dec(lib, state=A + 4) == ALIGN
+    assert call_dec(lib, k=A + 2) == ALIGN
+    assert call_dec(lib, beta=A + 1) == ALIGN
+    assert call_dec(lib, l2=-1) == INVALID
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(16, 1, 64, dtype=torch.bfloat16)
+    with pytest.raises((ValueError, RuntimeError)):
+        kda.chunk_fwd(x, x, x, x, torch.zeros(16, 1, dtype=torch.bfloat16), None,
+                      torch.tensor([0, 16], dtype=torch.int32))
