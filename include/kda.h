@@ -125,6 +125,36 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const void *g, co
                   void *workspace, size_t workspace_bytes, kda_stream_t stream);
 
 /*
+ * kda_chunk_fwd without a workspace argument, for callers that cannot
+ * allocate device memory when they run the layer (code running inside an
+ * allocator or memory-pool callback, runtimes that hand out only fixed
+ * buffers, hosts that forbid allocation after start-up).  The pages have no
+ * counterpart to this; it is a deployment convenience.
+ *
+ * Same arguments, semantics and results as kda_chunk_fwd, minus workspace.
+ * The scratch the prefill needs (piece plan, per-piece transitions and
+ * states) lives in a fixed 32 MiB array of device memory owned by the
+ * library: it exists on every GPU that loads this code and is held until the
+ * process exits.  The piece length is the usual one, lengthened until the
+ * scratch fits; sizes whose plan does not fit even with one piece per
+ * sequence are rejected with KDA_ERR_WORKSPACE.  Allocates nothing (no
+ * cudaMalloc/cudaFree, directly or through a library).
+ *
+ * The first call on each device, made while that device is current, looks up
+ * the array's device address (cudaGetSymbolAddress); make that first call
+ * before any stream capture.  All calls on a device share the array and its
+ * contents persist between calls: calls that overlap on the GPU (other
+ * streams, other host threads) race on it and must be serialised by the
+ * caller.  No entry needs to start at zero; each call writes what it reads.
+ */
+int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const void *g,
+                          const void *beta, const void *gate, void *out,
+                          const int32_t *cu_seqlens, const int32_t *cu_seqlens_host,
+                          int32_t num_seqs, int32_t total_tokens, int32_t H, int32_t dk,
+                          int32_t dv, kda_dtype dtype, float scale, int32_t qk_l2norm,
+                          const float *initial_state, float *final_state, kda_stream_t stream);
+
+/*
  * Decode: one token per sequence, the recurrence above applied once, state
  * updated in place.  Decode cost is this per-token state update
  * (prism.simon-ai.net page, section "推理瓶颈与Kimi K3的针对性优化").
