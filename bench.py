@@ -379,8 +379,8 @@ def main():
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": w.dtype, "data": "synthetic",
-                "config": {"workload": f"{w.name}: {N} x {T} tokens, H={w.H}, dk={w.dk}, "
-                                       f"dv={w.dv}, {w.dtype}, chunk=16",
+                "config": {"workload": f"{w.name}: {N} sequence(s), {T} tokens, H={w.H}, "
+                                       f"dk={w.dk}, dv={w.dv}, {w.dtype}, chunk=16",
                            "global_batch": ws * N, "seq_len": T,
                            "parallelism": f"replicas x{ws} (sequences/heads independent)",
                            "l2": "inputs larger than L2 (%.1f GB per step)" % (pbytes / 1e9),

@@ -15,8 +15,8 @@ cudaError_t launch_decode(bool bf16, int dk, int dv, const void *q, const void *
 cudaError_t launch_plan(const int32_t *cu, int num_seqs, int total_tokens, int piece_len, int P_max,
                         int32_t *header, int32_t *seq_first, int4 *pieces, cudaStream_t st);
 cudaError_t launch_scan(const PrefillParams &p, int dk, int dv, cudaStream_t st);
-cudaError_t launch_prefill_simt(const PrefillParams &p, bool bf16, int dk, int dv, bool summaries,
-                                cudaStream_t st);
+cudaError_t launch_prefill_chunks(const PrefillParams &p, bool bf16, int dk, int dv,
+                                  bool summaries, cudaStream_t st);
 }  // namespace kda
 
 namespace {
@@ -167,12 +167,12 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const void *g, co
     if (e != cudaSuccess) return KDA_ERR_CUDA;
     const bool multi = total_tokens > L;  // some sequence may have >1 piece
     if (multi) {
-        e = kda::launch_prefill_simt(p, bf16, dk, dv, true, stream);
+        e = kda::launch_prefill_chunks(p, bf16, dk, dv, true, stream);
         if (e != cudaSuccess) return KDA_ERR_CUDA;
         e = kda::launch_scan(p, dk, dv, stream);
         if (e != cudaSuccess) return KDA_ERR_CUDA;
     }
-    e = kda::launch_prefill_simt(p, bf16, dk, dv, false, stream);
+    e = kda::launch_prefill_chunks(p, bf16, dk, dv, false, stream);
     if (e != cudaSuccess) return KDA_ERR_CUDA;
     return KDA_OK;
 }

@@ -30,8 +30,8 @@ namespace kda {
 cudaError_t launch_plan(const int32_t *cu, int num_seqs, int total_tokens, int piece_len, int P_max,
                         int32_t *header, int32_t *seq_first, int4 *pieces, cudaStream_t st);
 cudaError_t launch_scan(const PrefillParams &p, int dk, int dv, cudaStream_t st);
-cudaError_t launch_prefill_simt(const PrefillParams &p, bool bf16, int dk, int dv, bool summaries,
-                                cudaStream_t st);
+cudaError_t launch_prefill_chunks(const PrefillParams &p, bool bf16, int dk, int dv,
+                                  bool summaries, cudaStream_t st);
 }  // namespace kda
 
 namespace {
@@ -178,11 +178,11 @@ extern "C" int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v
                                      (int4 *)(ws + WL.off_pieces), stream);
     if (e != cudaSuccess) return KDA_ERR_CUDA;
     if (summaries) {
-        e = kda::launch_prefill_simt(p, bf16, dk, dv, true, stream);
+        e = kda::launch_prefill_chunks(p, bf16, dk, dv, true, stream);
         if (e != cudaSuccess) return KDA_ERR_CUDA;
         e = kda::launch_scan(p, dk, dv, stream);
         if (e != cudaSuccess) return KDA_ERR_CUDA;
     }
-    e = kda::launch_prefill_simt(p, bf16, dk, dv, false, stream);
+    e = kda::launch_prefill_chunks(p, bf16, dk, dv, false, stream);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }

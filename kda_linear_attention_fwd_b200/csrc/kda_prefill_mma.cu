@@ -1,0 +1,574 @@
+// KDA prefill, bf16 tensor-core chunk pass (warp-level MMA, state resident
+// in registers).
+//
+// One CTA runs the 16-token chunk recurrence over one piece of one head.
+// The state S (dk x NC, fp32) never leaves the registers of the four state
+// warps: warp w holds S^T rows [w*NC/4, (w+1)*NC/4) -- i.e. NC/4 state
+// columns -- as m16n8k16 accumulator fragments, and the C-fragment layout of
+// those accumulators is exactly the A-fragment layout of the next chunk's
+// products, so each chunk only converts them to bf16 in registers.
+//
+// Per chunk (rows are the chunk's tokens, see kda_prefill_simt.cu for the
+// algebra):
+//   state warps:  U^T  = V^T Tb^T + S^T (-W)^T        (dv x 16, K = 16 and dk)
+//                 O^T  = S^T Qd^T + U^T P^T           (dv x 16)
+//                 S^T <- S^T Diag(exp G_C) + U^T Kb    (dv x dk, K = 16)
+//                 y    = gate (.) O
+//   prep warps:   cumulative decay, Qd / Kd / Ki / Kb (bf16), A = Kd Ki^T and
+//                 P = Qd Ki^T (tensor cores), Tb = (I + Diag(beta) A)^-1
+//                 Diag(beta) (fp32 forward substitution), W = Tb Kd (tensor
+//                 cores); all of it one chunk ahead of the state warps.
+// Raw input tiles are prefetched with cp.async one chunk further ahead.
+// The prep and state warps hand chunks over through two shared-memory stages
+// guarded by named barriers (FULL: prep -> state, EMPTY: state -> prep).
+//
+// The decay is applied as an absolute-position transform inside the chunk
+// (Qd, Kd carry exp(G), Ki carries exp(-G)): prism.simon-ai.net,
+// "从架构创新出发：K3的MoE与混合注意力设计", section "数值稳定性与 Co-Design：
+// BF16 约束下的衰减控制策略".  With at most 16 tokens and log-decay >= ln 0.0067
+// per token (affta.cn K3 explainer, section "第一关：KDA 解决算得动"), |G| <= 80
+// and exp(+-G) fit bf16/fp32.  exp(G_r) and exp(G_C - G_r) are built as prefix
+// and suffix products of exp(g), one exponential per element.
+#include <cstdlib>
+
+#include "kda_common.cuh"
+#include "kda_prefill.cuh"
+
+namespace kda {
+namespace tc {
+
+using bf16 = __nv_bfloat16;
+
+constexpr int kThreads = 256;     // 4 state warps + 4 prep warps
+constexpr int kPad = 8;           // bf16 row padding: conflict-free ldmatrix
+constexpr int kL16 = 16 + kPad;   // row length of the 16 x 16 bf16 tiles
+
+// named barriers (0 is __syncthreads)
+constexpr int BAR_PREP = 1;       // prep warps only (128 threads)
+constexpr int BAR_FULL = 2;       // + stage: prep arrives, state waits (256)
+constexpr int BAR_EMPTY = 4;      // + stage: state arrives, prep waits (256)
+
+KDA_DEVICE uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+KDA_DEVICE void bar_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+KDA_DEVICE void bar_arrive(int id, int n) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+KDA_DEVICE uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+KDA_DEVICE void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+KDA_DEVICE void ldsm4(uint32_t (&r)[4], const void *p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(smem_u32(p)));
+}
+KDA_DEVICE void ldsm4t(uint32_t (&r)[4], const void *p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(smem_u32(p)));
+}
+KDA_DEVICE void cp_async16(void *dst, const void *src, bool valid) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(dst)), "l"(src),
+                 "r"(valid ? 16 : 0)
+                 : "memory");
+}
+KDA_DEVICE void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N> KDA_DEVICE void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+// Lane addressing of ldmatrix.x4 for the three fragment kinds used here.
+//  A operand, row-major [m][k] storage:       row (l&7)+((l>>3)&1)*8, col (l>>4)*8
+//  B operand from [n][k] storage (k inner):   n (l&7)+(l>>4)*8,       k ((l>>3)&1)*8
+//  B operand from [k][n] storage, .trans:     k (l&7)+((l>>3)&1)*8,   n (l>>4)*8
+//  A operand from [k][m] storage, .trans:     k (l&7)+(l>>4)*8,       m ((l>>3)&1)*8
+// Results: A -> a0..a3; B -> {r0,r1} = n-tile 0 (k lo, k hi), {r2,r3} = n-tile 1.
+
+template <int DK, int NC>
+struct Layout {
+    static constexpr int LK = DK + kPad;  // row length of [16][DK] bf16 tiles
+    static constexpr int LC = NC + kPad;  // row length of [16][NC] bf16 tiles
+    static constexpr int MT = NC / 64;    // m16 tiles per state warp
+    static constexpr int CW = NC / 4;     // state columns per state warp
+    static constexpr int LY = CW + 4;     // output staging row (fp32)
+    struct Raw {                          // cp.async targets, unpadded rows
+        bf16 q[16 * DK], k[16 * DK], g[16 * DK], v[16 * NC], gate[16 * NC];
+    };
+    struct Stage {                        // handed from prep to state warps
+        bf16 qd[16 * LK], kb[16 * LK], wn[16 * LK];
+        bf16 v[16 * LC], gate[16 * LC];
+        bf16 p[16 * kL16], tb[16 * kL16];
+        float gam[DK];
+    };
+    struct Prep {                         // private to the prep warps
+        bf16 kd[16 * LK], ki[16 * LK];
+        float A[16 * 17];
+        float beta[2][16];
+        float red[2][4][16];
+        float rq[16], rk[16];
+    };
+    struct All {
+        Raw raw[2];
+        Stage st[2];
+        Prep pr;
+        float ys[4][16 * LY];
+    };
+    static constexpr size_t bytes = sizeof(All);
+};
+
+// Runs tokens [t0, t0 + len) of head h.  OUT: produce y.  USE_V: the write
+// uses v (false: the transition part, U0 = 0).  The state starts as the
+// identity, a copy of s_init ([DK][NC] fp32) or zeros and is written to s_out.
+template <int DK, int NC, bool OUT, bool USE_V>
+__device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const float *s_init,
+                          bool identity, float *s_out, unsigned char *smem_raw) {
+    using Lay = Layout<DK, NC>;
+    constexpr int LK = Lay::LK, LC = Lay::LC, MT = Lay::MT, CW = Lay::CW, LY = Lay::LY;
+    typename Lay::All &sm = *reinterpret_cast<typename Lay::All *>(smem_raw);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int H = p.H;
+    const int nchunks = (len + 15) / 16;
+
+    if (warp < 4) {
+        // ------------------------------------------------------------ state
+        const int g8 = lane >> 2, q4 = lane & 3;
+        const int jb = warp * CW;  // first state column of this warp
+        float s[MT][DK / 8][4];
+#pragma unroll
+        for (int m = 0; m < MT; ++m)
+#pragma unroll
+            for (int nt = 0; nt < DK / 8; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = jb + 16 * m + g8 + (e >= 2 ? 8 : 0);
+                    const int i = 8 * nt + 2 * q4 + (e & 1);
+                    s[m][nt][e] = identity ? (i == j ? 1.f : 0.f)
+                                           : (s_init ? s_init[(size_t)i * NC + j] : 0.f);
+                }
+        bf16 *out = (bf16 *)p.out;
+        for (int c = 0; c < nchunks; ++c) {
+            const int stg = c & 1;
+            bar_sync(BAR_FULL + stg, kThreads);
+            typename Lay::Stage &S = sm.st[stg];
+            float u[MT][2][4], o[MT][2][4];
+#pragma unroll
+            for (int m = 0; m < MT; ++m)
+#pragma unroll
+                for (int n = 0; n < 2; ++n)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) u[m][n][e] = o[m][n][e] = 0.f;
+            if (USE_V) {  // U0^T = V^T Tb^T
+                uint32_t bt[4];
+                ldsm4(bt, &S.tb[((lane & 7) + (lane >> 4) * 8) * kL16 + ((lane >> 3) & 1) * 8]);
+#pragma unroll
+                for (int m = 0; m < MT; ++m) {
+                    uint32_t a[4];
+                    ldsm4t(a, &S.v[((lane & 7) + (lane >> 4) * 8) * LC + jb + 16 * m +
+                                   ((lane >> 3) & 1) * 8]);
+                    mma16816(u[m][0], a, bt[0], bt[1]);
+                    mma16816(u[m][1], a, bt[2], bt[3]);
+                }
+            }
+            // U^T += S^T (-W)^T ;  O^T = S^T Qd^T
+#pragma unroll
+            for (int kk = 0; kk < DK / 16; ++kk) {
+                uint32_t bw[4], bq[4];
+                const int n_off = ((lane & 7) + (lane >> 4) * 8) * LK + 16 * kk + ((lane >> 3) & 1) * 8;
+                ldsm4(bw, &S.wn[n_off]);
+                if (OUT) ldsm4(bq, &S.qd[n_off]);
+#pragma unroll
+                for (int m = 0; m < MT; ++m) {
+                    uint32_t a[4];
+                    a[0] = pack_bf16(s[m][2 * kk][0], s[m][2 * kk][1]);
+                    a[1] = pack_bf16(s[m][2 * kk][2], s[m][2 * kk][3]);
+                    a[2] = pack_bf16(s[m][2 * kk + 1][0], s[m][2 * kk + 1][1]);
+                    a[3] = pack_bf16(s[m][2 * kk + 1][2], s[m][2 * kk + 1][3]);
+                    mma16816(u[m][0], a, bw[0], bw[1]);
+                    mma16816(u[m][1], a, bw[2], bw[3]);
+                    if (OUT) {
+                        mma16816(o[m][0], a, bq[0], bq[1]);
+                        mma16816(o[m][1], a, bq[2], bq[3]);
+                    }
+                }
+            }
+            uint32_t ua[MT][4];
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                ua[m][0] = pack_bf16(u[m][0][0], u[m][0][1]);
+                ua[m][1] = pack_bf16(u[m][0][2], u[m][0][3]);
+                ua[m][2] = pack_bf16(u[m][1][0], u[m][1][1]);
+                ua[m][3] = pack_bf16(u[m][1][2], u[m][1][3]);
+            }
+            if (OUT) {  // O^T += U^T P^T
+                uint32_t bp[4];
+                ldsm4(bp, &S.p[((lane & 7) + (lane >> 4) * 8) * kL16 + ((lane >> 3) & 1) * 8]);
+#pragma unroll
+                for (int m = 0; m < MT; ++m) {
+                    mma16816(o[m][0], ua[m], bp[0], bp[1]);
+                    mma16816(o[m][1], ua[m], bp[2], bp[3]);
+                }
+            }
+            // S^T <- S^T Diag(gamma) + U^T Kb
+#pragma unroll
+            for (int np = 0; np < DK / 16; ++np) {
+                uint32_t bk[4];
+                ldsm4t(bk, &S.kb[((lane & 7) + ((lane >> 3) & 1) * 8) * LK + 16 * np +
+                                 (lane >> 4) * 8]);
+                const float2 ga = *reinterpret_cast<const float2 *>(&S.gam[16 * np + 2 * q4]);
+                const float2 gb = *reinterpret_cast<const float2 *>(&S.gam[16 * np + 8 + 2 * q4]);
+#pragma unroll
+                for (int m = 0; m < MT; ++m) {
+                    float *x = s[m][2 * np];
+                    float *y = s[m][2 * np + 1];
+                    x[0] *= ga.x; x[1] *= ga.y; x[2] *= ga.x; x[3] *= ga.y;
+                    y[0] *= gb.x; y[1] *= gb.y; y[2] *= gb.x; y[3] *= gb.y;
+                    mma16816(s[m][2 * np], ua[m], bk[0], bk[1]);
+                    mma16816(s[m][2 * np + 1], ua[m], bk[2], bk[3]);
+                }
+            }
+            if (OUT) {
+                float *ys = sm.ys[warp];
+#pragma unroll
+                for (int m = 0; m < MT; ++m)
+#pragma unroll
+                    for (int n = 0; n < 2; ++n) {
+                        const int t = 8 * n + 2 * q4;
+                        const int jl = 16 * m + g8;
+                        ys[t * LY + jl] = o[m][n][0];
+                        ys[(t + 1) * LY + jl] = o[m][n][1];
+                        ys[t * LY + jl + 8] = o[m][n][2];
+                        ys[(t + 1) * LY + jl + 8] = o[m][n][3];
+                    }
+                __syncwarp();
+                const int rows = min(16, len - 16 * c);
+                // lane -> token row (lane >> 1), half of the warp's columns
+                const int r = lane >> 1;
+                constexpr int HALF = CW / 2;
+                if (r < rows) {
+                    const int jl0 = (lane & 1) * HALF;
+                    bf16 *dst = out + ((size_t)(t0 + 16 * c + r) * H + h) * NC + jb + jl0;
+#pragma unroll
+                    for (int v8 = 0; v8 < HALF / 8; ++v8) {
+                        uint32_t pk[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int jl = jl0 + 8 * v8 + 2 * e;
+                            const float g0 = __bfloat162float(S.gate[r * LC + jb + jl]);
+                            const float g1 = __bfloat162float(S.gate[r * LC + jb + jl + 1]);
+                            pk[e] = pack_bf16(g0 * ys[r * LY + jl], g1 * ys[r * LY + jl + 1]);
+                        }
+                        *reinterpret_cast<uint4 *>(dst + 8 * v8) =
+                            make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    }
+                }
+                __syncwarp();
+            }
+            bar_arrive(BAR_EMPTY + stg, kThreads);
+        }
+        if (s_out) {
+#pragma unroll
+            for (int m = 0; m < MT; ++m)
+#pragma unroll
+                for (int nt = 0; nt < DK / 8; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int j = jb + 16 * m + g8 + (e >= 2 ? 8 : 0);
+                        const int i = 8 * nt + 2 * q4 + (e & 1);
+                        s_out[(size_t)i * NC + j] = s[m][nt][e];
+                    }
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------------- prep
+    const int pt = tid - 128, pw = pt >> 5;
+    const bf16 *q = (const bf16 *)p.q, *k = (const bf16 *)p.k, *g = (const bf16 *)p.g;
+    const bf16 *v = (const bf16 *)p.v, *gate = (const bf16 *)p.gate, *beta = (const bf16 *)p.beta;
+    typename Lay::Prep &pr = sm.pr;
+    float beta_next = 0.f;
+
+    // raw tiles of chunk c -> raw[c & 1]; rows past the piece are zero-filled
+    auto issue = [&](int c) {
+        typename Lay::Raw &R = sm.raw[c & 1];
+        const int tc = t0 + 16 * c;
+        const int rows = min(16, len - 16 * c);
+        constexpr int PK = DK / 8;  // 16-byte pieces per row
+        for (int x = pt; x < 16 * PK; x += 128) {
+            const int r = x / PK, cc = x % PK;
+            const bool ok = r < rows;
+            const size_t off = ((size_t)(ok ? tc + r : t0) * H + h) * DK + cc * 8;
+            cp_async16(&R.k[r * DK + cc * 8], k + off, ok);
+            cp_async16(&R.g[r * DK + cc * 8], g + off, ok);
+            if (OUT) cp_async16(&R.q[r * DK + cc * 8], q + off, ok);
+        }
+        if (USE_V || OUT) {
+            constexpr int PV = NC / 8;
+            for (int x = pt; x < 16 * PV; x += 128) {
+                const int r = x / PV, cc = x % PV;
+                const bool ok = r < rows;
+                const size_t off = ((size_t)(ok ? tc + r : t0) * H + h) * NC + cc * 8;
+                if (USE_V) cp_async16(&R.v[r * NC + cc * 8], v + off, ok);
+                if (OUT) {
+                    if (gate) cp_async16(&R.gate[r * NC + cc * 8], gate + off, ok);
+                }
+            }
+        }
+        cp_async_commit();
+        if (pt < 16) beta_next = pt < rows ? __bfloat162float(beta[(size_t)(tc + pt) * H + h]) : 0.f;
+    };
+
+    if (nchunks > 0) issue(0);
+    for (int c = 0; c < nchunks; ++c) {
+        const int stg = c & 1;
+        typename Lay::Raw &R = sm.raw[stg];
+        if (pt < 16) pr.beta[stg][pt] = beta_next;
+        if (c + 1 < nchunks) {
+            issue(c + 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        if (c >= 2) bar_sync(BAR_EMPTY + stg, kThreads);
+        bar_sync(BAR_PREP, 128);
+        typename Lay::Stage &S = sm.st[stg];
+        const float *bet = pr.beta[stg];
+
+        if (p.qk_l2norm) {  // 1/|q_r|, 1/|k_r| over the head dimension
+            for (int r = 0; r < 16; ++r) {
+                float kk = 0.f, qq = 0.f;
+                for (int i = pt; i < DK; i += 128) {
+                    const float kv = __bfloat162float(R.k[r * DK + i]);
+                    kk += kv * kv;
+                    if (OUT) {
+                        const float qv = __bfloat162float(R.q[r * DK + i]);
+                        qq += qv * qv;
+                    }
+                }
+                kk = warp_sum(kk);
+                qq = warp_sum(qq);
+                if (lane == 0) {
+                    pr.red[0][pw][r] = kk;
+                    pr.red[1][pw][r] = qq;
+                }
+            }
+            bar_sync(BAR_PREP, 128);
+            if (pt < 16) {
+                const float kk = pr.red[0][0][pt] + pr.red[0][1][pt] + pr.red[0][2][pt] + pr.red[0][3][pt];
+                const float qq = pr.red[1][0][pt] + pr.red[1][1][pt] + pr.red[1][2][pt] + pr.red[1][3][pt];
+                pr.rk[pt] = rsqrtf(kk + 1e-6f);
+                pr.rq[pt] = rsqrtf(qq + 1e-6f);
+            }
+            bar_sync(BAR_PREP, 128);
+        }
+
+        // 1. per key channel: decay factors and the decayed bf16 operands
+        if (pt < DK) {
+            const int i = pt;
+            float e[16], E[16], F[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) e[r] = __expf(__bfloat162float(R.g[r * DK + i]));
+            float acc = 1.f;
+#pragma unroll
+            for (int r = 0; r < 16; ++r) { acc *= e[r]; E[r] = acc; }
+            acc = 1.f;
+#pragma unroll
+            for (int r = 15; r >= 0; --r) { F[r] = acc; acc *= e[r]; }
+            const float El = E[15];
+            const float invEl = 1.f / El;
+            S.gam[i] = El;
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                float kv = __bfloat162float(R.k[r * DK + i]);
+                if (p.qk_l2norm) kv *= pr.rk[r];
+                pr.kd[r * LK + i] = __float2bfloat16_rn(kv * E[r]);
+                pr.ki[r * LK + i] = __float2bfloat16_rn(kv * (F[r] * invEl));
+                S.kb[r * LK + i] = __float2bfloat16_rn(kv * F[r]);
+                if (OUT) {
+                    float qv = __bfloat162float(R.q[r * DK + i]) * p.scale;
+                    if (p.qk_l2norm) qv *= pr.rq[r];
+                    S.qd[r * LK + i] = __float2bfloat16_rn(qv * E[r]);
+                }
+            }
+        }
+        // copy v and gate into the stage (the raw buffer is refilled early)
+        if (USE_V || OUT) {
+            constexpr int PV = NC / 8;
+            for (int x = pt; x < 16 * PV; x += 128) {
+                const int r = x / PV, cc = x % PV;
+                if (USE_V)
+                    *reinterpret_cast<uint4 *>(&S.v[r * LC + cc * 8]) =
+                        *reinterpret_cast<const uint4 *>(&R.v[r * NC + cc * 8]);
+                if (OUT) {
+                    uint4 gv;
+                    if (gate) {
+                        gv = *reinterpret_cast<const uint4 *>(&R.gate[r * NC + cc * 8]);
+                    } else {
+                        const uint32_t one = pack_bf16(1.f, 1.f);
+                        gv = make_uint4(one, one, one, one);
+                    }
+                    *reinterpret_cast<uint4 *>(&S.gate[r * LC + cc * 8]) = gv;
+                }
+            }
+        }
+        bar_sync(BAR_PREP, 128);
+
+        // 2. A = Kd Ki^T (strictly lower, fp32) and P = Qd Ki^T (lower, bf16)
+        if (pw == 0 || (OUT && pw == 1)) {
+            const bf16 *Aop = pw == 0 ? pr.kd : S.qd;
+            float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int kk = 0; kk < DK / 16; ++kk) {
+                uint32_t a[4], b[4];
+                ldsm4(a, &Aop[((lane & 7) + ((lane >> 3) & 1) * 8) * LK + 16 * kk + (lane >> 4) * 8]);
+                ldsm4(b, &pr.ki[((lane & 7) + (lane >> 4) * 8) * LK + 16 * kk + ((lane >> 3) & 1) * 8]);
+                mma16816(acc0, a, b[0], b[1]);
+                mma16816(acc1, a, b[2], b[3]);
+            }
+            const int r0 = lane >> 2, c0 = 2 * (lane & 3);
+            const float vals[8] = {acc0[0], acc0[1], acc0[2], acc0[3],
+                                   acc1[0], acc1[1], acc1[2], acc1[3]};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int r = r0 + ((e & 2) ? 8 : 0);
+                const int sc = c0 + (e & 1) + ((e & 4) ? 8 : 0);
+                if (pw == 0) {
+                    pr.A[r * 17 + sc] = sc < r ? vals[e] : 0.f;
+                } else {
+                    S.p[r * kL16 + sc] = __float2bfloat16_rn(sc <= r ? vals[e] : 0.f);
+                }
+            }
+        }
+        bar_sync(BAR_PREP, 128);
+
+        // 3. Tb = (I + Diag(beta) A)^-1 Diag(beta): forward substitution, lane = column
+        if (pw == 0 && lane < 16) {
+            const int j = lane;
+            float col[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                float acc = 0.f;
+#pragma unroll
+                for (int s2 = 0; s2 < r; ++s2) acc += pr.A[r * 17 + s2] * col[s2];
+                col[r] = (r == j ? 1.f : 0.f) - bet[r] * acc;
+            }
+            const float bj = bet[j];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) S.tb[r * kL16 + j] = __float2bfloat16_rn(col[r] * bj);
+        }
+        bar_sync(BAR_PREP, 128);
+
+        // 4. W = Tb Kd -> stage holds -W (bf16); prep warp pw owns DK/4 columns
+        {
+            uint32_t a[4];
+            ldsm4(a, &S.tb[((lane & 7) + ((lane >> 3) & 1) * 8) * kL16 + (lane >> 4) * 8]);
+#pragma unroll
+            for (int np = 0; np < DK / 64; ++np) {
+                const int n0 = pw * (DK / 4) + 16 * np;
+                uint32_t b[4];
+                ldsm4t(b, &pr.kd[((lane & 7) + ((lane >> 3) & 1) * 8) * LK + n0 + (lane >> 4) * 8]);
+                float w0[4] = {0.f, 0.f, 0.f, 0.f}, w1[4] = {0.f, 0.f, 0.f, 0.f};
+                mma16816(w0, a, b[0], b[1]);
+                mma16816(w1, a, b[2], b[3]);
+                const int r = lane >> 2, cc = n0 + 2 * (lane & 3);
+                *reinterpret_cast<uint32_t *>(&S.wn[r * LK + cc]) = pack_bf16(-w0[0], -w0[1]);
+                *reinterpret_cast<uint32_t *>(&S.wn[(r + 8) * LK + cc]) = pack_bf16(-w0[2], -w0[3]);
+                *reinterpret_cast<uint32_t *>(&S.wn[r * LK + cc + 8]) = pack_bf16(-w1[0], -w1[1]);
+                *reinterpret_cast<uint32_t *>(&S.wn[(r + 8) * LK + cc + 8]) = pack_bf16(-w1[2], -w1[3]);
+            }
+        }
+        bar_arrive(BAR_FULL + stg, kThreads);
+    }
+    // balance the state warps' last EMPTY arrivals
+    for (int c = nchunks - 2 < 0 ? 0 : nchunks - 2; c < nchunks; ++c) bar_sync(BAR_EMPTY + (c & 1), kThreads);
+}
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(kThreads, 1) summary_kernel(PrefillParams p) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int4 pc = p.pieces[blockIdx.x];
+    if (pc.x < 0) return;
+    const int n = pc.x, j = pc.w, h = blockIdx.y;
+    const int np = p.seq_first[n + 1] - p.seq_first[n];
+    if (j >= np - 1) return;
+    const size_t ph = (size_t)blockIdx.x * p.H + h;
+    if (blockIdx.z == 0) {
+        const float *init = (j == 0 && p.initial_state)
+                                ? p.initial_state + ((size_t)n * p.H + h) * DK * DV
+                                : nullptr;
+        run_piece<DK, DV, false, true>(p, pc.y, pc.z, h, init, false, p.Szero + ph * DK * DV, smem);
+    } else {
+        if (j == 0) return;
+        run_piece<DK, DK, false, false>(p, pc.y, pc.z, h, nullptr, true, p.M + ph * DK * DK, smem);
+    }
+}
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(kThreads, 1) output_kernel(PrefillParams p) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int4 pc = p.pieces[blockIdx.x];
+    if (pc.x < 0) return;
+    const int n = pc.x, j = pc.w, h = blockIdx.y;
+    const int np = p.seq_first[n + 1] - p.seq_first[n];
+    const size_t nh = (size_t)n * p.H + h;
+    const float *init = (np == 1) ? (p.initial_state ? p.initial_state + nh * DK * DV : nullptr)
+                                  : p.Sin + ((size_t)blockIdx.x * p.H + h) * DK * DV;
+    float *fin = (j == np - 1 && p.final_state) ? p.final_state + nh * DK * DV : nullptr;
+    run_piece<DK, DV, true, true>(p, pc.y, pc.z, h, init, false, fin, smem);
+}
+
+template <int DK, int DV>
+static cudaError_t launch_t(const PrefillParams &p, bool summaries, cudaStream_t st) {
+    cudaError_t e;
+    if (summaries) {
+        const size_t sm = Layout<DK, DV>::bytes > Layout<DK, DK>::bytes ? Layout<DK, DV>::bytes
+                                                                        : Layout<DK, DK>::bytes;
+        e = cudaFuncSetAttribute(summary_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)sm);
+        if (e != cudaSuccess) return e;
+        summary_kernel<DK, DV><<<dim3(p.P_max, p.H, 2), kThreads, sm, st>>>(p);
+        return cudaGetLastError();
+    }
+    const size_t sm = Layout<DK, DV>::bytes;
+    e = cudaFuncSetAttribute(output_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sm);
+    if (e != cudaSuccess) return e;
+    output_kernel<DK, DV><<<dim3(p.P_max, p.H, 1), kThreads, sm, st>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace tc
+
+cudaError_t launch_prefill_simt(const PrefillParams &p, bool bf16, int dk, int dv, bool summaries,
+                                cudaStream_t st);
+
+cudaError_t launch_prefill_tc(const PrefillParams &p, int dk, int dv, bool summaries,
+                              cudaStream_t st) {
+    if (dk == 128 && dv == 128) return tc::launch_t<128, 128>(p, summaries, st);
+    if (dk == 128 && dv == 64) return tc::launch_t<128, 64>(p, summaries, st);
+    if (dk == 64 && dv == 128) return tc::launch_t<64, 128>(p, summaries, st);
+    return tc::launch_t<64, 64>(p, summaries, st);
+}
+
+// The chunk pass for one call: bf16 inputs run on the tensor cores; fp32
+// inputs run the fp32 CUDA-core kernel (bf16 operands would not reach fp32
+// accuracy).  KDA_PREFILL_SIMT=1 forces the CUDA-core kernel for bf16 too.
+cudaError_t launch_prefill_chunks(const PrefillParams &p, bool bf16, int dk, int dv,
+                                  bool summaries, cudaStream_t st) {
+    static const bool force_simt = [] {
+        const char *e = std::getenv("KDA_PREFILL_SIMT");
+        return e && e[0] == '1';
+    }();
+    if (bf16 && !force_simt) return launch_prefill_tc(p, dk, dv, summaries, st);
+    return launch_prefill_simt(p, bf16, dk, dv, summaries, st);
+}
+
+}  // namespace kda
