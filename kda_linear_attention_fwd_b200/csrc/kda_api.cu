@@ -40,27 +40,8 @@ int sm_count() {
     return cache[dev];
 }
 
-long env_long(const char *name, long dflt) {
-    const char *s = std::getenv(name);
-    if (!s || !*s) return dflt;
-    char *end = nullptr;
-    const long v = std::strtol(s, &end, 10);
-    return (end && *end == 0 && v > 0) ? v : dflt;
-}
-
-// Piece length (tokens, multiple of 16, >= 256): enough independent
-// (piece, head) chains to cover the GPU about twice over, and no more --
-// every extra piece boundary costs a summary pass over the piece's tokens.
-int choose_piece_len(long total_tokens, int H) {
-    const long forced = env_long("KDA_PIECE_LEN", 0);
-    if (forced > 0) return (int)(((forced + 15) / 16) * 16);
-    const long chains = env_long("KDA_TARGET_CHAINS", 2L * sm_count());
-    long work = total_tokens * (long)H;
-    long L = (work + chains - 1) / chains;
-    L = ((L + 15) / 16) * 16;
-    if (L < 256) L = 256;
-    if (L > (1L << 30)) L = 1L << 30;
-    return (int)L;
+int choose_piece_len(long total_tokens, int num_seqs, int H, const int32_t *cu_host = nullptr) {
+    return kda::plan_piece_len(total_tokens, num_seqs, H, sm_count(), cu_host);
 }
 
 long max_pieces(long total_tokens, int num_seqs, int piece_len) {
@@ -88,7 +69,7 @@ size_t kda_chunk_fwd_workspace_size(int32_t total_tokens, int32_t num_seqs, int3
                                     int32_t dv, kda_dtype dtype) {
     if (total_tokens < 0 || num_seqs < 0 || H < 1 || !dim_ok(dk) || !dim_ok(dv)) return 0;
     if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return 0;
-    const int L = choose_piece_len(total_tokens, H);
+    const int L = choose_piece_len(total_tokens, num_seqs, H);
     const long P = max_pieces(total_tokens, num_seqs, L);
     return kda::workspace_layout(P, num_seqs, H, dk, dv).total;
 }
@@ -96,7 +77,7 @@ size_t kda_chunk_fwd_workspace_size(int32_t total_tokens, int32_t num_seqs, int3
 int kda_chunk_fwd_plan(int32_t total_tokens, int32_t num_seqs, int32_t H, int32_t *piece_len,
                        int32_t *max_pieces_out, int32_t *launches) {
     if (total_tokens < 0 || num_seqs < 0 || H < 1) return KDA_ERR_INVALID_ARG;
-    const int L = choose_piece_len(total_tokens, H);
+    const int L = choose_piece_len(total_tokens, num_seqs, H);
     const long P = max_pieces(total_tokens, num_seqs, L);
     if (piece_len) *piece_len = L;
     if (max_pieces_out) *max_pieces_out = (int32_t)(P > 0x7fffffffL ? 0x7fffffffL : P);
@@ -135,7 +116,9 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const void *g, co
         for (int n = 0; n < num_seqs; ++n)
             if (cu_seqlens_host[n + 1] < cu_seqlens_host[n]) return KDA_ERR_INVALID_ARG;
     }
-    const int L = choose_piece_len(total_tokens, H);
+    // the piece length with the real lengths, when known, is never shorter
+    // than the length-blind one the workspace was sized for
+    const int L = choose_piece_len(total_tokens, num_seqs, H, cu_seqlens_host);
     const long P_max = max_pieces(total_tokens, num_seqs, L);
     if (P_max > (1L << 30) || (long)H * P_max > (1L << 31)) return KDA_ERR_UNSUPPORTED;
     const kda::WorkspaceLayout WL = kda::workspace_layout(P_max, num_seqs, H, dk, dv);

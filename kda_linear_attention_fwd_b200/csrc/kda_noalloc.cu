@@ -68,14 +68,6 @@ int scratch_address(void **out) {
 bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
 bool dim_ok(int d) { return d == 64 || d == 128; }
 
-long env_piece_len() {
-    const char *s = std::getenv("KDA_PIECE_LEN");
-    if (!s || !*s) return 0;
-    char *end = nullptr;
-    const long v = std::strtol(s, &end, 10);
-    return (end && *end == 0 && v > 0) ? ((v + 15) / 16) * 16 : 0;
-}
-
 int sm_count() {
     int dev = 0, n = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -121,18 +113,11 @@ extern "C" int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v
             if (cu_seqlens_host[n + 1] < cu_seqlens_host[n]) return KDA_ERR_INVALID_ARG;
     }
 
-    // Piece length: the usual choice (about two (piece, head) chains per SM,
-    // at least 256 tokens), lengthened until the piece summaries fit in the
+    // Piece length: the usual plan, lengthened until the piece summaries fit in the
     // fixed scratch array.  Once a piece spans the whole input no summaries
     // are needed and only the plan table remains; if even that does not fit,
     // the sizes are beyond what this entry point supports.
-    long L = env_piece_len();
-    if (L == 0) {
-        const long chains = 2L * sm_count();
-        L = ((long)total_tokens * H + chains - 1) / chains;
-        L = ((L + 15) / 16) * 16;
-        if (L < 256) L = 256;
-    }
+    long L = kda::plan_piece_len(total_tokens, num_seqs, H, sm_count(), cu_seqlens_host);
     const long L_all = ((long)total_tokens + 15) / 16 * 16 + 16;
     for (;;) {
         const long P = (long)num_seqs + ((long)total_tokens + L - 1) / L;

@@ -79,53 +79,85 @@ __global__ void __launch_bounds__(1024)
 }
 
 // Prefix scan over the pieces of one sequence, for one head and one block of
-// 32 state columns:
+// 16 state columns:
 //   Sin[first]     = initial state (or zeros)
 //   Sin[first + 1] = Szero[first]       (piece 0 is summarised from the
 //                                         initial state itself, no M needed)
 //   Sin[first + j] = M[first + j - 1] Sin[first + j - 1] + Szero[first + j - 1]
-// fp32 throughout.  One warp per DK/8 rows, one lane per column.
+// fp32 throughout.  Each M (dk x dk) is staged in shared memory with cp.async,
+// the next one loading while the current product runs.  Thread t: column
+// t % 16, rows (t / 16) * DK/16 ... + DK/16 - 1.
+constexpr int kScanCols = 16;
+
+template <int DK, int DV>
+struct ScanSmem {
+    float M[2][DK * DK];
+    float Sp[DK][kScanCols + 1];
+    static constexpr size_t bytes() { return sizeof(float) * (2 * DK * DK + DK * (kScanCols + 1)); }
+};
+
 template <int DK, int DV>
 __global__ void __launch_bounds__(256) scan_kernel(PrefillParams p) {
-    constexpr int RW = DK / 8;  // rows per warp
-    __shared__ float Sp[DK][33];
-    const int n = blockIdx.x, h = blockIdx.y, c = blockIdx.z * 32 + (threadIdx.x & 31);
-    const int wid = threadIdx.x >> 5;
+    constexpr int RW = DK / 16;  // rows per thread
+    extern __shared__ __align__(16) unsigned char scan_smem[];
+    ScanSmem<DK, DV> &sm = *reinterpret_cast<ScanSmem<DK, DV> *>(scan_smem);
+    const int n = blockIdx.x, h = blockIdx.y;
+    const int col = threadIdx.x % kScanCols, rg = threadIdx.x / kScanCols;
+    const int c = blockIdx.z * kScanCols + col;
     const int f = p.seq_first[n];
     const int np = p.seq_first[n + 1] - f;
     if (np <= 1 || f + np > p.P_max) return;
     const int H = p.H;
     const size_t SS = (size_t)DK * DV, MS = (size_t)DK * DK;
     const float *init = p.initial_state ? p.initial_state + ((size_t)n * H + h) * SS : nullptr;
+
+    auto load_M = [&](int buf, int piece) {
+        const float4 *src = reinterpret_cast<const float4 *>(p.M + ((size_t)piece * H + h) * MS);
+        float4 *dst = reinterpret_cast<float4 *>(sm.M[buf]);
+        for (int x = threadIdx.x; x < DK * DK / 4; x += 256) {
+            const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst + x));
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(src + x)
+                         : "memory");
+        }
+        asm volatile("cp.async.commit_group;\n" ::: "memory");
+    };
+    if (np > 2) load_M(0, f + 1);
+
 #pragma unroll
     for (int r = 0; r < RW; ++r) {
-        const int i = wid * RW + r;
+        const int i = rg * RW + r;
         p.Sin[((size_t)f * H + h) * SS + (size_t)i * DV + c] = init ? init[(size_t)i * DV + c] : 0.f;
         const float z = p.Szero[((size_t)f * H + h) * SS + (size_t)i * DV + c];
         p.Sin[((size_t)(f + 1) * H + h) * SS + (size_t)i * DV + c] = z;
-        Sp[i][threadIdx.x & 31] = z;
+        sm.Sp[i][col] = z;
     }
-    __syncthreads();
     for (int j = 2; j < np; ++j) {
+        const int buf = j & 1;
+        if (j + 1 < np) {
+            load_M(buf ^ 1, f + j);
+            asm volatile("cp.async.wait_group 1;\n" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+        }
+        __syncthreads();
         const size_t pp = (size_t)(f + j - 1) * H + h;
-        const float *M = p.M + pp * MS;
+        const float *Ms = sm.M[buf];
         float acc[RW];
 #pragma unroll
-        for (int r = 0; r < RW; ++r)
-            acc[r] = p.Szero[pp * SS + (size_t)(wid * RW + r) * DV + c];
+        for (int r = 0; r < RW; ++r) acc[r] = p.Szero[pp * SS + (size_t)(rg * RW + r) * DV + c];
+#pragma unroll 4
         for (int kk = 0; kk < DK; ++kk) {
-            const float s = Sp[kk][threadIdx.x & 31];
+            const float sv = sm.Sp[kk][col];
 #pragma unroll
-            for (int r = 0; r < RW; ++r) acc[r] += M[(size_t)(wid * RW + r) * DK + kk] * s;
+            for (int r = 0; r < RW; ++r) acc[r] += Ms[(rg * RW + r) * DK + kk] * sv;
         }
         __syncthreads();
 #pragma unroll
         for (int r = 0; r < RW; ++r) {
-            const int i = wid * RW + r;
-            Sp[i][threadIdx.x & 31] = acc[r];
+            const int i = rg * RW + r;
+            sm.Sp[i][col] = acc[r];
             p.Sin[((size_t)(f + j) * H + h) * SS + (size_t)i * DV + c] = acc[r];
         }
-        __syncthreads();
     }
 }
 
@@ -136,13 +168,21 @@ cudaError_t launch_plan(const int32_t *cu, int num_seqs, int total_tokens, int p
     return cudaGetLastError();
 }
 
-cudaError_t launch_scan(const PrefillParams &p, int dk, int dv, cudaStream_t st) {
-    const dim3 grid(p.num_seqs, p.H, dv / 32);
-    if (dk == 128 && dv == 128) scan_kernel<128, 128><<<grid, 256, 0, st>>>(p);
-    else if (dk == 128 && dv == 64) scan_kernel<128, 64><<<grid, 256, 0, st>>>(p);
-    else if (dk == 64 && dv == 128) scan_kernel<64, 128><<<grid, 256, 0, st>>>(p);
-    else scan_kernel<64, 64><<<grid, 256, 0, st>>>(p);
+template <int DK, int DV>
+static cudaError_t launch_scan_t(const PrefillParams &p, cudaStream_t st) {
+    const size_t sm = ScanSmem<DK, DV>::bytes();
+    cudaError_t e = cudaFuncSetAttribute(scan_kernel<DK, DV>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    scan_kernel<DK, DV><<<dim3(p.num_seqs, p.H, DV / kScanCols), 256, sm, st>>>(p);
     return cudaGetLastError();
+}
+
+cudaError_t launch_scan(const PrefillParams &p, int dk, int dv, cudaStream_t st) {
+    if (dk == 128 && dv == 128) return launch_scan_t<128, 128>(p, st);
+    if (dk == 128 && dv == 64) return launch_scan_t<128, 64>(p, st);
+    if (dk == 64 && dv == 128) return launch_scan_t<64, 128>(p, st);
+    return launch_scan_t<64, 64>(p, st);
 }
 
 }  // namespace kda

@@ -24,6 +24,9 @@
 #pragma once
 
 #include <stdint.h>
+#include <stdlib.h>
+
+#include <algorithm>
 
 namespace kda {
 
@@ -53,6 +56,75 @@ inline WorkspaceLayout workspace_layout(long P_max, int num_seqs, int H, int dk,
     L.off_Sin = o;       o = align256(o + (size_t)P_max * H * dk * dv * sizeof(float));
     L.total = o;
     return L;
+}
+
+// ---------------------------------------------------------------- the plan
+// Piece length (tokens, a multiple of 16).  Each (piece, head) is one CTA of
+// the chunk kernels, which run one CTA per SM, so time is counted in whole
+// waves of `slots` CTAs.  A sequence of p > 1 pieces costs an output pass over
+// all p pieces plus a summary pass over 2p - 3 (piece, part) units (pieces
+// 0..p-2 summarise their zero-start state, pieces 1..p-2 their transition)
+// and p - 1 steps of the prefix scan.  With equal-length sequences (the
+// lengths are not known on the host in general) the model is
+//   cost(L) = waves(output) * chunks(L) + 0.8 * waves(summary) * chunks(L)
+//             + 2 * (pieces - 1)
+// in units of one chunk step; the summary pass has no outputs, hence 0.8.
+// When the host copy of the offsets is given, the real lengths are used, and
+// only piece lengths at least as long as the length-blind choice are
+// considered, so that the workspace sized without the lengths still fits.
+inline double plan_cost(long L, int num_seqs, int H, int slots, const int32_t *cu_host,
+                        long total_tokens) {
+    long out = 0, sum = 0, max_chunks = 0, max_pieces = 1;
+    for (int n = 0; n < (cu_host ? num_seqs : 1); ++n) {
+        const long len = cu_host ? (long)cu_host[n + 1] - cu_host[n]
+                                 : (total_tokens + num_seqs - 1) / num_seqs;
+        const long pcs = len <= 0 ? 1 : (len + L - 1) / L;
+        const long mult = cu_host ? 1 : num_seqs;
+        out += mult * pcs;
+        if (pcs > 1) sum += mult * (2 * pcs - 3);
+        const long ch = (std::min(len, L) + 15) / 16;
+        if (ch > max_chunks) max_chunks = ch;
+        if (pcs > max_pieces) max_pieces = pcs;
+    }
+    const long w_out = (out * H + slots - 1) / slots;
+    const long w_sum = (sum * H + slots - 1) / slots;
+    return (double)w_out * max_chunks + 0.8 * (double)w_sum * max_chunks +
+           2.0 * (double)(max_pieces - 1);
+}
+
+inline long env_positive(const char *name) {
+    const char *s = getenv(name);
+    if (!s || !*s) return 0;
+    char *end = nullptr;
+    const long v = strtol(s, &end, 10);
+    return (end && *end == 0 && v > 0) ? v : 0;
+}
+
+inline int plan_piece_len(long total_tokens, int num_seqs, int H, int sms,
+                          const int32_t *cu_host) {
+    const long forced = env_positive("KDA_PIECE_LEN");
+    if (forced > 0) return (int)(((forced + 15) / 16) * 16);
+    const long slots = env_positive("KDA_SLOTS") ? env_positive("KDA_SLOTS") : sms;
+    if (num_seqs <= 0 || total_tokens <= 0) return 256;
+    auto search = [&](const int32_t *cu, long Lref, long L_floor) {
+        long best_L = std::max<long>(((Lref + 15) / 16) * 16, 256);
+        best_L = std::max(best_L, L_floor);
+        double best = plan_cost(best_L, num_seqs, H, (int)slots, cu, total_tokens);
+        for (int pcs = 2; pcs <= 128; ++pcs) {
+            long L = ((Lref + pcs - 1) / pcs + 15) / 16 * 16;
+            if (L < 256 || L < L_floor) break;
+            const double c = plan_cost(L, num_seqs, H, (int)slots, cu, total_tokens);
+            if (c < best) { best = c; best_L = L; }
+        }
+        return best_L;
+    };
+    const long Lavg = (total_tokens + num_seqs - 1) / num_seqs;
+    const long L_blind = search(nullptr, Lavg, 0);
+    // the exact model walks every sequence per candidate: only for modest N
+    if (!cu_host || num_seqs > 8192) return (int)std::min<long>(L_blind, 1L << 30);
+    long Lmax = 0;
+    for (int n = 0; n < num_seqs; ++n) Lmax = std::max<long>(Lmax, (long)cu_host[n + 1] - cu_host[n]);
+    return (int)std::min<long>(search(cu_host, std::max(Lmax, L_blind), L_blind), 1L << 30);
 }
 
 struct PrefillParams {

@@ -40,13 +40,16 @@ namespace tc {
 using bf16 = __nv_bfloat16;
 
 constexpr int kThreads = 256;     // 4 state warps + 4 prep warps
+constexpr int kStages = 4;        // one stage per prep warp
 constexpr int kPad = 8;           // bf16 row padding: conflict-free ldmatrix
 constexpr int kL16 = 16 + kPad;   // row length of the 16 x 16 bf16 tiles
 
-// named barriers (0 is __syncthreads)
-constexpr int BAR_PREP = 1;       // prep warps only (128 threads)
-constexpr int BAR_FULL = 2;       // + stage: prep arrives, state waits (256)
-constexpr int BAR_EMPTY = 4;      // + stage: state arrives, prep waits (256)
+// Named barriers (0 is __syncthreads).  Stage s is filled by prep warp s and
+// drained by the four state warps: FULL[s] (prep arrives, state waits) and
+// EMPTY[s] (state arrives, prep waits), 32 + 128 threads each.
+constexpr int BAR_FULL = 1;       // ids 1..4
+constexpr int BAR_EMPTY = 5;      // ids 5..8
+constexpr int kBarCount = 160;
 
 KDA_DEVICE uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -58,6 +61,10 @@ KDA_DEVICE void bar_arrive(int id, int n) {
 KDA_DEVICE uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
+}
+KDA_DEVICE float2 unpack_bf16(uint32_t x) {
+    __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162 *>(&x);
+    return __bfloat1622float2(v);
 }
 KDA_DEVICE void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -86,7 +93,7 @@ template <int N> KDA_DEVICE void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
-// Lane addressing of ldmatrix.x4 for the three fragment kinds used here.
+// Lane addressing of ldmatrix.x4 for the fragment kinds used here.
 //  A operand, row-major [m][k] storage:       row (l&7)+((l>>3)&1)*8, col (l>>4)*8
 //  B operand from [n][k] storage (k inner):   n (l&7)+(l>>4)*8,       k ((l>>3)&1)*8
 //  B operand from [k][n] storage, .trans:     k (l&7)+((l>>3)&1)*8,   n (l>>4)*8
@@ -100,26 +107,25 @@ struct Layout {
     static constexpr int MT = NC / 64;    // m16 tiles per state warp
     static constexpr int CW = NC / 4;     // state columns per state warp
     static constexpr int LY = CW + 4;     // output staging row (fp32)
-    struct Raw {                          // cp.async targets, unpadded rows
-        bf16 q[16 * DK], k[16 * DK], g[16 * DK], v[16 * NC], gate[16 * NC];
+    struct Raw {                          // cp.async targets of one prep warp
+        bf16 q[16 * DK], k[16 * DK], g[16 * DK];
     };
-    struct Stage {                        // handed from prep to state warps
+    struct Stage {                        // handed from a prep warp to the state warps
         bf16 qd[16 * LK], kb[16 * LK], wn[16 * LK];
         bf16 v[16 * LC], gate[16 * LC];
         bf16 p[16 * kL16], tb[16 * kL16];
         float gam[DK];
     };
-    struct Prep {                         // private to the prep warps
+    struct Prep {                         // private to one prep warp
         bf16 kd[16 * LK], ki[16 * LK];
         float A[16 * 17];
-        float beta[2][16];
-        float red[2][4][16];
+        float beta[16];
         float rq[16], rk[16];
     };
     struct All {
-        Raw raw[2];
-        Stage st[2];
-        Prep pr;
+        Raw raw[kStages];
+        Stage st[kStages];
+        Prep pr[kStages];
         float ys[4][16 * LY];
     };
     static constexpr size_t bytes = sizeof(All);
@@ -156,8 +162,8 @@ __device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const 
                 }
         bf16 *out = (bf16 *)p.out;
         for (int c = 0; c < nchunks; ++c) {
-            const int stg = c & 1;
-            bar_sync(BAR_FULL + stg, kThreads);
+            const int stg = c & (kStages - 1);
+            bar_sync(BAR_FULL + stg, kBarCount);
             typename Lay::Stage &S = sm.st[stg];
             float u[MT][2][4], o[MT][2][4];
 #pragma unroll
@@ -258,13 +264,14 @@ __device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const 
                     bf16 *dst = out + ((size_t)(t0 + 16 * c + r) * H + h) * NC + jb + jl0;
 #pragma unroll
                     for (int v8 = 0; v8 < HALF / 8; ++v8) {
+                        const uint4 gv = *reinterpret_cast<const uint4 *>(&S.gate[r * LC + jb + jl0 + 8 * v8]);
+                        const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
                         uint32_t pk[4];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const int jl = jl0 + 8 * v8 + 2 * e;
-                            const float g0 = __bfloat162float(S.gate[r * LC + jb + jl]);
-                            const float g1 = __bfloat162float(S.gate[r * LC + jb + jl + 1]);
-                            pk[e] = pack_bf16(g0 * ys[r * LY + jl], g1 * ys[r * LY + jl + 1]);
+                            const float2 gg = unpack_bf16(gw[e]);
+                            pk[e] = pack_bf16(gg.x * ys[r * LY + jl], gg.y * ys[r * LY + jl + 1]);
                         }
                         *reinterpret_cast<uint4 *>(dst + 8 * v8) =
                             make_uint4(pk[0], pk[1], pk[2], pk[3]);
@@ -272,7 +279,7 @@ __device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const 
                 }
                 __syncwarp();
             }
-            bar_arrive(BAR_EMPTY + stg, kThreads);
+            bar_arrive(BAR_EMPTY + stg, kBarCount);
         }
         if (s_out) {
 #pragma unroll
@@ -290,19 +297,22 @@ __device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const 
     }
 
     // ---------------------------------------------------------------- prep
-    const int pt = tid - 128, pw = pt >> 5;
+    // Prep warp pw prepares chunks pw, pw + 4, pw + 8, ... into stage pw.
+    const int pw = warp - 4;
     const bf16 *q = (const bf16 *)p.q, *k = (const bf16 *)p.k, *g = (const bf16 *)p.g;
     const bf16 *v = (const bf16 *)p.v, *gate = (const bf16 *)p.gate, *beta = (const bf16 *)p.beta;
-    typename Lay::Prep &pr = sm.pr;
+    typename Lay::Prep &pr = sm.pr[pw];
+    typename Lay::Raw &R = sm.raw[pw];
+    typename Lay::Stage &S = sm.st[pw];
     float beta_next = 0.f;
 
-    // raw tiles of chunk c -> raw[c & 1]; rows past the piece are zero-filled
-    auto issue = [&](int c) {
-        typename Lay::Raw &R = sm.raw[c & 1];
+    // q, k, g of chunk c -> this warp's raw buffer (rows past the piece are zero)
+    auto issue_raw = [&](int c) {
         const int tc = t0 + 16 * c;
         const int rows = min(16, len - 16 * c);
         constexpr int PK = DK / 8;  // 16-byte pieces per row
-        for (int x = pt; x < 16 * PK; x += 128) {
+#pragma unroll 4
+        for (int x = lane; x < 16 * PK; x += 32) {
             const int r = x / PK, cc = x % PK;
             const bool ok = r < rows;
             const size_t off = ((size_t)(ok ? tc + r : t0) * H + h) * DK + cc * 8;
@@ -310,42 +320,37 @@ __device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const 
             cp_async16(&R.g[r * DK + cc * 8], g + off, ok);
             if (OUT) cp_async16(&R.q[r * DK + cc * 8], q + off, ok);
         }
-        if (USE_V || OUT) {
-            constexpr int PV = NC / 8;
-            for (int x = pt; x < 16 * PV; x += 128) {
-                const int r = x / PV, cc = x % PV;
-                const bool ok = r < rows;
-                const size_t off = ((size_t)(ok ? tc + r : t0) * H + h) * NC + cc * 8;
-                if (USE_V) cp_async16(&R.v[r * NC + cc * 8], v + off, ok);
-                if (OUT) {
-                    if (gate) cp_async16(&R.gate[r * NC + cc * 8], gate + off, ok);
-                }
-            }
+        cp_async_commit();
+        beta_next = lane < rows ? __bfloat162float(beta[(size_t)(tc + lane) * H + h]) : 0.f;
+    };
+    // v and gate of chunk c -> the stage itself (padded rows)
+    auto issue_vg = [&](int c) {
+        const int tc = t0 + 16 * c;
+        const int rows = min(16, len - 16 * c);
+        constexpr int PV = NC / 8;
+#pragma unroll 4
+        for (int x = lane; x < 16 * PV; x += 32) {
+            const int r = x / PV, cc = x % PV;
+            const bool ok = r < rows;
+            const size_t off = ((size_t)(ok ? tc + r : t0) * H + h) * NC + cc * 8;
+            if (USE_V) cp_async16(&S.v[r * LC + cc * 8], v + off, ok);
+            if (OUT && gate) cp_async16(&S.gate[r * LC + cc * 8], gate + off, ok);
         }
         cp_async_commit();
-        if (pt < 16) beta_next = pt < rows ? __bfloat162float(beta[(size_t)(tc + pt) * H + h]) : 0.f;
     };
 
-    if (nchunks > 0) issue(0);
-    for (int c = 0; c < nchunks; ++c) {
-        const int stg = c & 1;
-        typename Lay::Raw &R = sm.raw[stg];
-        if (pt < 16) pr.beta[stg][pt] = beta_next;
-        if (c + 1 < nchunks) {
-            issue(c + 1);
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
-        }
-        if (c >= 2) bar_sync(BAR_EMPTY + stg, kThreads);
-        bar_sync(BAR_PREP, 128);
-        typename Lay::Stage &S = sm.st[stg];
-        const float *bet = pr.beta[stg];
+    if (pw < nchunks) issue_raw(pw);
+    for (int c = pw; c < nchunks; c += kStages) {
+        if (c >= kStages) bar_sync(BAR_EMPTY + pw, kBarCount);  // stage free again
+        issue_vg(c);
+        if (lane < 16) pr.beta[lane] = beta_next;
+        cp_async_wait<1>();  // raw q, k, g of chunk c have landed
+        __syncwarp();
 
         if (p.qk_l2norm) {  // 1/|q_r|, 1/|k_r| over the head dimension
             for (int r = 0; r < 16; ++r) {
                 float kk = 0.f, qq = 0.f;
-                for (int i = pt; i < DK; i += 128) {
+                for (int i = lane; i < DK; i += 32) {
                     const float kv = __bfloat162float(R.k[r * DK + i]);
                     kk += kv * kv;
                     if (OUT) {
@@ -355,75 +360,68 @@ __device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const 
                 }
                 kk = warp_sum(kk);
                 qq = warp_sum(qq);
-                if (lane == 0) {
-                    pr.red[0][pw][r] = kk;
-                    pr.red[1][pw][r] = qq;
+                if (lane == r) {
+                    pr.rk[r] = rsqrtf(kk + 1e-6f);
+                    pr.rq[r] = rsqrtf(qq + 1e-6f);
                 }
             }
-            bar_sync(BAR_PREP, 128);
-            if (pt < 16) {
-                const float kk = pr.red[0][0][pt] + pr.red[0][1][pt] + pr.red[0][2][pt] + pr.red[0][3][pt];
-                const float qq = pr.red[1][0][pt] + pr.red[1][1][pt] + pr.red[1][2][pt] + pr.red[1][3][pt];
-                pr.rk[pt] = rsqrtf(kk + 1e-6f);
-                pr.rq[pt] = rsqrtf(qq + 1e-6f);
-            }
-            bar_sync(BAR_PREP, 128);
+            __syncwarp();
         }
 
-        // 1. per key channel: decay factors and the decayed bf16 operands
-        if (pt < DK) {
-            const int i = pt;
-            float e[16], E[16], F[16];
+        // 1. decay factors and the decayed bf16 operands; lane owns channel
+        //    pairs (2 lane, 2 lane + 1) + 64 x
 #pragma unroll
-            for (int r = 0; r < 16; ++r) e[r] = __expf(__bfloat162float(R.g[r * DK + i]));
-            float acc = 1.f;
-#pragma unroll
-            for (int r = 0; r < 16; ++r) { acc *= e[r]; E[r] = acc; }
-            acc = 1.f;
-#pragma unroll
-            for (int r = 15; r >= 0; --r) { F[r] = acc; acc *= e[r]; }
-            const float El = E[15];
-            const float invEl = 1.f / El;
-            S.gam[i] = El;
+        for (int cp2 = 0; cp2 < DK / 64; ++cp2) {
+            const int i = 64 * cp2 + 2 * lane;
+            float2 e[16], E[16];
 #pragma unroll
             for (int r = 0; r < 16; ++r) {
-                float kv = __bfloat162float(R.k[r * DK + i]);
-                if (p.qk_l2norm) kv *= pr.rk[r];
-                pr.kd[r * LK + i] = __float2bfloat16_rn(kv * E[r]);
-                pr.ki[r * LK + i] = __float2bfloat16_rn(kv * (F[r] * invEl));
-                S.kb[r * LK + i] = __float2bfloat16_rn(kv * F[r]);
+                const float2 gg = unpack_bf16(*reinterpret_cast<const uint32_t *>(&R.g[r * DK + i]));
+                e[r] = make_float2(__expf(gg.x), __expf(gg.y));
+            }
+            float2 acc = make_float2(1.f, 1.f);
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                acc.x *= e[r].x; acc.y *= e[r].y;
+                E[r] = acc;
+            }
+            const float2 El = acc;
+            const float2 invEl = make_float2(1.f / El.x, 1.f / El.y);
+            *reinterpret_cast<float2 *>(&S.gam[i]) = El;
+            float2 F = make_float2(1.f, 1.f);  // exp(G_C - G_r), suffix products
+#pragma unroll
+            for (int r = 15; r >= 0; --r) {
+                float2 kv = unpack_bf16(*reinterpret_cast<const uint32_t *>(&R.k[r * DK + i]));
+                if (p.qk_l2norm) { kv.x *= pr.rk[r]; kv.y *= pr.rk[r]; }
+                *reinterpret_cast<uint32_t *>(&pr.kd[r * LK + i]) = pack_bf16(kv.x * E[r].x, kv.y * E[r].y);
+                *reinterpret_cast<uint32_t *>(&pr.ki[r * LK + i]) =
+                    pack_bf16(kv.x * (F.x * invEl.x), kv.y * (F.y * invEl.y));
+                *reinterpret_cast<uint32_t *>(&S.kb[r * LK + i]) = pack_bf16(kv.x * F.x, kv.y * F.y);
                 if (OUT) {
-                    float qv = __bfloat162float(R.q[r * DK + i]) * p.scale;
-                    if (p.qk_l2norm) qv *= pr.rq[r];
-                    S.qd[r * LK + i] = __float2bfloat16_rn(qv * E[r]);
+                    float2 qv = unpack_bf16(*reinterpret_cast<const uint32_t *>(&R.q[r * DK + i]));
+                    float sc = p.scale;
+                    if (p.qk_l2norm) sc *= pr.rq[r];
+                    *reinterpret_cast<uint32_t *>(&S.qd[r * LK + i]) =
+                        pack_bf16(qv.x * sc * E[r].x, qv.y * sc * E[r].y);
                 }
+                F.x *= e[r].x; F.y *= e[r].y;
             }
         }
-        // copy v and gate into the stage (the raw buffer is refilled early)
-        if (USE_V || OUT) {
-            constexpr int PV = NC / 8;
-            for (int x = pt; x < 16 * PV; x += 128) {
-                const int r = x / PV, cc = x % PV;
-                if (USE_V)
-                    *reinterpret_cast<uint4 *>(&S.v[r * LC + cc * 8]) =
-                        *reinterpret_cast<const uint4 *>(&R.v[r * NC + cc * 8]);
-                if (OUT) {
-                    uint4 gv;
-                    if (gate) {
-                        gv = *reinterpret_cast<const uint4 *>(&R.gate[r * NC + cc * 8]);
-                    } else {
-                        const uint32_t one = pack_bf16(1.f, 1.f);
-                        gv = make_uint4(one, one, one, one);
-                    }
-                    *reinterpret_cast<uint4 *>(&S.gate[r * LC + cc * 8]) = gv;
-                }
+        if (OUT && !gate) {
+            const uint32_t one = pack_bf16(1.f, 1.f);
+            for (int x = lane; x < 16 * NC / 8; x += 32) {
+                const int r = x / (NC / 8), cc = x % (NC / 8);
+                *reinterpret_cast<uint4 *>(&S.gate[r * LC + cc * 8]) = make_uint4(one, one, one, one);
             }
         }
-        bar_sync(BAR_PREP, 128);
+        __syncwarp();
+        // the raw buffer is free: prefetch this warp's next chunk
+        if (c + kStages < nchunks) issue_raw(c + kStages);
 
         // 2. A = Kd Ki^T (strictly lower, fp32) and P = Qd Ki^T (lower, bf16)
-        if (pw == 0 || (OUT && pw == 1)) {
-            const bf16 *Aop = pw == 0 ? pr.kd : S.qd;
+#pragma unroll
+        for (int which = 0; which < (OUT ? 2 : 1); ++which) {
+            const bf16 *Aop = which == 0 ? pr.kd : S.qd;
             float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int kk = 0; kk < DK / 16; ++kk) {
@@ -440,39 +438,43 @@ __device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const 
             for (int e = 0; e < 8; ++e) {
                 const int r = r0 + ((e & 2) ? 8 : 0);
                 const int sc = c0 + (e & 1) + ((e & 4) ? 8 : 0);
-                if (pw == 0) {
+                if (which == 0) {
                     pr.A[r * 17 + sc] = sc < r ? vals[e] : 0.f;
                 } else {
                     S.p[r * kL16 + sc] = __float2bfloat16_rn(sc <= r ? vals[e] : 0.f);
                 }
             }
         }
-        bar_sync(BAR_PREP, 128);
+        __syncwarp();
 
-        // 3. Tb = (I + Diag(beta) A)^-1 Diag(beta): forward substitution, lane = column
-        if (pw == 0 && lane < 16) {
+        // 3. Tb = (I + Diag(beta) A)^-1 Diag(beta): forward substitution.
+        //    Lane j < 16 owns column j; after row r is final it is pushed into
+        //    the partial sums of every later row (independent updates).
+        if (lane < 16) {
             const int j = lane;
             float col[16];
 #pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                float acc = 0.f;
+            for (int r = 0; r < 16; ++r) col[r] = (r == j) ? 1.f : 0.f;
 #pragma unroll
-                for (int s2 = 0; s2 < r; ++s2) acc += pr.A[r * 17 + s2] * col[s2];
-                col[r] = (r == j ? 1.f : 0.f) - bet[r] * acc;
+            for (int r = 0; r < 16; ++r) {
+                // col[r] is final here: delta_rj - beta_r sum_{s<r} A[r][s] col[s]
+#pragma unroll
+                for (int r2 = r + 1; r2 < 16; ++r2)
+                    col[r2] -= pr.beta[r2] * pr.A[r2 * 17 + r] * col[r];
             }
-            const float bj = bet[j];
+            const float bj = pr.beta[j];
 #pragma unroll
             for (int r = 0; r < 16; ++r) S.tb[r * kL16 + j] = __float2bfloat16_rn(col[r] * bj);
         }
-        bar_sync(BAR_PREP, 128);
+        __syncwarp();
 
-        // 4. W = Tb Kd -> stage holds -W (bf16); prep warp pw owns DK/4 columns
+        // 4. W = Tb Kd -> the stage holds -W (bf16)
         {
             uint32_t a[4];
             ldsm4(a, &S.tb[((lane & 7) + ((lane >> 3) & 1) * 8) * kL16 + (lane >> 4) * 8]);
 #pragma unroll
-            for (int np = 0; np < DK / 64; ++np) {
-                const int n0 = pw * (DK / 4) + 16 * np;
+            for (int np = 0; np < DK / 16; ++np) {
+                const int n0 = 16 * np;
                 uint32_t b[4];
                 ldsm4t(b, &pr.kd[((lane & 7) + ((lane >> 3) & 1) * 8) * LK + n0 + (lane >> 4) * 8]);
                 float w0[4] = {0.f, 0.f, 0.f, 0.f}, w1[4] = {0.f, 0.f, 0.f, 0.f};
@@ -485,10 +487,13 @@ __device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const 
                 *reinterpret_cast<uint32_t *>(&S.wn[(r + 8) * LK + cc + 8]) = pack_bf16(-w1[2], -w1[3]);
             }
         }
-        bar_arrive(BAR_FULL + stg, kThreads);
+        // v and gate of chunk c have landed (the raw prefetch may still run)
+        if (c + kStages < nchunks) cp_async_wait<1>(); else cp_async_wait<0>();
+        __syncwarp();
+        bar_arrive(BAR_FULL + pw, kBarCount);
     }
-    // balance the state warps' last EMPTY arrivals
-    for (int c = nchunks - 2 < 0 ? 0 : nchunks - 2; c < nchunks; ++c) bar_sync(BAR_EMPTY + (c & 1), kThreads);
+    // consume the state warps' EMPTY arrival for this warp's last chunk
+    if (pw < nchunks) bar_sync(BAR_EMPTY + pw, kBarCount);
 }
 
 template <int DK, int DV>

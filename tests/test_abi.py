@@ -64,8 +64,16 @@ def test_workspace_size(lib):
     assert f(16, 1, 1, 96, 64, F32) == 0
     assert f(16, 1, 0, 64, 64, F32) == 0
     assert f(16, 1, 1, 64, 64, 7) == 0
-    # grows with the number of heads and with the state size
-    assert f(8192, 2, 32, 128, 128, BF16) > f(8192, 2, 16, 128, 128, BF16)
+    # covers the plan: one transition and two states per (piece, head)
+    for T, N, H, dk, dv in [(8192, 2, 32, 128, 128), (8192, 2, 16, 128, 128),
+                            (131072, 1, 32, 128, 128), (48317, 8, 32, 128, 128),
+                            (5000, 7, 3, 64, 128)]:
+        plan = kda.plan(T, N, H)
+        per_piece = H * (dk * dk + 2 * dk * dv) * 4
+        assert plan["piece_len"] % 16 == 0 and plan["piece_len"] >= 256
+        assert plan["max_pieces"] >= N + (T + plan["piece_len"] - 1) // plan["piece_len"] - 1
+        assert f(T, N, H, dk, dv, BF16) >= plan["max_pieces"] * per_piece
+    # a larger state needs more workspace for the same plan
     assert f(8192, 2, 16, 128, 128, BF16) > f(8192, 2, 16, 64, 64, BF16)
 
 
