@@ -123,16 +123,23 @@ class Clocks:
                 "samples": len(sm)}
 
 
-def dist_setup(args):
-    ws = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+def rank_env():
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def dist_setup(backend="nccl"):
+    """One process per GPU: a process group for the barrier and the
+    max-over-ranks timing only (the work itself needs no collective)."""
+    ws, rank, local = rank_env()
     if ws > 1:
         import torch.distributed as dist
         from datetime import timedelta
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=timedelta(seconds=300), **kw)
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return ws, rank, local
@@ -144,13 +151,19 @@ def barrier(ws):
         dist.barrier()
 
 
-def reduce_max(x, ws):
+def reduce_max(x, ws, device="cuda"):
+    """Max over ranks (device time of the slowest rank)."""
     if ws == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate(units_per_rank, ms_total, ws):
+    """Whole-job throughput: units processed by all ranks / slowest time."""
+    return ws * units_per_rank / (ms_total / 1e3)
 
 
 def cpu_baseline(w, threads=None, tokens=None):
@@ -182,15 +195,13 @@ def run_reference(args, ws, rank):
         return
     w = W.get(args.workload)
     cores = os.cpu_count() or 1
-    tokens = int(min(w.lengths[0], max(1024, 256 * cores)))
+    tokens = args.ref_tokens or int(min(w.lengths[0], max(1024, 256 * cores)))
     for _ in range(args.warmup):
         cpu_baseline(w, cores, tokens)
-    vals = []
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
+    el = 0.0
+    for _ in range(args.steps):  # oracle time only (input generation excluded)
         v, used, sample = cpu_baseline(w, cores, tokens)
-        vals.append(v)
-    el = time.perf_counter() - t0
+        el += tokens / v
     value = args.steps * tokens / el
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup,
@@ -220,16 +231,18 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--out-dir", default=os.path.join(ROOT, "gpurun_out"))
+    ap.add_argument("--ref-tokens", type=int, default=0,
+                    help="reference arm: tokens per step sample (0 = scale with cores)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
 
-    ws, rank, local = dist_setup(args)
     if args.impl == "reference":
+        # CPU oracle on rank 0 only; other ranks exit without work and
+        # without a process group (no collective can wait on them)
+        ws, rank, _ = rank_env()
         run_reference(args, ws, rank)
-        if ws > 1:
-            import torch.distributed as dist
-            dist.destroy_process_group()
         return
+    ws, rank, local = dist_setup("nccl")
 
     from kda_linear_attention_fwd_b200 import build
     if rank == 0:
@@ -274,7 +287,7 @@ def main():
     ms_total = reduce_max(e0.elapsed_time(e1), ws)
     clk = clocks.stop()
     ms = ms_total / args.steps
-    value = ws * T * args.steps / (ms_total / 1e3)
+    value = aggregate(T * args.steps, ms_total, ws)
     pbytes = prefill_bytes(w, T, N)
     pflops = prefill_flops(w, T)
     hbm = pk["hbm_gbs"]
