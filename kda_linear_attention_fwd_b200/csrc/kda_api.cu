@@ -129,6 +129,7 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const void *g, co
     p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.gate = gate; p.out = out;
     p.cu_seqlens = cu_seqlens;
     p.header = (const int32_t *)(ws + WL.off_header);
+    p.err = (int32_t *)(ws + WL.off_header) + 2;
     p.seq_first = (const int32_t *)(ws + WL.off_seq_first);
     p.pieces = (const int4 *)(ws + WL.off_pieces);
     p.M = (float *)(ws + WL.off_M);

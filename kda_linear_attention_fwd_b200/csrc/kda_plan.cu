@@ -62,6 +62,7 @@ __global__ void __launch_bounds__(1024)
         seq_first[num_seqs] = P;
         header[0] = min(P, P_max);
         header[1] = bad_s | (P > P_max ? 2 : 0);
+        header[2] = 0;
     }
     __syncthreads();
     for (int n = tid; n < num_seqs; n += 1024) {

@@ -33,7 +33,8 @@ namespace kda {
 constexpr int kChunk = 16;
 
 // Workspace layout (all offsets 256-byte aligned), for P_max pieces:
-//   int32 plan header [64]           : [0] = number of pieces P
+//   int32 plan header [64]           : [0] = number of pieces P, [1] = offsets
+//                                      inconsistent, [2] = device wait timed out
 //   int32 seq_first   [num_seqs + 1] : first piece of each sequence
 //   int4  pieces      [P_max]        : {seq, token start, length, index in seq}
 //   fp32  M           [P_max][H][dk][dk]   transition of each piece
@@ -60,8 +61,8 @@ inline WorkspaceLayout workspace_layout(long P_max, int num_seqs, int H, int dk,
 
 // ---------------------------------------------------------------- the plan
 // Piece length (tokens, a multiple of 16).  Each (piece, head) is one CTA of
-// the chunk kernels, which run one CTA per SM, so time is counted in whole
-// waves of `slots` CTAs.  A sequence of p > 1 pieces costs an output pass over
+// the chunk kernels, which run two CTAs per SM, so time is counted in whole
+// waves of `slots` = 2 x SMs CTAs.  A sequence of p > 1 pieces costs an output pass over
 // all p pieces plus a summary pass over 2p - 3 (piece, part) units (pieces
 // 0..p-2 summarise their zero-start state, pieces 1..p-2 their transition)
 // and p - 1 steps of the prefix scan.  With equal-length sequences (the
@@ -104,7 +105,8 @@ inline int plan_piece_len(long total_tokens, int num_seqs, int H, int sms,
                           const int32_t *cu_host) {
     const long forced = env_positive("KDA_PIECE_LEN");
     if (forced > 0) return (int)(((forced + 15) / 16) * 16);
-    const long slots = env_positive("KDA_SLOTS") ? env_positive("KDA_SLOTS") : sms;
+    // the bf16 dk = dv = 128 chunk kernels run two CTAs per SM
+    const long slots = env_positive("KDA_SLOTS") ? env_positive("KDA_SLOTS") : 2L * sms;
     if (num_seqs <= 0 || total_tokens <= 0) return 256;
     auto search = [&](const int32_t *cu, long Lref, long L_floor) {
         long best_L = std::max<long>(((Lref + 15) / 16) * 16, 256);
@@ -137,6 +139,7 @@ struct PrefillParams {
     float *M, *Szero, *Sin;
     const float *initial_state;
     float *final_state;
+    int32_t *err;  // header[2]: set to nonzero when a bounded device wait gave up
     int num_seqs, H, P_max;
     float scale;
     int qk_l2norm;

@@ -563,17 +563,24 @@ cudaError_t launch_prefill_tc(const PrefillParams &p, int dk, int dv, bool summa
     return tc::launch_t<64, 64>(p, summaries, st);
 }
 
-// The chunk pass for one call: bf16 inputs run on the tensor cores; fp32
-// inputs run the fp32 CUDA-core kernel (bf16 operands would not reach fp32
-// accuracy).  KDA_PREFILL_SIMT=1 forces the CUDA-core kernel for bf16 too.
+cudaError_t launch_prefill_tc5(const PrefillParams &p, bool summaries, cudaStream_t st);
+
+// The chunk pass for one call.  bf16 inputs run on the tensor cores: the
+// tcgen05 kernel for dk = dv = 128, the warp-level MMA kernel for the other
+// head sizes.  fp32 inputs run the fp32 CUDA-core kernel (bf16 operands would
+// not reach fp32 accuracy).  KDA_PREFILL_IMPL=mma|simt forces a kernel.
 cudaError_t launch_prefill_chunks(const PrefillParams &p, bool bf16, int dk, int dv,
                                   bool summaries, cudaStream_t st) {
-    static const bool force_simt = [] {
-        const char *e = std::getenv("KDA_PREFILL_SIMT");
-        return e && e[0] == '1';
+    static const int forced = [] {
+        const char *e = std::getenv("KDA_PREFILL_IMPL");
+        if (!e) return 0;
+        if (e[0] == 'm') return 1;
+        if (e[0] == 's') return 2;
+        return 0;
     }();
-    if (bf16 && !force_simt) return launch_prefill_tc(p, dk, dv, summaries, st);
-    return launch_prefill_simt(p, bf16, dk, dv, summaries, st);
+    if (!bf16 || forced == 2) return launch_prefill_simt(p, bf16, dk, dv, summaries, st);
+    if (forced == 0 && dk == 128 && dv == 128) return launch_prefill_tc5(p, summaries, st);
+    return launch_prefill_tc(p, dk, dv, summaries, st);
 }
 
 }  // namespace kda

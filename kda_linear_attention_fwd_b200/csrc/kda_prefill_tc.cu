@@ -1,0 +1,674 @@
+// KDA prefill, 16-token chunk pass with the state contractions on the
+// 5th-generation tensor cores (tcgen05, accumulators in tensor memory).
+//
+// One CTA runs one piece of one head (dk = dv = 128).  Warps 0-3 form the
+// state warpgroup: thread j owns state column j -- row j of S^T, fp32, in
+// registers -- and TMEM lane j.  Per chunk (see kda_prefill_simt.cu for the
+// algebra), with everything the chunk needs prepared one chunk ahead by the
+// prep warps:
+//
+//   MMA 1  D1      = V^T [Tb^T | 0]             (M=128, N=32, K=16; A MN-major smem)
+//   MMA 2  D1     += S^T [-W^T | Qd^T]          (K=128; A = bf16 S^T in TMEM)
+//          -> D1[:, 0:16] = U^T, D1[:, 16:32] = (Qd S)^T
+//   WG     U^T (bf16) -> shared memory (A operand of the next two)
+//   MMA 3  D2      = U^T Kb                     (M=128, N=128, K=16)
+//   MMA 4  D1[16:] += U^T P^T                   (M=128, N=16, K=16) -> O^T
+//   WG     y = gate (.) O;  S^T <- S^T Diag(exp G_C) + D2 (fp32, registers);
+//          bf16 copy of S^T -> TMEM (A operand of the next chunk's MMA 2)
+//
+// One thread issues the MMAs; tcgen05.commit arrives on an mbarrier that the
+// warpgroup waits on with a time bound (2 s): a wait that gives up records an
+// error in the workspace header and the kernel drains without further tensor
+// work, keeping every named-barrier hand-off so that no warp is left waiting.
+//
+// Prep warps 4-7 each own every fourth chunk: cp.async of q, k, g into a
+// private buffer and of v and gate straight into the stage, exp(G) as prefix
+// and suffix products of exp(g), the Gram matrices A = Kd Ki^T and
+// P = Qd Ki^T and W = Tb Kd on warp-level MMA (16x16 tiles are far below the
+// smallest tcgen05 tile), and the 16x16 unit-lower solve in fp32.  Every MMA
+// operand is written in the canonical no-swizzle K-major / MN-major layout.
+//
+// Sources: the token pipeline and the decay floor -- affta.cn K3 explainer,
+// section "第一关：KDA 解决算得动"; decay as an absolute-position transform over a
+// 16-token tile -- prism.simon-ai.net, "从架构创新出发：K3的MoE与混合注意力设计",
+// section "数值稳定性与 Co-Design：BF16 约束下的衰减控制策略"; the split into
+// parallel per-chunk preparation and a sequential state pass -- affta.cn page,
+// section "FlashKDA ，让线性计算也能沾上并行的光".
+#include "kda_common.cuh"
+#include "kda_prefill.cuh"
+#include "kda_sm100.cuh"
+
+// Optional timeline hooks for one CTA (piece 1, head 0), compiled only with
+// -DKDA_TC5_TRACE: SM clock at fixed points of the state warpgroup's and the
+// prep warps' chunk loops, read back through kda_tc5_trace_copy().
+#ifdef KDA_TC5_TRACE
+__device__ unsigned long long g_kda_tc5_trace[8192];
+#define KDA_MARK(cond, slot)                                                          \
+    do {                                                                              \
+        if ((cond) && blockIdx.x == 1 && blockIdx.y == 0 && blockIdx.z == 0 &&        \
+            (slot) < 8192)                                                            \
+            g_kda_tc5_trace[(slot)] = clock64();                                      \
+        __syncwarp();                                                                 \
+    } while (0)
+extern "C" int kda_tc5_trace_copy(unsigned long long *host, int n) {
+    return cudaMemcpyFromSymbol(host, g_kda_tc5_trace, sizeof(unsigned long long) * n) ==
+                   cudaSuccess ? 0 : -1;
+}
+#else
+#define KDA_MARK(cond, slot) do { } while (0)
+#endif
+
+namespace kda {
+namespace tc5 {
+
+using namespace sm100;
+
+constexpr int kPrepWarps = 3;                 // = stages; chunk c -> prep warp c % 3
+constexpr int kThreads = 128 + 32 * kPrepWarps;
+constexpr int kBlocksPerSM = 2;
+constexpr int BAR_FULL = 1;    // ids 1..3: prep warp s arrives, state warpgroup waits
+constexpr int BAR_EMPTY = 4;   // ids 4..6: state warpgroup arrives, prep warp s waits
+constexpr int BAR_WG = 7;      // state warpgroup only
+constexpr int kBarCount = 160;
+constexpr int NC = 128;        // state columns = TMEM lanes = MMA M
+constexpr int kPad = 8;
+constexpr uint32_t kTmemCols = 256;
+
+template <int DK>
+struct Layout {
+    static constexpr int LK = DK + kPad;
+    // TMEM columns (per CTA: 256 of the SM's 512)
+    static constexpr uint32_t COL_S = 0;          // S^T, fp32: DK columns (MMA 3 accumulator)
+    static constexpr uint32_t COL_D1 = DK;        // 2 x [U^T | O^T]: 2 x 32 fp32 columns
+    static constexpr uint32_t COL_AS = DK + 64;   // bf16 S^T (MMA A operand): DK/2 columns
+    static_assert(COL_AS + DK / 2 <= kTmemCols, "TMEM budget");
+    struct Work {                                 // cp.async targets, overwritten in place:
+        alignas(16) bf16 q[16 * LK];              //   q -> Qd
+        alignas(16) bf16 k[16 * LK];              //   k -> Kd
+        alignas(16) bf16 g[16 * LK];              //   g -> Ki
+    };
+    struct Stage {
+        alignas(16) bf16 b1[32 * DK];   // K-major [32][DK]: rows 0-15 = -W, 16-31 = Qd
+        alignas(16) bf16 b0[32 * 16];   // K-major [32][16]: rows 0-15 = Tb, 16-31 = 0
+        alignas(16) bf16 b2[DK * 16];   // K-major [DK][16]: Kb^T
+        alignas(16) bf16 b3[16 * 16];   // K-major [16][16]: P
+        alignas(16) bf16 v[NC * 16];    // MN-major [NC][16]: V^T as the A operand
+        alignas(16) float gam[DK];      // exp(G_C) per key channel
+    };
+    struct Prep {
+        alignas(16) float AT[16 * 16];  // AT[s][r] = beta_r A[r][s], r > s
+        float beta[16];
+        float rq[16], rk[16];
+    };
+    struct All {
+        Work work[kPrepWarps];
+        Stage st[kPrepWarps];
+        Prep pr[kPrepWarps];
+        alignas(16) bf16 au[NC * 16];   // K-major [NC][16]: U^T as the A operand
+        alignas(16) bf16 io[2][16 * NC];  // gate tile in, y tile out (row-major [16][NC])
+        alignas(8) unsigned long long mbar[2];
+        uint32_t tmem_base;
+    };
+    static constexpr size_t bytes = sizeof(All);
+};
+
+template <typename T>
+KDA_DEVICE T *at_bytes(T *base, uint32_t off) {
+    return reinterpret_cast<T *>(reinterpret_cast<unsigned char *>(base) + off);
+}
+
+// Runs tokens [t0, t0 + len) of head h (see the file comment).  OUT: produce
+// y.  USE_V: the write uses v (false: the transition part, U0 = 0).  The
+// state starts as the identity, a copy of s_init ([DK][NC] fp32) or zeros and
+// is written to s_out.  The fp32 state lives in tensor memory.
+template <int DK, bool OUT, bool USE_V>
+__device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const float *s_init,
+                          bool identity, float *s_out, unsigned char *smem_raw) {
+    using Lay = Layout<DK>;
+    constexpr int LK = Lay::LK;
+    typename Lay::All &sm = *reinterpret_cast<typename Lay::All *>(smem_raw);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int H = p.H;
+    const int nchunks = (len + 15) / 16;
+
+    // ---- set-up: TMEM columns and the two MMA-completion barriers
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(&sm.tmem_base)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (tid == 32) {
+        mbar_init(smem_u32(&sm.mbar[0]), 1);
+        mbar_init(smem_u32(&sm.mbar[1]), 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = sm.tmem_base;
+
+    if (warp < 4) {
+        // ------------------------------------------------------ state warpgroup
+        const int j = tid;
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const uint32_t t_s = tbase + lane_off + Lay::COL_S;
+        const uint32_t t_d1 = tbase + lane_off + Lay::COL_D1;
+        const uint32_t t_as = tbase + lane_off + Lay::COL_AS;
+        const uint32_t mb1 = smem_u32(&sm.mbar[0]), mb2 = smem_u32(&sm.mbar[1]);
+        constexpr int N1 = OUT ? 32 : 16;
+        constexpr uint32_t ID_U0 = idesc_bf16(128, N1, 1, 0);
+        constexpr uint32_t ID_WS = idesc_bf16(128, N1, 0, 0);
+        constexpr uint32_t ID_UK = idesc_bf16(128, DK, 0, 0);
+        constexpr uint32_t ID_UP = idesc_bf16(128, 16, 0, 0);
+        const bf16 *gate = (const bf16 *)p.gate;
+        bf16 *out = (bf16 *)p.out;
+
+        bool ok = true;
+        // gate of this thread's column for the chunk whose output is pending;
+        // loaded one chunk ahead so the loads are off the critical path
+        // gate tile of chunk c -> io[c & 1] (two 16-byte pieces per thread)
+        auto load_gate = [&](int c) {
+            const int rows = min(16, len - 16 * c);
+            bf16 *tile = sm.io[c & 1];
+#pragma unroll
+            for (int x2 = 0; x2 < 2; ++x2) {
+                const int x = tid + 128 * x2;
+                const int r = x >> 4, cc = x & 15;
+                const bool okr = gate && r < rows;
+                const size_t off = ((size_t)(okr ? t0 + 16 * c + r : t0) * H + h) * NC + cc * 8;
+                if (gate) {
+                    cp_async16(&tile[r * NC + cc * 8], gate + off, okr);
+                } else {
+                    const uint32_t one = pack_bf16(1.f, 1.f);
+                    *reinterpret_cast<uint4 *>(&tile[r * NC + cc * 8]) = make_uint4(one, one, one, one);
+                }
+            }
+            cp_async_commit();
+        };
+        // y = gate (.) O of chunk c: column j of the tile, in place
+        auto finish_chunk = [&](int c) {
+            const int stg = c % kPrepWarps;
+            if (OUT && ok) {
+                uint32_t o[16];
+                tmem_ld16_wait(t_d1 + 32 * (c & 1) + 16, o);
+                bf16 *tile = sm.io[c & 1];
+#pragma unroll
+                for (int t = 0; t < 16; ++t)
+                    tile[t * NC + j] = __float2bfloat16_rn(__bfloat162float(tile[t * NC + j]) * __uint_as_float(o[t]));
+            }
+            tc_fence_before();
+            bar_arrive(BAR_EMPTY + stg, kBarCount);
+        };
+        // the y tile of chunk c -> global (after a warpgroup barrier)
+        auto store_y = [&](int c) {
+            const int rows = min(16, len - 16 * c);
+            const bf16 *tile = sm.io[c & 1];
+#pragma unroll
+            for (int x2 = 0; x2 < 2; ++x2) {
+                const int x = tid + 128 * x2;
+                const int r = x >> 4, cc = x & 15;
+                if (r < rows)
+                    *reinterpret_cast<uint4 *>(out + ((size_t)(t0 + 16 * c + r) * H + h) * NC + cc * 8) =
+                        *reinterpret_cast<const uint4 *>(&tile[r * NC + cc * 8]);
+            }
+        };
+        // One pass over the fp32 state in TMEM (32 columns at a time): its
+        // bf16 copy becomes the A operand of the next chunk's MMA 2, and, when
+        // a next chunk exists, the state is pre-scaled by that chunk's
+        // exp(G_C) so that its MMA 3 can accumulate U^T Kb straight into it.
+        // src: nullptr = read the state from TMEM; else an initial state.
+        auto state_pass = [&](const float *gam_next, bool from_init) {
+#pragma unroll 1
+            for (int cb = 0; cb < DK / 32; ++cb) {
+                uint32_t d[32];
+                if (from_init) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int i = 32 * cb + e;
+                        d[e] = __float_as_uint(identity ? (i == j ? 1.f : 0.f)
+                                                        : (s_init ? s_init[(size_t)i * NC + j] : 0.f));
+                    }
+                } else {
+                    tmem_ld32_wait(t_s + 32 * cb, d);
+                }
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    pk[e] = pack_bf16(__uint_as_float(d[2 * e]), __uint_as_float(d[2 * e + 1]));
+                tmem_st16(t_as + 16 * cb, pk);
+                if (gam_next) {
+                    uint32_t lo[16], hi[16];
+#pragma unroll
+                    for (int e4 = 0; e4 < 8; ++e4) {
+                        const float4 gm = *reinterpret_cast<const float4 *>(&gam_next[32 * cb + 4 * e4]);
+                        const float2 a = f2mul(make_float2(__uint_as_float(d[4 * e4]), __uint_as_float(d[4 * e4 + 1])),
+                                               make_float2(gm.x, gm.y));
+                        const float2 b = f2mul(make_float2(__uint_as_float(d[4 * e4 + 2]), __uint_as_float(d[4 * e4 + 3])),
+                                               make_float2(gm.z, gm.w));
+                        uint32_t *dst = e4 < 4 ? lo : hi;
+                        const int o = (e4 & 3) * 4;
+                        dst[o + 0] = __float_as_uint(a.x);
+                        dst[o + 1] = __float_as_uint(a.y);
+                        dst[o + 2] = __float_as_uint(b.x);
+                        dst[o + 3] = __float_as_uint(b.y);
+                    }
+                    tmem_st16(t_s + 32 * cb, lo);
+                    tmem_st16(t_s + 32 * cb + 16, hi);
+                } else if (s_out) {  // after the last chunk: the final state
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) s_out[(size_t)(32 * cb + e) * NC + j] = __uint_as_float(d[e]);
+                }
+            }
+            tc_wait_st();
+            tc_fence_before();
+        };
+
+        if (nchunks == 0) {
+            if (s_out) {
+#pragma unroll 4
+                for (int i = 0; i < DK; ++i)
+                    s_out[(size_t)i * NC + j] = identity ? (i == j ? 1.f : 0.f)
+                                                         : (s_init ? s_init[(size_t)i * NC + j] : 0.f);
+            }
+        } else {
+            bar_sync(BAR_FULL + 0, kBarCount);  // stage of chunk 0: its exp(G_C)
+            state_pass(sm.st[0].gam, true);
+        }
+        // MMA operand descriptors of stage 0; stages are contiguous, so stage s
+        // adds s * sizeof(Stage) / 16 to the start-address field (all of shared
+        // memory is below 256 KB: the 14-bit field never carries)
+        const uint64_t dsc_v0 = sdesc(smem_u32(sm.st[0].v), 128, 256);
+        const uint64_t dsc_b00 = sdesc(smem_u32(sm.st[0].b0), 128, 256);
+        const uint64_t dsc_b10 = sdesc(smem_u32(sm.st[0].b1), 128, DK * 16);
+        const uint64_t dsc_b20 = sdesc(smem_u32(sm.st[0].b2), 128, 256);
+        const uint64_t dsc_b30 = sdesc(smem_u32(sm.st[0].b3), 128, 256);
+        const uint64_t dsc_au = sdesc(smem_u32(sm.au), 128, 256);
+        constexpr uint64_t kStageStep = sizeof(typename Lay::Stage) / 16;
+        static_assert(sizeof(typename Lay::Stage) % 16 == 0, "stage stride");
+
+        // Per chunk c:  [gate(c) -> io]  MMA 1/2 (c)  |  y(c-1) = gate (.) O
+        //               U -> smem  MMA 3/4 (c)  |  y(c-1) -> global
+        //               next stage; state pass
+        for (int c = 0; c < nchunks; ++c) {
+            const int stg = c % kPrepWarps;
+            const uint32_t d1_col = Lay::COL_D1 + 32 * (c & 1);
+            KDA_MARK(tid == 0 && c < 128, c * 16 + 0);
+            if (OUT) cp_async_wait<0>();  // this thread's pieces of the gate tile of chunk c - 1
+            bar_sync(BAR_WG, 128);        // state-pass TMEM stores; gate tile; y(c - 2) stored
+            if (OUT) load_gate(c);
+            KDA_MARK(tid == 0 && c < 128, c * 16 + 1);
+            if (tid == 0 && ok) {  // U0^T and [-W | Qd] S^T: needs only the bf16 copy
+                tc_fence_after();
+                const uint32_t d1 = tbase + d1_col;
+                const uint64_t so = kStageStep * stg;
+                if (USE_V) tc_mma_ss(d1, dsc_v0 + so, dsc_b00 + so, ID_U0, 0);
+#pragma unroll
+                for (int kk = 0; kk < DK / 16; ++kk)  // +256 bytes of K = +16 in the start field
+                    tc_mma_ts(d1, tbase + Lay::COL_AS + 8 * kk, dsc_b10 + so + 16 * kk, ID_WS,
+                              (USE_V || kk > 0) ? 1u : 0u);
+                tc_commit(mb1);
+            }
+            __syncwarp();  // reconverge warp 0 before the aligned TMEM loads below
+            KDA_MARK(tid == 0 && c < 128, c * 16 + 2);
+            if (c > 0) finish_chunk(c - 1);
+            KDA_MARK(tid == 0 && c < 128, c * 16 + 5);
+            if (ok) ok = mbar_wait(mb1, c & 1);
+            ok = __all_sync(0xffffffffu, ok);
+            tc_fence_after();
+            KDA_MARK(tid == 0 && c < 128, c * 16 + 6);
+            if (ok) {  // U^T row j -> bf16 A operand in shared memory
+                uint32_t u[16];
+                tmem_ld16_wait(t_d1 + 32 * (c & 1), u);
+                uint32_t pk[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    pk[e] = pack_bf16(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1]));
+                *reinterpret_cast<uint4 *>(at_bytes(sm.au, kmaj(j, 0, 16))) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                *reinterpret_cast<uint4 *>(at_bytes(sm.au, kmaj(j, 8, 16))) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            }
+            fence_async_smem();
+            tc_fence_before();
+            KDA_MARK(tid == 0 && c < 128, c * 16 + 7);
+            bar_sync(BAR_WG, 128);
+            if (tid == 0 && ok) {  // S^T += U^T Kb (into the state itself);  O^T += U^T P^T
+                tc_fence_after();
+                const uint64_t so = kStageStep * stg;
+                tc_mma_ss(tbase + Lay::COL_S, dsc_au, dsc_b20 + so, ID_UK, 1);
+                if (OUT) tc_mma_ss(tbase + d1_col + 16, dsc_au, dsc_b30 + so, ID_UP, 1);
+                tc_commit(mb2);
+            }
+            __syncwarp();  // reconverge warp 0 before the aligned barrier below
+            const bool has_next = c + 1 < nchunks;
+            if (OUT && c > 0) store_y(c - 1);
+            KDA_MARK(tid == 0 && c < 128, c * 16 + 8);
+            if (has_next) bar_sync(BAR_FULL + (c + 1) % kPrepWarps, kBarCount);
+            KDA_MARK(tid == 0 && c < 128, c * 16 + 9);
+            if (ok) ok = mbar_wait(mb2, c & 1);
+            ok = __all_sync(0xffffffffu, ok);
+            tc_fence_after();
+            KDA_MARK(tid == 0 && c < 128, c * 16 + 10);
+            if (ok) {
+                state_pass(has_next ? sm.st[(c + 1) % kPrepWarps].gam : nullptr, false);
+            } else {
+                tc_fence_before();
+            }
+            KDA_MARK(tid == 0 && c < 128, c * 16 + 11);
+        }
+        if (nchunks > 0) {
+            if (OUT) cp_async_wait<0>();
+            bar_sync(BAR_WG, 128);
+            finish_chunk(nchunks - 1);
+            if (OUT) {
+                bar_sync(BAR_WG, 128);
+                store_y(nchunks - 1);
+            }
+        }
+        if (!ok && lane == 0 && p.err) atomicOr(p.err, 1);
+    } else {
+        // ----------------------------------------------------------- prep warps
+        const int pw = warp - 4;
+        const bf16 *q = (const bf16 *)p.q, *k = (const bf16 *)p.k, *g = (const bf16 *)p.g;
+        const bf16 *v = (const bf16 *)p.v, *beta = (const bf16 *)p.beta;
+        typename Lay::Prep &pr = sm.pr[pw];
+        typename Lay::Work &Wk = sm.work[pw];
+        typename Lay::Stage &St = sm.st[pw];
+        float beta_next = 0.f;
+
+        // rows 16-31 of the [Tb^T | 0] operand stay zero
+        reinterpret_cast<uint4 *>(at_bytes(St.b0, kmaj(16, 0, 16)))[lane] = make_uint4(0, 0, 0, 0);
+
+        auto issue_raw = [&](int c) {
+            const int tc = t0 + 16 * c;
+            const int rows = min(16, len - 16 * c);
+            constexpr int PK = DK / 8;
+#pragma unroll 4
+            for (int x = lane; x < 16 * PK; x += 32) {
+                const int r = x / PK, cc = x % PK;
+                const bool okr = r < rows;
+                const size_t off = ((size_t)(okr ? tc + r : t0) * H + h) * DK + cc * 8;
+                cp_async16(&Wk.k[r * LK + cc * 8], k + off, okr);
+                cp_async16(&Wk.g[r * LK + cc * 8], g + off, okr);
+                if (OUT) cp_async16(&Wk.q[r * LK + cc * 8], q + off, okr);
+            }
+            cp_async_commit();
+            beta_next = lane < rows ? __bfloat162float(beta[(size_t)(tc + lane) * H + h]) : 0.f;
+        };
+        auto issue_v = [&](int c) {
+            if (USE_V) {
+                const int tc = t0 + 16 * c;
+                const int rows = min(16, len - 16 * c);
+                constexpr int PV = NC / 8;
+#pragma unroll 4
+                for (int x = lane; x < 16 * PV; x += 32) {
+                    const int r = x / PV, cc = x % PV;
+                    const bool okr = r < rows;
+                    const size_t off = ((size_t)(okr ? tc + r : t0) * H + h) * NC + cc * 8;
+                    cp_async16(at_bytes(St.v, mnmaj(cc * 8, r, 16)), v + off, okr);
+                }
+            }
+            cp_async_commit();
+        };
+
+        if (pw < nchunks) issue_raw(pw);
+        for (int c = pw; c < nchunks; c += kPrepWarps) {
+            KDA_MARK(lane == 0 && c < 128, 2048 + c * 8 + 0);
+            if (c >= kPrepWarps) bar_sync(BAR_EMPTY + pw, kBarCount);  // stage free again
+            KDA_MARK(lane == 0 && c < 128, 2048 + c * 8 + 1);
+            issue_v(c);
+            if (lane < 16) pr.beta[lane] = beta_next;
+            cp_async_wait<1>();  // q, k, g of chunk c
+            __syncwarp();
+            KDA_MARK(lane == 0 && c < 128, 2048 + c * 8 + 2);
+
+            if (p.qk_l2norm) {
+                for (int r = 0; r < 16; ++r) {
+                    float kk = 0.f, qq = 0.f;
+                    for (int i = lane; i < DK; i += 32) {
+                        const float kv = __bfloat162float(Wk.k[r * LK + i]);
+                        kk += kv * kv;
+                        if (OUT) {
+                            const float qv = __bfloat162float(Wk.q[r * LK + i]);
+                            qq += qv * qv;
+                        }
+                    }
+                    kk = warp_sum(kk);
+                    qq = warp_sum(qq);
+                    if (lane == r) {
+                        pr.rk[r] = rsqrtf(kk + 1e-6f);
+                        pr.rq[r] = rsqrtf(qq + 1e-6f);
+                    }
+                }
+                __syncwarp();
+            }
+
+            // 1. decay factors and decayed operands (in place: k -> Kd,
+            //    g -> Ki, q -> Qd); lane owns channel pairs (2 lane, 2 lane + 1)
+#pragma unroll 1
+            for (int cp2 = 0; cp2 < DK / 64; ++cp2) {
+                const int i = 64 * cp2 + 2 * lane;
+                float2 e[16], E[16];
+#pragma unroll
+                for (int r = 0; r < 16; ++r) {
+                    const float2 gg = unpack_bf16(*reinterpret_cast<const uint32_t *>(&Wk.g[r * LK + i]));
+                    e[r] = make_float2(__expf(gg.x), __expf(gg.y));
+                }
+                float2 acc = make_float2(1.f, 1.f);
+#pragma unroll
+                for (int r = 0; r < 16; ++r) {
+                    acc = f2mul(acc, e[r]);
+                    E[r] = acc;
+                }
+                const float2 El = acc;
+                const float2 invEl = make_float2(1.f / El.x, 1.f / El.y);
+                *reinterpret_cast<float2 *>(&St.gam[i]) = El;
+                float2 F = make_float2(1.f, 1.f);  // exp(G_C - G_r): suffix products
+                uint32_t kb0[8], kb1[8];           // Kb^T rows i, i+1 (token pairs)
+                float2 kb_hi = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int r = 15; r >= 0; --r) {
+                    float2 kv = unpack_bf16(*reinterpret_cast<const uint32_t *>(&Wk.k[r * LK + i]));
+                    if (p.qk_l2norm) kv = f2mul(kv, make_float2(pr.rk[r], pr.rk[r]));
+                    *reinterpret_cast<uint32_t *>(&Wk.k[r * LK + i]) = pack_bf16(f2mul(kv, E[r]));
+                    *reinterpret_cast<uint32_t *>(&Wk.g[r * LK + i]) = pack_bf16(f2mul(kv, f2mul(F, invEl)));
+                    const float2 kbv = f2mul(kv, F);
+                    if (r & 1) {
+                        kb_hi = kbv;
+                    } else {
+                        kb0[r >> 1] = pack_bf16(kbv.x, kb_hi.x);
+                        kb1[r >> 1] = pack_bf16(kbv.y, kb_hi.y);
+                    }
+                    if (OUT) {
+                        const float2 qv = unpack_bf16(*reinterpret_cast<const uint32_t *>(&Wk.q[r * LK + i]));
+                        float sc = p.scale;
+                        if (p.qk_l2norm) sc *= pr.rq[r];
+                        *reinterpret_cast<uint32_t *>(&Wk.q[r * LK + i]) =
+                            pack_bf16(f2mul(f2mul(qv, make_float2(sc, sc)), E[r]));
+                    }
+                    F = f2mul(F, e[r]);
+                }
+                *reinterpret_cast<uint4 *>(at_bytes(St.b2, kmaj(i, 0, 16))) = make_uint4(kb0[0], kb0[1], kb0[2], kb0[3]);
+                *reinterpret_cast<uint4 *>(at_bytes(St.b2, kmaj(i, 8, 16))) = make_uint4(kb0[4], kb0[5], kb0[6], kb0[7]);
+                *reinterpret_cast<uint4 *>(at_bytes(St.b2, kmaj(i + 1, 0, 16))) = make_uint4(kb1[0], kb1[1], kb1[2], kb1[3]);
+                *reinterpret_cast<uint4 *>(at_bytes(St.b2, kmaj(i + 1, 8, 16))) = make_uint4(kb1[4], kb1[5], kb1[6], kb1[7]);
+            }
+            __syncwarp();
+            KDA_MARK(lane == 0 && c < 128, 2048 + c * 8 + 3);
+            const bf16 *Kd = Wk.k, *Ki = Wk.g, *Qd = Wk.q;
+
+            if (OUT) {  // Qd -> rows 16-31 of the [-W | Qd] operand (canonical layout)
+#pragma unroll
+                for (int it = 0; it < DK / 16; ++it) {
+                    const int x = lane + 32 * it;
+                    const int r = x & 15, kc = x >> 4;
+                    *reinterpret_cast<uint4 *>(at_bytes(St.b1, kmaj(16 + r, 8 * kc, DK))) =
+                        *reinterpret_cast<const uint4 *>(&Qd[r * LK + 8 * kc]);
+                }
+            }
+
+            // 2. A = Kd Ki^T (strictly lower) and P = Qd Ki^T (lower)
+#pragma unroll
+            for (int which = 0; which < (OUT ? 2 : 1); ++which) {
+                const bf16 *Aop = which == 0 ? Kd : Qd;
+                float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int kk = 0; kk < DK / 16; ++kk) {
+                    uint32_t a[4], b[4];
+                    ldsm4(a, &Aop[((lane & 7) + ((lane >> 3) & 1) * 8) * LK + 16 * kk + (lane >> 4) * 8]);
+                    ldsm4(b, &Ki[((lane & 7) + (lane >> 4) * 8) * LK + 16 * kk + ((lane >> 3) & 1) * 8]);
+                    mma16816(acc0, a, b[0], b[1]);
+                    mma16816(acc1, a, b[2], b[3]);
+                }
+                const int r0 = lane >> 2, c0 = 2 * (lane & 3);
+                if (which == 0) {
+                    // AT[s][r] = beta_r A[r][s] for s < r (the solve's column sweeps)
+                    const float vals[8] = {acc0[0], acc0[1], acc0[2], acc0[3],
+                                           acc1[0], acc1[1], acc1[2], acc1[3]};
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int r = r0 + ((e & 2) ? 8 : 0);
+                        const int sc = c0 + (e & 1) + ((e & 4) ? 8 : 0);
+                        pr.AT[sc * 16 + r] = sc < r ? pr.beta[r] * vals[e] : 0.f;
+                    }
+                } else {
+                    auto pv = [&](float x, int r, int sc) { return sc <= r ? x : 0.f; };
+                    *reinterpret_cast<uint32_t *>(at_bytes(St.b3, kmaj(r0, c0, 16))) =
+                        pack_bf16(pv(acc0[0], r0, c0), pv(acc0[1], r0, c0 + 1));
+                    *reinterpret_cast<uint32_t *>(at_bytes(St.b3, kmaj(r0 + 8, c0, 16))) =
+                        pack_bf16(pv(acc0[2], r0 + 8, c0), pv(acc0[3], r0 + 8, c0 + 1));
+                    *reinterpret_cast<uint32_t *>(at_bytes(St.b3, kmaj(r0, c0 + 8, 16))) =
+                        pack_bf16(pv(acc1[0], r0, c0 + 8), pv(acc1[1], r0, c0 + 9));
+                    *reinterpret_cast<uint32_t *>(at_bytes(St.b3, kmaj(r0 + 8, c0 + 8, 16))) =
+                        pack_bf16(pv(acc1[2], r0 + 8, c0 + 8), pv(acc1[3], r0 + 8, c0 + 9));
+                }
+            }
+            __syncwarp();
+
+            KDA_MARK(lane == 0 && c < 128, 2048 + c * 8 + 4);
+            // 3. Tb = (I + Diag(beta) A)^-1 Diag(beta); lane j < 16 owns column j.
+            //    After row r is final it is pushed into every later row.
+            if (lane < 16) {
+                const int jj = lane;
+                float col[16];
+#pragma unroll
+                for (int r = 0; r < 16; ++r) col[r] = (r == jj) ? 1.f : 0.f;
+#pragma unroll
+                for (int r = 0; r < 15; ++r) {
+                    float at[16];
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const float4 a4 = *reinterpret_cast<const float4 *>(&pr.AT[r * 16 + 4 * q4]);
+                        at[4 * q4 + 0] = a4.x; at[4 * q4 + 1] = a4.y;
+                        at[4 * q4 + 2] = a4.z; at[4 * q4 + 3] = a4.w;
+                    }
+#pragma unroll
+                    for (int r2 = r + 1; r2 < 16; ++r2) col[r2] = fmaf(-at[r2], col[r], col[r2]);
+                }
+                const float bj = pr.beta[jj];
+#pragma unroll
+                for (int r = 0; r < 16; ++r)
+                    *at_bytes(St.b0, kmaj(r, jj, 16)) = __float2bfloat16_rn(col[r] * bj);
+            }
+            __syncwarp();
+
+            KDA_MARK(lane == 0 && c < 128, 2048 + c * 8 + 5);
+            // 4. W = Tb Kd -> rows 0-15 of the [-W | Qd] operand hold -W
+            {
+                uint32_t a[4];
+                ldsm4(a, at_bytes(St.b0, kmaj((lane & 7) + ((lane >> 3) & 1) * 8, (lane >> 4) * 8, 16)));
+#pragma unroll
+                for (int np = 0; np < DK / 16; ++np) {
+                    const int n0 = 16 * np;
+                    uint32_t b[4];
+                    ldsm4t(b, &Kd[((lane & 7) + ((lane >> 3) & 1) * 8) * LK + n0 + (lane >> 4) * 8]);
+                    float w0[4] = {0.f, 0.f, 0.f, 0.f}, w1[4] = {0.f, 0.f, 0.f, 0.f};
+                    mma16816(w0, a, b[0], b[1]);
+                    mma16816(w1, a, b[2], b[3]);
+                    const int r = lane >> 2, cc = n0 + 2 * (lane & 3);
+                    *reinterpret_cast<uint32_t *>(at_bytes(St.b1, kmaj(r, cc, DK))) = pack_bf16(-w0[0], -w0[1]);
+                    *reinterpret_cast<uint32_t *>(at_bytes(St.b1, kmaj(r + 8, cc, DK))) = pack_bf16(-w0[2], -w0[3]);
+                    *reinterpret_cast<uint32_t *>(at_bytes(St.b1, kmaj(r, cc + 8, DK))) = pack_bf16(-w1[0], -w1[1]);
+                    *reinterpret_cast<uint32_t *>(at_bytes(St.b1, kmaj(r + 8, cc + 8, DK))) = pack_bf16(-w1[2], -w1[3]);
+                }
+            }
+            __syncwarp();
+            KDA_MARK(lane == 0 && c < 128, 2048 + c * 8 + 6);
+            // the work buffers are free: prefetch this warp's next chunk
+            const bool more = c + kPrepWarps < nchunks;
+            if (more) issue_raw(c + kPrepWarps);
+            if (more) cp_async_wait<1>(); else cp_async_wait<0>();  // v of chunk c
+            // generic-proxy writes of the stage must be visible to the tensor core
+            fence_async_smem();
+            __syncwarp();
+            KDA_MARK(lane == 0 && c < 128, 2048 + c * 8 + 7);
+            bar_arrive(BAR_FULL + pw, kBarCount);
+        }
+        if (pw < nchunks) bar_sync(BAR_EMPTY + pw, kBarCount);
+    }
+
+    // ---- tear-down: every TMEM access of the CTA is complete
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "r"(kTmemCols)
+                     : "memory");
+}
+
+template <int DK>
+__global__ void __launch_bounds__(kThreads, kBlocksPerSM) summary_kernel(PrefillParams p) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int4 pc = p.pieces[blockIdx.x];
+    if (pc.x < 0) return;
+    const int n = pc.x, j = pc.w, h = blockIdx.y;
+    const int np = p.seq_first[n + 1] - p.seq_first[n];
+    if (j >= np - 1) return;
+    const size_t ph = (size_t)blockIdx.x * p.H + h;
+    if (blockIdx.z == 0) {
+        const float *init = (j == 0 && p.initial_state)
+                                ? p.initial_state + ((size_t)n * p.H + h) * DK * NC
+                                : nullptr;
+        run_piece<DK, false, true>(p, pc.y, pc.z, h, init, false, p.Szero + ph * DK * NC, smem);
+    } else {
+        if (j == 0) return;
+        run_piece<DK, false, false>(p, pc.y, pc.z, h, nullptr, true, p.M + ph * DK * DK, smem);
+    }
+}
+
+template <int DK>
+__global__ void __launch_bounds__(kThreads, kBlocksPerSM) output_kernel(PrefillParams p) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int4 pc = p.pieces[blockIdx.x];
+    if (pc.x < 0) return;
+    const int n = pc.x, j = pc.w, h = blockIdx.y;
+    const int np = p.seq_first[n + 1] - p.seq_first[n];
+    const size_t nh = (size_t)n * p.H + h;
+    const float *init = (np == 1) ? (p.initial_state ? p.initial_state + nh * DK * NC : nullptr)
+                                  : p.Sin + ((size_t)blockIdx.x * p.H + h) * DK * NC;
+    float *fin = (j == np - 1 && p.final_state) ? p.final_state + nh * DK * NC : nullptr;
+    run_piece<DK, true, true>(p, pc.y, pc.z, h, init, false, fin, smem);
+}
+
+}  // namespace tc5
+
+// dk = dv = 128 only (one state column per TMEM lane; the transition part has
+// dk columns too).
+cudaError_t launch_prefill_tc5(const PrefillParams &p, bool summaries, cudaStream_t st) {
+    const size_t sm = tc5::Layout<128>::bytes;
+    cudaError_t e;
+    if (summaries) {
+        e = cudaFuncSetAttribute(tc5::summary_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)sm);
+        if (e != cudaSuccess) return e;
+        tc5::summary_kernel<128><<<dim3(p.P_max, p.H, 2), tc5::kThreads, sm, st>>>(p);
+        return cudaGetLastError();
+    }
+    e = cudaFuncSetAttribute(tc5::output_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sm);
+    if (e != cudaSuccess) return e;
+    tc5::output_kernel<128><<<dim3(p.P_max, p.H, 1), tc5::kThreads, sm, st>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace kda

@@ -161,3 +161,19 @@ def test_decay_at_the_floor_stays_finite(cuda_lib, monkeypatch, dtype):
     y, S = run(inp)
     yr, Sr = oracle_prefill(inp)
     compare(inp, y, S, yr, Sr, dtype, what="floor")
+
+
+def test_device_error_word_stays_clear(cuda_lib, monkeypatch):
+    """Bounded device waits record a failure in the workspace header (int32 at
+    byte 8); a normal call leaves it zero."""
+    monkeypatch.setenv("KDA_PIECE_LEN", "256")
+    w = W.custom(dtype="bf16", H=2, dk=128, dv=128, lengths=(700, 33), init_state=True, seed=12)
+    inp = W.pack_prefill(w, device="cuda")
+    T, H = inp["q"].shape[:2]
+    ws = torch.full((kda.workspace_size(T, 2, H, 128, 128),), 0x7F, dtype=torch.uint8,
+                    device="cuda")
+    kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["gate"],
+                  inp["cu_seqlens"], initial_state=inp["initial_state"], workspace=ws)
+    torch.cuda.synchronize()
+    header = ws[:16].view(torch.int32).cpu().tolist()
+    assert header[2] == 0 and header[1] == 0 and header[0] > 2
