@@ -499,13 +499,16 @@ __device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const 
 template <int DK, int DV>
 __global__ void __launch_bounds__(kThreads, 1) summary_kernel(PrefillParams p) {
     extern __shared__ __align__(128) unsigned char smem[];
-    const int4 pc = p.pieces[blockIdx.x];
+    // (piece, head) pairs with the head fastest: co-resident CTAs cover all
+    // heads of a few pieces, spreading their rows over every memory channel
+    const int h = blockIdx.x % p.H, pi = blockIdx.x / p.H;
+    const int4 pc = p.pieces[pi];
     if (pc.x < 0) return;
-    const int n = pc.x, j = pc.w, h = blockIdx.y;
+    const int n = pc.x, j = pc.w;
     const int np = p.seq_first[n + 1] - p.seq_first[n];
     if (j >= np - 1) return;
-    const size_t ph = (size_t)blockIdx.x * p.H + h;
-    if (blockIdx.z == 0) {
+    const size_t ph = (size_t)pi * p.H + h;
+    if (blockIdx.y == 0) {
         const float *init = (j == 0 && p.initial_state)
                                 ? p.initial_state + ((size_t)n * p.H + h) * DK * DV
                                 : nullptr;
@@ -519,13 +522,16 @@ __global__ void __launch_bounds__(kThreads, 1) summary_kernel(PrefillParams p) {
 template <int DK, int DV>
 __global__ void __launch_bounds__(kThreads, 1) output_kernel(PrefillParams p) {
     extern __shared__ __align__(128) unsigned char smem[];
-    const int4 pc = p.pieces[blockIdx.x];
+    // (piece, head) pairs with the head fastest: co-resident CTAs cover all
+    // heads of a few pieces, spreading their rows over every memory channel
+    const int h = blockIdx.x % p.H, pi = blockIdx.x / p.H;
+    const int4 pc = p.pieces[pi];
     if (pc.x < 0) return;
-    const int n = pc.x, j = pc.w, h = blockIdx.y;
+    const int n = pc.x, j = pc.w;
     const int np = p.seq_first[n + 1] - p.seq_first[n];
     const size_t nh = (size_t)n * p.H + h;
     const float *init = (np == 1) ? (p.initial_state ? p.initial_state + nh * DK * DV : nullptr)
-                                  : p.Sin + ((size_t)blockIdx.x * p.H + h) * DK * DV;
+                                  : p.Sin + ((size_t)pi * p.H + h) * DK * DV;
     float *fin = (j == np - 1 && p.final_state) ? p.final_state + nh * DK * DV : nullptr;
     run_piece<DK, DV, true, true>(p, pc.y, pc.z, h, init, false, fin, smem);
 }
@@ -539,14 +545,14 @@ static cudaError_t launch_t(const PrefillParams &p, bool summaries, cudaStream_t
         e = cudaFuncSetAttribute(summary_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)sm);
         if (e != cudaSuccess) return e;
-        summary_kernel<DK, DV><<<dim3(p.P_max, p.H, 2), kThreads, sm, st>>>(p);
+        summary_kernel<DK, DV><<<dim3((unsigned)(p.P_max * p.H), 2), kThreads, sm, st>>>(p);
         return cudaGetLastError();
     }
     const size_t sm = Layout<DK, DV>::bytes;
     e = cudaFuncSetAttribute(output_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)sm);
     if (e != cudaSuccess) return e;
-    output_kernel<DK, DV><<<dim3(p.P_max, p.H, 1), kThreads, sm, st>>>(p);
+    output_kernel<DK, DV><<<dim3((unsigned)(p.P_max * p.H)), kThreads, sm, st>>>(p);
     return cudaGetLastError();
 }
 

@@ -220,13 +220,16 @@ __device__ void simt_piece(const PrefillParams &p, int t0, int len, int h, const
 template <int DK, int DV, typename T>
 __global__ void __launch_bounds__(256) simt_summary_kernel(PrefillParams p) {
     extern __shared__ float smem[];
-    const int4 pc = p.pieces[blockIdx.x];
+    // (piece, head) pairs with the head fastest: co-resident CTAs cover all
+    // heads of a few pieces, spreading their rows over every memory channel
+    const int h = blockIdx.x % p.H, pi = blockIdx.x / p.H;
+    const int4 pc = p.pieces[pi];
     if (pc.x < 0) return;
-    const int n = pc.x, j = pc.w, h = blockIdx.y;
+    const int n = pc.x, j = pc.w;
     const int np = p.seq_first[n + 1] - p.seq_first[n];
     if (j >= np - 1) return;
-    const size_t ph = (size_t)blockIdx.x * p.H + h;
-    if (blockIdx.z == 0) {
+    const size_t ph = (size_t)pi * p.H + h;
+    if (blockIdx.y == 0) {
         const float *init = (j == 0 && p.initial_state)
                                 ? p.initial_state + ((size_t)n * p.H + h) * DK * DV
                                 : nullptr;
@@ -242,13 +245,16 @@ __global__ void __launch_bounds__(256) simt_summary_kernel(PrefillParams p) {
 template <int DK, int DV, typename T>
 __global__ void __launch_bounds__(256) simt_output_kernel(PrefillParams p) {
     extern __shared__ float smem[];
-    const int4 pc = p.pieces[blockIdx.x];
+    // (piece, head) pairs with the head fastest: co-resident CTAs cover all
+    // heads of a few pieces, spreading their rows over every memory channel
+    const int h = blockIdx.x % p.H, pi = blockIdx.x / p.H;
+    const int4 pc = p.pieces[pi];
     if (pc.x < 0) return;
-    const int n = pc.x, j = pc.w, h = blockIdx.y;
+    const int n = pc.x, j = pc.w;
     const int np = p.seq_first[n + 1] - p.seq_first[n];
     const size_t nh = (size_t)n * p.H + h;
     const float *init = (np == 1) ? (p.initial_state ? p.initial_state + nh * DK * DV : nullptr)
-                                  : p.Sin + ((size_t)blockIdx.x * p.H + h) * DK * DV;
+                                  : p.Sin + ((size_t)pi * p.H + h) * DK * DV;
     float *fin = (j == np - 1 && p.final_state) ? p.final_state + nh * DK * DV : nullptr;
     simt_piece<DK, DV, true, true, T>(p, pc.y, pc.z, h, init, false, fin, smem);
 }
@@ -262,13 +268,13 @@ static cudaError_t launch_simt_t(const PrefillParams &p, bool summaries, cudaStr
         e = cudaFuncSetAttribute(simt_summary_kernel<DK, DV, T>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_sum);
         if (e != cudaSuccess) return e;
-        simt_summary_kernel<DK, DV, T><<<dim3(p.P_max, p.H, 2), 256, sm_sum, st>>>(p);
+        simt_summary_kernel<DK, DV, T><<<dim3((unsigned)(p.P_max * p.H), 2), 256, sm_sum, st>>>(p);
         return cudaGetLastError();
     }
     e = cudaFuncSetAttribute(simt_output_kernel<DK, DV, T>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_out);
     if (e != cudaSuccess) return e;
-    simt_output_kernel<DK, DV, T><<<dim3(p.P_max, p.H, 1), 256, sm_out, st>>>(p);
+    simt_output_kernel<DK, DV, T><<<dim3((unsigned)(p.P_max * p.H)), 256, sm_out, st>>>(p);
     return cudaGetLastError();
 }
 

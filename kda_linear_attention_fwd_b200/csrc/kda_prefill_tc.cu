@@ -45,7 +45,7 @@
 __device__ unsigned long long g_kda_tc5_trace[8192];
 #define KDA_MARK(cond, slot)                                                          \
     do {                                                                              \
-        if ((cond) && blockIdx.x == 1 && blockIdx.y == 0 && blockIdx.z == 0 &&        \
+        if ((cond) && blockIdx.x == 1 && blockIdx.y == 0 &&        \
             (slot) < 8192)                                                            \
             g_kda_tc5_trace[(slot)] = clock64();                                      \
         __syncwarp();                                                                 \
@@ -189,7 +189,6 @@ __device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const 
         };
         // y = gate (.) O of chunk c: column j of the tile, in place
         auto finish_chunk = [&](int c) {
-            const int stg = c % kPrepWarps;
             if (OUT && ok) {
                 uint32_t o[16];
                 tmem_ld16_wait(t_d1 + 32 * (c & 1) + 16, o);
@@ -198,8 +197,6 @@ __device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const 
                 for (int t = 0; t < 16; ++t)
                     tile[t * NC + j] = __float2bfloat16_rn(__bfloat162float(tile[t * NC + j]) * __uint_as_float(o[t]));
             }
-            tc_fence_before();
-            bar_arrive(BAR_EMPTY + stg, kBarCount);
         };
         // the y tile of chunk c -> global (after a warpgroup barrier)
         auto store_y = [&](int c) {
@@ -348,6 +345,8 @@ __device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const 
             if (ok) ok = mbar_wait(mb2, c & 1);
             ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
+            tc_fence_before();
+            bar_arrive(BAR_EMPTY + stg, kBarCount);  // every reader of this stage is done
             KDA_MARK(tid == 0 && c < 128, c * 16 + 10);
             if (ok) {
                 state_pass(has_next ? sm.st[(c + 1) % kPrepWarps].gam : nullptr, false);
@@ -594,15 +593,14 @@ __device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const 
             }
             __syncwarp();
             KDA_MARK(lane == 0 && c < 128, 2048 + c * 8 + 6);
-            // the work buffers are free: prefetch this warp's next chunk
-            const bool more = c + kPrepWarps < nchunks;
-            if (more) issue_raw(c + kPrepWarps);
-            if (more) cp_async_wait<1>(); else cp_async_wait<0>();  // v of chunk c
+            cp_async_wait<0>();  // v of chunk c (the only group in flight)
             // generic-proxy writes of the stage must be visible to the tensor core
             fence_async_smem();
             __syncwarp();
             KDA_MARK(lane == 0 && c < 128, 2048 + c * 8 + 7);
             bar_arrive(BAR_FULL + pw, kBarCount);
+            // the work buffers are free: fetch this warp's next chunk
+            if (c + kPrepWarps < nchunks) issue_raw(c + kPrepWarps);
         }
         if (pw < nchunks) bar_sync(BAR_EMPTY + pw, kBarCount);
     }
@@ -619,13 +617,16 @@ __device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const 
 template <int DK>
 __global__ void __launch_bounds__(kThreads, kBlocksPerSM) summary_kernel(PrefillParams p) {
     extern __shared__ __align__(128) unsigned char smem[];
-    const int4 pc = p.pieces[blockIdx.x];
+    // (piece, head) pairs with the head fastest: co-resident CTAs cover all
+    // heads of a few pieces, spreading their rows over every memory channel
+    const int h = blockIdx.x % p.H, pi = blockIdx.x / p.H;
+    const int4 pc = p.pieces[pi];
     if (pc.x < 0) return;
-    const int n = pc.x, j = pc.w, h = blockIdx.y;
+    const int n = pc.x, j = pc.w;
     const int np = p.seq_first[n + 1] - p.seq_first[n];
     if (j >= np - 1) return;
-    const size_t ph = (size_t)blockIdx.x * p.H + h;
-    if (blockIdx.z == 0) {
+    const size_t ph = (size_t)pi * p.H + h;
+    if (blockIdx.y == 0) {
         const float *init = (j == 0 && p.initial_state)
                                 ? p.initial_state + ((size_t)n * p.H + h) * DK * NC
                                 : nullptr;
@@ -639,13 +640,16 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSM) summary_kernel(Prefill
 template <int DK>
 __global__ void __launch_bounds__(kThreads, kBlocksPerSM) output_kernel(PrefillParams p) {
     extern __shared__ __align__(128) unsigned char smem[];
-    const int4 pc = p.pieces[blockIdx.x];
+    // (piece, head) pairs with the head fastest: co-resident CTAs cover all
+    // heads of a few pieces, spreading their rows over every memory channel
+    const int h = blockIdx.x % p.H, pi = blockIdx.x / p.H;
+    const int4 pc = p.pieces[pi];
     if (pc.x < 0) return;
-    const int n = pc.x, j = pc.w, h = blockIdx.y;
+    const int n = pc.x, j = pc.w;
     const int np = p.seq_first[n + 1] - p.seq_first[n];
     const size_t nh = (size_t)n * p.H + h;
     const float *init = (np == 1) ? (p.initial_state ? p.initial_state + nh * DK * NC : nullptr)
-                                  : p.Sin + ((size_t)blockIdx.x * p.H + h) * DK * NC;
+                                  : p.Sin + ((size_t)pi * p.H + h) * DK * NC;
     float *fin = (j == np - 1 && p.final_state) ? p.final_state + nh * DK * NC : nullptr;
     run_piece<DK, true, true>(p, pc.y, pc.z, h, init, false, fin, smem);
 }
@@ -661,13 +665,13 @@ cudaError_t launch_prefill_tc5(const PrefillParams &p, bool summaries, cudaStrea
         e = cudaFuncSetAttribute(tc5::summary_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)sm);
         if (e != cudaSuccess) return e;
-        tc5::summary_kernel<128><<<dim3(p.P_max, p.H, 2), tc5::kThreads, sm, st>>>(p);
+        tc5::summary_kernel<128><<<dim3((unsigned)(p.P_max * p.H), 2), tc5::kThreads, sm, st>>>(p);
         return cudaGetLastError();
     }
     e = cudaFuncSetAttribute(tc5::output_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)sm);
     if (e != cudaSuccess) return e;
-    tc5::output_kernel<128><<<dim3(p.P_max, p.H, 1), tc5::kThreads, sm, st>>>(p);
+    tc5::output_kernel<128><<<dim3((unsigned)(p.P_max * p.H)), tc5::kThreads, sm, st>>>(p);
     return cudaGetLastError();
 }
 
