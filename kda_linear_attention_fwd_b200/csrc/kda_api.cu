@@ -142,6 +142,7 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const void *g, co
     p.P_max = (int)P_max;
     p.scale = scale;
     p.qk_l2norm = qk_l2norm;
+    p.total_tokens = total_tokens;
 
     const bool bf16 = dtype == KDA_DTYPE_BF16;
     cudaError_t e = kda::launch_plan(cu_seqlens, num_seqs, total_tokens, L, (int)P_max,

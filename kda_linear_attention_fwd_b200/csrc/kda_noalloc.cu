@@ -156,6 +156,7 @@ extern "C" int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v
     p.P_max = (int)P_max;
     p.scale = scale;
     p.qk_l2norm = qk_l2norm;
+    p.total_tokens = total_tokens;
 
     const bool bf16 = dtype == KDA_DTYPE_BF16;
     cudaError_t e = kda::launch_plan(cu_seqlens, num_seqs, total_tokens, (int)L, (int)P_max,

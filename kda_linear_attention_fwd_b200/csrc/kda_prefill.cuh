@@ -141,6 +141,7 @@ struct PrefillParams {
     float *final_state;
     int32_t *err;  // header[2]: set to nonzero when a bounded device wait gave up
     int num_seqs, H, P_max;
+    int total_tokens;
     float scale;
     int qk_l2norm;
 };

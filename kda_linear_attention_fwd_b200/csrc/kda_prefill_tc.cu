@@ -2,31 +2,36 @@
 // 5th-generation tensor cores (tcgen05, accumulators in tensor memory).
 //
 // One CTA runs one piece of one head (dk = dv = 128).  Warps 0-3 form the
-// state warpgroup: thread j owns state column j -- row j of S^T, fp32, in
-// registers -- and TMEM lane j.  Per chunk (see kda_prefill_simt.cu for the
-// algebra), with everything the chunk needs prepared one chunk ahead by the
-// prep warps:
+// state warpgroup: thread j owns state column j -- row j of S^T -- which
+// lives in TMEM lane j (fp32, plus a bf16 copy as an MMA operand).  Per chunk
+// (see kda_prefill_simt.cu for the algebra), with everything the chunk needs
+// prepared ahead by the prep team:
 //
 //   MMA 1  D1      = V^T [Tb^T | 0]             (M=128, N=32, K=16; A MN-major smem)
 //   MMA 2  D1     += S^T [-W^T | Qd^T]          (K=128; A = bf16 S^T in TMEM)
 //          -> D1[:, 0:16] = U^T, D1[:, 16:32] = (Qd S)^T
 //   WG     U^T (bf16) -> shared memory (A operand of the next two)
-//   MMA 3  D2      = U^T Kb                     (M=128, N=128, K=16)
+//   MMA 3  S^T    += U^T Kb                     (M=128, N=128, K=16; S^T pre-scaled)
 //   MMA 4  D1[16:] += U^T P^T                   (M=128, N=16, K=16) -> O^T
-//   WG     y = gate (.) O;  S^T <- S^T Diag(exp G_C) + D2 (fp32, registers);
-//          bf16 copy of S^T -> TMEM (A operand of the next chunk's MMA 2)
+//   WG     y = gate (.) O;  one pass over S^T: its bf16 copy, and S^T scaled
+//          by the next chunk's exp(G_C) so that its MMA 3 accumulates into it
 //
-// One thread issues the MMAs; tcgen05.commit arrives on an mbarrier that the
-// warpgroup waits on with a time bound (2 s): a wait that gives up records an
-// error in the workspace header and the kernel drains without further tensor
-// work, keeping every named-barrier hand-off so that no warp is left waiting.
+// One elected lane issues the MMAs; tcgen05.commit arrives on an mbarrier that
+// the warpgroup waits on with a time bound (2 s): a wait that gives up records
+// an error in the workspace header and the kernel drains without further
+// tensor work, keeping every named-barrier hand-off so that no warp is left
+// waiting.
 //
-// Prep warps 4-7 each own every fourth chunk: cp.async of q, k, g into a
-// private buffer and of v and gate straight into the stage, exp(G) as prefix
-// and suffix products of exp(g), the Gram matrices A = Kd Ki^T and
-// P = Qd Ki^T and W = Tb Kd on warp-level MMA (16x16 tiles are far below the
-// smallest tcgen05 tile), and the 16x16 unit-lower solve in fp32.  Every MMA
-// operand is written in the canonical no-swizzle K-major / MN-major layout.
+// The prep team (warps 4-7) prepares one chunk at a time into one of three
+// stages: cp.async of q, k, g two chunks ahead into a ring of raw tiles and of
+// v into the stage; exp(G) as prefix and suffix products of exp(g) with one
+// thread per key-channel pair and half of the rows; the Gram matrices
+// A = Kd Ki^T and P = Qd Ki^T on two warps in parallel (16x16 tiles are far
+// below the smallest tcgen05 tile, so these use warp-level MMA); the 16x16
+// unit-lower solve in fp32 on one warp; W = Tb Kd split over the four warps
+// by key channel.  Every MMA operand is written in the canonical no-swizzle
+// K-major / MN-major layout.  A stage goes back to the team as soon as the
+// update MMAs that read it have completed.
 //
 // Sources: the token pipeline and the decay floor -- affta.cn K3 explainer,
 // section "第一关：KDA 解决算得动"; decay as an absolute-position transform over a
@@ -37,6 +42,12 @@
 #include "kda_common.cuh"
 #include "kda_prefill.cuh"
 #include "kda_sm100.cuh"
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cstring>
+#include <type_traits>
 
 // Optional timeline hooks for one CTA (piece 1, head 0), compiled only with
 // -DKDA_TC5_TRACE: SM clock at fixed points of the state warpgroup's and the
@@ -63,29 +74,47 @@ namespace tc5 {
 
 using namespace sm100;
 
-constexpr int kPrepWarps = 3;                 // = stages; chunk c -> prep warp c % 3
-constexpr int kThreads = 128 + 32 * kPrepWarps;
+constexpr int kStages = 3;     // prepared chunks in flight: chunk c -> stage c % 3
+constexpr int kRaw = 3;        // q, k, g tiles in flight: chunk c -> raw[c % 3]
+constexpr int kPair = 64;      // threads of the decay pair (warps 4-5) and of the matrix pair (6-7)
+constexpr int kThreads = 128 + 2 * kPair;
 constexpr int kBlocksPerSM = 2;
-constexpr int BAR_FULL = 1;    // ids 1..3: prep warp s arrives, state warpgroup waits
-constexpr int BAR_EMPTY = 4;   // ids 4..6: state warpgroup arrives, prep warp s waits
+constexpr int BAR_FULL = 1;    // ids 1..3: the matrix pair arrives, the state warpgroup waits
+constexpr int BAR_EMPTY = 4;   // ids 4..6: the state warpgroup arrives, the decay pair waits
 constexpr int BAR_WG = 7;      // state warpgroup only
-constexpr int kBarCount = 160;
+constexpr int BAR_DEC = 8;     // ids 8..10: the decay pair arrives, the matrix pair waits
+constexpr int BAR_DPAIR = 11;  // decay pair only
+constexpr int BAR_MPAIR = 12;  // matrix pair only
+constexpr int kBarCount = 128 + kPair;  // FULL and EMPTY: the state warpgroup and one pair
+constexpr int kDecCount = 2 * kPair;
 constexpr int NC = 128;        // state columns = TMEM lanes = MMA M
-constexpr int kPad = 8;
 constexpr uint32_t kTmemCols = 256;
+
+// TMA descriptors of q, k and g as [T][H][128] bf16 (3-D: channel, head,
+// token); one box = 64 channels x 1 head x 16 tokens, 128-byte swizzle.
+struct TmaMaps {
+    CUtensorMap q, k, g;
+};
+
+// Byte offset of element (r, ch) of a 16 x 128 bf16 tile that TMA wrote as two
+// 64-channel boxes with the 128-byte swizzle: 16-byte chunk j of row r lands
+// in chunk j ^ (r & 7) of that row (each box 1024-byte aligned).
+KDA_DEVICE uint32_t sw128(int r, int ch) {
+    return (uint32_t)((ch >> 6) * 2048 + r * 128 + ((((ch & 63) >> 3) ^ (r & 7)) << 4) + ((ch & 7) << 1));
+}
 
 template <int DK>
 struct Layout {
-    static constexpr int LK = DK + kPad;
     // TMEM columns (per CTA: 256 of the SM's 512)
     static constexpr uint32_t COL_S = 0;          // S^T, fp32: DK columns (MMA 3 accumulator)
     static constexpr uint32_t COL_D1 = DK;        // 2 x [U^T | O^T]: 2 x 32 fp32 columns
     static constexpr uint32_t COL_AS = DK + 64;   // bf16 S^T (MMA A operand): DK/2 columns
     static_assert(COL_AS + DK / 2 <= kTmemCols, "TMEM budget");
-    struct Work {                                 // cp.async targets, overwritten in place:
-        alignas(16) bf16 q[16 * LK];              //   q -> Qd
-        alignas(16) bf16 k[16 * LK];              //   k -> Kd
-        alignas(16) bf16 g[16 * LK];              //   g -> Ki
+    static_assert(DK == 128, "one tile row = two 64-channel TMA boxes");
+    struct Raw {                                  // TMA targets (swizzled), overwritten in place:
+        alignas(1024) unsigned char q[16 * DK * 2];  //   q -> Qd
+        alignas(1024) unsigned char k[16 * DK * 2];  //   k -> Kd
+        alignas(1024) unsigned char g[16 * DK * 2];  //   g -> Ki
     };
     struct Stage {
         alignas(16) bf16 b1[32 * DK];   // K-major [32][DK]: rows 0-15 = -W, 16-31 = Qd
@@ -96,20 +125,22 @@ struct Layout {
         alignas(16) float gam[DK];      // exp(G_C) per key channel
     };
     struct Prep {
-        alignas(16) float AT[16 * 16];  // AT[s][r] = beta_r A[r][s], r > s
-        float beta[16];
-        float rq[16], rk[16];
+        alignas(16) float AT[16 * 16];  // AT[s][r] = beta_r A[r][s], r > s (matrix pair)
+        float beta[kStages][16];        // beta of the chunk in each stage
+        float nk[2][16], nq[2][16];     // per decay warp and row: partial sums of k^2, q^2
     };
     struct All {
-        Work work[kPrepWarps];
-        Stage st[kPrepWarps];
-        Prep pr[kPrepWarps];
+        Raw raw[kRaw];
+        Stage st[kStages];
+        Prep pr;
         alignas(16) bf16 au[NC * 16];   // K-major [NC][16]: U^T as the A operand
         alignas(16) bf16 io[2][16 * NC];  // gate tile in, y tile out (row-major [16][NC])
         alignas(8) unsigned long long mbar[2];
+        alignas(8) unsigned long long mbar_raw[kRaw];  // TMA completion of raw[i]
         uint32_t tmem_base;
     };
-    static constexpr size_t bytes = sizeof(All);
+    // plus slack to align the start to 1024 bytes (the swizzle's period)
+    static constexpr size_t bytes = sizeof(All) + 1024;
 };
 
 template <typename T>
@@ -121,12 +152,12 @@ KDA_DEVICE T *at_bytes(T *base, uint32_t off) {
 // y.  USE_V: the write uses v (false: the transition part, U0 = 0).  The
 // state starts as the identity, a copy of s_init ([DK][NC] fp32) or zeros and
 // is written to s_out.  The fp32 state lives in tensor memory.
-template <int DK, bool OUT, bool USE_V>
-__device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const float *s_init,
-                          bool identity, float *s_out, unsigned char *smem_raw) {
+template <int DK, bool OUT, bool USE_V, bool L2N>
+__device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, int len, int h,
+                          const float *s_init, bool identity, float *s_out, unsigned char *smem_raw) {
     using Lay = Layout<DK>;
-    constexpr int LK = Lay::LK;
-    typename Lay::All &sm = *reinterpret_cast<typename Lay::All *>(smem_raw);
+    typename Lay::All &sm = *reinterpret_cast<typename Lay::All *>(
+        smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int H = p.H;
     const int nchunks = (len + 15) / 16;
@@ -142,6 +173,7 @@ __device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const 
     if (tid == 32) {
         mbar_init(smem_u32(&sm.mbar[0]), 1);
         mbar_init(smem_u32(&sm.mbar[1]), 1);
+        for (int i = 0; i < kRaw; ++i) mbar_init(smem_u32(&sm.mbar_raw[i]), 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     tc_fence_before();
@@ -289,25 +321,27 @@ __device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const 
         //               U -> smem  MMA 3/4 (c)  |  y(c-1) -> global
         //               next stage; state pass
         for (int c = 0; c < nchunks; ++c) {
-            const int stg = c % kPrepWarps;
+            const int stg = c % kStages;
             const uint32_t d1_col = Lay::COL_D1 + 32 * (c & 1);
             KDA_MARK(tid == 0 && c < 128, c * 16 + 0);
             if (OUT) cp_async_wait<0>();  // this thread's pieces of the gate tile of chunk c - 1
             bar_sync(BAR_WG, 128);        // state-pass TMEM stores; gate tile; y(c - 2) stored
             if (OUT) load_gate(c);
             KDA_MARK(tid == 0 && c < 128, c * 16 + 1);
-            if (tid == 0 && ok) {  // U0^T and [-W | Qd] S^T: needs only the bf16 copy
-                tc_fence_after();
+            if (warp == 0 && ok) {  // U0^T and [-W | Qd] S^T: needs only the bf16 copy
                 const uint32_t d1 = tbase + d1_col;
                 const uint64_t so = kStageStep * stg;
-                if (USE_V) tc_mma_ss(d1, dsc_v0 + so, dsc_b00 + so, ID_U0, 0);
+                if (elect_one_sync()) {
+                    tc_fence_after();
+                    if (USE_V) tc_mma_ss(d1, dsc_v0 + so, dsc_b00 + so, ID_U0, 0);
 #pragma unroll
-                for (int kk = 0; kk < DK / 16; ++kk)  // +256 bytes of K = +16 in the start field
-                    tc_mma_ts(d1, tbase + Lay::COL_AS + 8 * kk, dsc_b10 + so + 16 * kk, ID_WS,
-                              (USE_V || kk > 0) ? 1u : 0u);
-                tc_commit(mb1);
+                    for (int kk = 0; kk < DK / 16; ++kk)  // +256 bytes of K = +16 in the start field
+                        tc_mma_ts(d1, tbase + Lay::COL_AS + 8 * kk, dsc_b10 + so + 16 * kk, ID_WS,
+                                  (USE_V || kk > 0) ? 1u : 0u);
+                    tc_commit(mb1);
+                }
+                __syncwarp();  // reconverge warp 0 before the aligned TMEM loads below
             }
-            __syncwarp();  // reconverge warp 0 before the aligned TMEM loads below
             KDA_MARK(tid == 0 && c < 128, c * 16 + 2);
             if (c > 0) finish_chunk(c - 1);
             KDA_MARK(tid == 0 && c < 128, c * 16 + 5);
@@ -329,18 +363,20 @@ __device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const 
             tc_fence_before();
             KDA_MARK(tid == 0 && c < 128, c * 16 + 7);
             bar_sync(BAR_WG, 128);
-            if (tid == 0 && ok) {  // S^T += U^T Kb (into the state itself);  O^T += U^T P^T
-                tc_fence_after();
+            if (warp == 0 && ok) {  // S^T += U^T Kb (into the state itself);  O^T += U^T P^T
                 const uint64_t so = kStageStep * stg;
-                tc_mma_ss(tbase + Lay::COL_S, dsc_au, dsc_b20 + so, ID_UK, 1);
-                if (OUT) tc_mma_ss(tbase + d1_col + 16, dsc_au, dsc_b30 + so, ID_UP, 1);
-                tc_commit(mb2);
+                if (elect_one_sync()) {
+                    tc_fence_after();
+                    tc_mma_ss(tbase + Lay::COL_S, dsc_au, dsc_b20 + so, ID_UK, 1);
+                    if (OUT) tc_mma_ss(tbase + d1_col + 16, dsc_au, dsc_b30 + so, ID_UP, 1);
+                    tc_commit(mb2);
+                }
+                __syncwarp();  // reconverge warp 0 before the aligned barrier below
             }
-            __syncwarp();  // reconverge warp 0 before the aligned barrier below
             const bool has_next = c + 1 < nchunks;
             if (OUT && c > 0) store_y(c - 1);
             KDA_MARK(tid == 0 && c < 128, c * 16 + 8);
-            if (has_next) bar_sync(BAR_FULL + (c + 1) % kPrepWarps, kBarCount);
+            if (has_next) bar_sync(BAR_FULL + (c + 1) % kStages, kBarCount);
             KDA_MARK(tid == 0 && c < 128, c * 16 + 9);
             if (ok) ok = mbar_wait(mb2, c & 1);
             ok = __all_sync(0xffffffffu, ok);
@@ -349,7 +385,7 @@ __device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const 
             bar_arrive(BAR_EMPTY + stg, kBarCount);  // every reader of this stage is done
             KDA_MARK(tid == 0 && c < 128, c * 16 + 10);
             if (ok) {
-                state_pass(has_next ? sm.st[(c + 1) % kPrepWarps].gam : nullptr, false);
+                state_pass(has_next ? sm.st[(c + 1) % kStages].gam : nullptr, false);
             } else {
                 tc_fence_before();
             }
@@ -365,170 +401,209 @@ __device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const 
             }
         }
         if (!ok && lane == 0 && p.err) atomicOr(p.err, 1);
-    } else {
-        // ----------------------------------------------------------- prep warps
-        const int pw = warp - 4;
-        const bf16 *q = (const bf16 *)p.q, *k = (const bf16 *)p.k, *g = (const bf16 *)p.g;
+    } else if (warp < 6) {
+        // ------------------------------------------------------------ decay pair
+        // Warps 4-5: thread d owns the key-channel pair (ip, ip + 1) on all 16
+        // rows of a chunk; it runs up to kRaw chunks ahead of the matrix pair.
+        const int d = tid - 128, dw = d >> 5, ip = 2 * d;
         const bf16 *v = (const bf16 *)p.v, *beta = (const bf16 *)p.beta;
-        typename Lay::Prep &pr = sm.pr[pw];
-        typename Lay::Work &Wk = sm.work[pw];
-        typename Lay::Stage &St = sm.st[pw];
-        float beta_next = 0.f;
-
-        // rows 16-31 of the [Tb^T | 0] operand stay zero
-        reinterpret_cast<uint4 *>(at_bytes(St.b0, kmaj(16, 0, 16)))[lane] = make_uint4(0, 0, 0, 0);
-
-        auto issue_raw = [&](int c) {
-            const int tc = t0 + 16 * c;
+        typename Lay::Prep &pr = sm.pr;
+        // beta of chunks c and c + 1 (threads d < 16), kept as raw bf16 bits so
+        // that the load of chunk c + 2 is not waited for until it is stored
+        unsigned short bq0 = 0, bq1 = 0;
+        auto load_beta = [&](int c) -> unsigned short {
             const int rows = min(16, len - 16 * c);
-            constexpr int PK = DK / 8;
-#pragma unroll 4
-            for (int x = lane; x < 16 * PK; x += 32) {
-                const int r = x / PK, cc = x % PK;
-                const bool okr = r < rows;
-                const size_t off = ((size_t)(okr ? tc + r : t0) * H + h) * DK + cc * 8;
-                cp_async16(&Wk.k[r * LK + cc * 8], k + off, okr);
-                cp_async16(&Wk.g[r * LK + cc * 8], g + off, okr);
-                if (OUT) cp_async16(&Wk.q[r * LK + cc * 8], q + off, okr);
-            }
-            cp_async_commit();
-            beta_next = lane < rows ? __bfloat162float(beta[(size_t)(tc + lane) * H + h]) : 0.f;
+            return d < rows ? reinterpret_cast<const unsigned short *>(beta)[(size_t)(t0 + 16 * c + d) * H + h]
+                            : (unsigned short)0;
         };
+        // V^T of chunk c -> its stage (MN-major A operand of MMA 1)
         auto issue_v = [&](int c) {
             if (USE_V) {
-                const int tc = t0 + 16 * c;
-                const int rows = min(16, len - 16 * c);
+                typename Lay::Stage &Sv = sm.st[c % kStages];
+                const int tc = t0 + 16 * c, rows = min(16, len - 16 * c);
                 constexpr int PV = NC / 8;
-#pragma unroll 4
-                for (int x = lane; x < 16 * PV; x += 32) {
+#pragma unroll
+                for (int x = d; x < 16 * PV; x += kPair) {
                     const int r = x / PV, cc = x % PV;
                     const bool okr = r < rows;
                     const size_t off = ((size_t)(okr ? tc + r : t0) * H + h) * NC + cc * 8;
-                    cp_async16(at_bytes(St.v, mnmaj(cc * 8, r, 16)), v + off, okr);
+                    cp_async16(at_bytes(Sv.v, mnmaj(cc * 8, r, 16)), v + off, okr);
                 }
             }
-            cp_async_commit();
         };
+        if (d < 16) {
+            if (nchunks > 0) bq0 = load_beta(0);
+            if (nchunks > 1) bq1 = load_beta(1);
+        }
+        bool tok = true;  // every raw tile arrived within the time bound
 
-        if (pw < nchunks) issue_raw(pw);
-        for (int c = pw; c < nchunks; c += kPrepWarps) {
-            KDA_MARK(lane == 0 && c < 128, 2048 + c * 8 + 0);
-            if (c >= kPrepWarps) bar_sync(BAR_EMPTY + pw, kBarCount);  // stage free again
-            KDA_MARK(lane == 0 && c < 128, 2048 + c * 8 + 1);
+        for (int c = 0; c < nchunks; ++c) {
+            const int stg = c % kStages;
+            typename Lay::Raw &Wk = sm.raw[c % kRaw];
+            typename Lay::Stage &St = sm.st[stg];
+            KDA_MARK(d == 0 && c < 128, 2048 + c * 8 + 0);
+            if (c >= kStages) bar_sync(BAR_EMPTY + stg, kBarCount);  // the stage is free again
+            KDA_MARK(d == 0 && c < 128, 2048 + c * 8 + 1);
             issue_v(c);
-            if (lane < 16) pr.beta[lane] = beta_next;
-            cp_async_wait<1>();  // q, k, g of chunk c
-            __syncwarp();
-            KDA_MARK(lane == 0 && c < 128, 2048 + c * 8 + 2);
-
-            if (p.qk_l2norm) {
-                for (int r = 0; r < 16; ++r) {
-                    float kk = 0.f, qq = 0.f;
-                    for (int i = lane; i < DK; i += 32) {
-                        const float kv = __bfloat162float(Wk.k[r * LK + i]);
-                        kk += kv * kv;
-                        if (OUT) {
-                            const float qv = __bfloat162float(Wk.q[r * LK + i]);
-                            qq += qv * qv;
-                        }
+            cp_async_commit();
+            unsigned short bq2 = 0;
+            if (d < 16 && c + 2 < nchunks) bq2 = load_beta(c + 2);
+            if (tok) tok = mbar_wait(smem_u32(&sm.mbar_raw[c % kRaw]), (c / kRaw) & 1);
+            {   // rows past the end of the piece read as zero (decay 1, no write)
+                const int rows = min(16, len - 16 * c);
+                if (rows < 16) {
+                    const int n = (16 - rows) * 2 * 8;  // 16-byte pieces per array
+                    for (int x = d; x < 3 * n; x += kPair) {
+                        const int a = x / n, y = x % n, r = rows + y / 16, hf = (y / 8) & 1, pc = y % 8;
+                        unsigned char *base = a == 0 ? Wk.k : (a == 1 ? Wk.g : Wk.q);
+                        *reinterpret_cast<uint4 *>(base + hf * 2048 + r * 128 + pc * 16) = make_uint4(0, 0, 0, 0);
                     }
-                    kk = warp_sum(kk);
-                    qq = warp_sum(qq);
-                    if (lane == r) {
-                        pr.rk[r] = rsqrtf(kk + 1e-6f);
-                        pr.rq[r] = rsqrtf(qq + 1e-6f);
+                }
+            }
+            if (d < 16) pr.beta[stg][d] = __bfloat162float(__ushort_as_bfloat16(bq0));
+            __syncwarp();
+            bar_sync(BAR_DPAIR, kPair);             // the tiles (with cleared rows) are visible
+            KDA_MARK(d == 0 && c < 128, 2048 + c * 8 + 2);
+            if (L2N) {  // row norms of k and q: the two warps cover all channels
+#pragma unroll
+                for (int r = 0; r < 16; ++r) {
+                    const float2 kv = unpack_bf16(*reinterpret_cast<const uint32_t *>(Wk.k + sw128(r, ip)));
+                    float sk = kv.x * kv.x + kv.y * kv.y, sq = 0.f;
+                    if (OUT) {
+                        const float2 qv = unpack_bf16(*reinterpret_cast<const uint32_t *>(Wk.q + sw128(r, ip)));
+                        sq = qv.x * qv.x + qv.y * qv.y;
+                    }
+                    sk = warp_sum(sk);
+                    sq = warp_sum(sq);
+                    if (lane == 0) {
+                        pr.nk[dw][r] = sk;
+                        pr.nq[dw][r] = sq;
                     }
                 }
                 __syncwarp();
+                bar_sync(BAR_DPAIR, kPair);
             }
 
-            // 1. decay factors and decayed operands (in place: k -> Kd,
-            //    g -> Ki, q -> Qd); lane owns channel pairs (2 lane, 2 lane + 1)
-#pragma unroll 1
-            for (int cp2 = 0; cp2 < DK / 64; ++cp2) {
-                const int i = 64 * cp2 + 2 * lane;
-                float2 e[16], E[16];
+            // exp(G_r) (inclusive prefix products of exp(g)), exp(G_C) and the
+            // exclusive suffix products exp(G_C - G_r), in fp32
+            float2 e[16], E[16];
 #pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    const float2 gg = unpack_bf16(*reinterpret_cast<const uint32_t *>(&Wk.g[r * LK + i]));
-                    e[r] = make_float2(__expf(gg.x), __expf(gg.y));
-                }
+            for (int r = 0; r < 16; ++r) {
+                const float2 gg = unpack_bf16(*reinterpret_cast<const uint32_t *>(Wk.g + sw128(r, ip)));
+                e[r] = make_float2(__expf(gg.x), __expf(gg.y));
+            }
+            {
                 float2 acc = make_float2(1.f, 1.f);
 #pragma unroll
                 for (int r = 0; r < 16; ++r) {
                     acc = f2mul(acc, e[r]);
                     E[r] = acc;
                 }
-                const float2 El = acc;
-                const float2 invEl = make_float2(1.f / El.x, 1.f / El.y);
-                *reinterpret_cast<float2 *>(&St.gam[i]) = El;
-                float2 F = make_float2(1.f, 1.f);  // exp(G_C - G_r): suffix products
-                uint32_t kb0[8], kb1[8];           // Kb^T rows i, i+1 (token pairs)
-                float2 kb_hi = make_float2(0.f, 0.f);
-#pragma unroll
-                for (int r = 15; r >= 0; --r) {
-                    float2 kv = unpack_bf16(*reinterpret_cast<const uint32_t *>(&Wk.k[r * LK + i]));
-                    if (p.qk_l2norm) kv = f2mul(kv, make_float2(pr.rk[r], pr.rk[r]));
-                    *reinterpret_cast<uint32_t *>(&Wk.k[r * LK + i]) = pack_bf16(f2mul(kv, E[r]));
-                    *reinterpret_cast<uint32_t *>(&Wk.g[r * LK + i]) = pack_bf16(f2mul(kv, f2mul(F, invEl)));
-                    const float2 kbv = f2mul(kv, F);
-                    if (r & 1) {
-                        kb_hi = kbv;
-                    } else {
-                        kb0[r >> 1] = pack_bf16(kbv.x, kb_hi.x);
-                        kb1[r >> 1] = pack_bf16(kbv.y, kb_hi.y);
-                    }
-                    if (OUT) {
-                        const float2 qv = unpack_bf16(*reinterpret_cast<const uint32_t *>(&Wk.q[r * LK + i]));
-                        float sc = p.scale;
-                        if (p.qk_l2norm) sc *= pr.rq[r];
-                        *reinterpret_cast<uint32_t *>(&Wk.q[r * LK + i]) =
-                            pack_bf16(f2mul(f2mul(qv, make_float2(sc, sc)), E[r]));
-                    }
-                    F = f2mul(F, e[r]);
-                }
-                *reinterpret_cast<uint4 *>(at_bytes(St.b2, kmaj(i, 0, 16))) = make_uint4(kb0[0], kb0[1], kb0[2], kb0[3]);
-                *reinterpret_cast<uint4 *>(at_bytes(St.b2, kmaj(i, 8, 16))) = make_uint4(kb0[4], kb0[5], kb0[6], kb0[7]);
-                *reinterpret_cast<uint4 *>(at_bytes(St.b2, kmaj(i + 1, 0, 16))) = make_uint4(kb1[0], kb1[1], kb1[2], kb1[3]);
-                *reinterpret_cast<uint4 *>(at_bytes(St.b2, kmaj(i + 1, 8, 16))) = make_uint4(kb1[4], kb1[5], kb1[6], kb1[7]);
             }
-            __syncwarp();
-            KDA_MARK(lane == 0 && c < 128, 2048 + c * 8 + 3);
-            const bf16 *Kd = Wk.k, *Ki = Wk.g, *Qd = Wk.q;
-
-            if (OUT) {  // Qd -> rows 16-31 of the [-W | Qd] operand (canonical layout)
+            const float2 El = E[15];
+            const float2 invEl = make_float2(__frcp_rn(El.x), __frcp_rn(El.y));
+            *reinterpret_cast<float2 *>(&St.gam[ip]) = El;
+            float2 F = make_float2(1.f, 1.f);
+            uint32_t kb0[8], kb1[8];  // Kb^T rows ip, ip + 1 (token pairs)
+            float2 kb_hi = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int it = 0; it < DK / 16; ++it) {
-                    const int x = lane + 32 * it;
-                    const int r = x & 15, kc = x >> 4;
-                    *reinterpret_cast<uint4 *>(at_bytes(St.b1, kmaj(16 + r, 8 * kc, DK))) =
-                        *reinterpret_cast<const uint4 *>(&Qd[r * LK + 8 * kc]);
+            for (int r = 15; r >= 0; --r) {
+                float2 kv = unpack_bf16(*reinterpret_cast<const uint32_t *>(Wk.k + sw128(r, ip)));
+                float sc = p.scale;
+                if (L2N) {
+                    const float rk = rsqrtf(pr.nk[0][r] + pr.nk[1][r] + 1e-6f);
+                    kv = f2mul(kv, make_float2(rk, rk));
+                    sc *= rsqrtf(pr.nq[0][r] + pr.nq[1][r] + 1e-6f);
                 }
+                *reinterpret_cast<uint32_t *>(Wk.k + sw128(r, ip)) = pack_bf16(f2mul(kv, E[r]));
+                *reinterpret_cast<uint32_t *>(Wk.g + sw128(r, ip)) = pack_bf16(f2mul(kv, f2mul(F, invEl)));
+                const float2 kbv = f2mul(kv, F);
+                if (r & 1) {
+                    kb_hi = kbv;
+                } else {
+                    kb0[r >> 1] = pack_bf16(kbv.x, kb_hi.x);
+                    kb1[r >> 1] = pack_bf16(kbv.y, kb_hi.y);
+                }
+                if (OUT) {
+                    const float2 qv = unpack_bf16(*reinterpret_cast<const uint32_t *>(Wk.q + sw128(r, ip)));
+                    *reinterpret_cast<uint32_t *>(Wk.q + sw128(r, ip)) =
+                        pack_bf16(f2mul(f2mul(qv, make_float2(sc, sc)), E[r]));
+                }
+                F = f2mul(F, e[r]);
             }
-
-            // 2. A = Kd Ki^T (strictly lower) and P = Qd Ki^T (lower)
+            *reinterpret_cast<uint4 *>(at_bytes(St.b2, kmaj(ip, 0, 16))) = make_uint4(kb0[0], kb0[1], kb0[2], kb0[3]);
+            *reinterpret_cast<uint4 *>(at_bytes(St.b2, kmaj(ip, 8, 16))) = make_uint4(kb0[4], kb0[5], kb0[6], kb0[7]);
+            *reinterpret_cast<uint4 *>(at_bytes(St.b2, kmaj(ip + 1, 0, 16))) = make_uint4(kb1[0], kb1[1], kb1[2], kb1[3]);
+            *reinterpret_cast<uint4 *>(at_bytes(St.b2, kmaj(ip + 1, 8, 16))) = make_uint4(kb1[4], kb1[5], kb1[6], kb1[7]);
+            KDA_MARK(d == 0 && c < 128, 2048 + c * 8 + 3);
+            // v of chunk c has landed; the stage's and the tile's generic writes
+            // become visible to the tensor core and ordered before a TMA refill
+            cp_async_wait<0>();
+            fence_async_smem();
+            bar_arrive(BAR_DEC + c % kRaw, kDecCount);
+            bq0 = bq1;
+            bq1 = bq2;
+        }
+        if (!tok && p.err) atomicOr(p.err, 2);
+        // the stages of the last chunks come back before the CTA tears down
+        for (int c = max(nchunks - kStages, 0); c < nchunks; ++c) bar_sync(BAR_EMPTY + c % kStages, kBarCount);
+    } else {
+        // ----------------------------------------------------------- matrix pair
+        // Warps 6-7: the Gram matrices, the unit-lower solve, W, and the TMA
+        // loads of q, k, g (thread 0).
+        const int m = tid - 192, mw = m >> 5;
+        typename Lay::Prep &pr = sm.pr;
+        auto issue_raw = [&](int c) {
+            typename Lay::Raw &R = sm.raw[c % kRaw];
+            const uint32_t mb = smem_u32(&sm.mbar_raw[c % kRaw]);
+            const int tc = t0 + 16 * c;
+            mbar_arrive_expect_tx(mb, (OUT ? 3u : 2u) * 16u * DK * 2u);
 #pragma unroll
-            for (int which = 0; which < (OUT ? 2 : 1); ++which) {
-                const bf16 *Aop = which == 0 ? Kd : Qd;
+            for (int hf = 0; hf < 2; ++hf) {
+                tma_load_3d(smem_u32(R.k) + 2048 * hf, &maps.k, 64 * hf, h, tc, mb);
+                tma_load_3d(smem_u32(R.g) + 2048 * hf, &maps.g, 64 * hf, h, tc, mb);
+                if (OUT) tma_load_3d(smem_u32(R.q) + 2048 * hf, &maps.q, 64 * hf, h, tc, mb);
+            }
+        };
+        if (m == 0)
+            for (int c = 0; c < min(nchunks, kRaw); ++c) issue_raw(c);
+        // rows 16-31 of every stage's [Tb^T | 0] operand stay zero
+        for (int x = m; x < kStages * 32; x += kPair)
+            reinterpret_cast<uint4 *>(at_bytes(sm.st[x / 32].b0, kmaj(16, 0, 16)))[x % 32] =
+                make_uint4(0, 0, 0, 0);
+
+        for (int c = 0; c < nchunks; ++c) {
+            const int stg = c % kStages;
+            typename Lay::Raw &Wk = sm.raw[c % kRaw];
+            typename Lay::Stage &St = sm.st[stg];
+            const float *bet = pr.beta[stg];
+            KDA_MARK(m == 0 && c < 128, 2048 + c * 8 + 4);
+            bar_sync(BAR_DEC + c % kRaw, kDecCount);  // Kd, Ki, Qd, Kb^T, exp(G_C), v of chunk c
+            KDA_MARK(m == 0 && c < 128, 2048 + c * 8 + 5);
+            const unsigned char *Kd = Wk.k, *Ki = Wk.g, *Qd = Wk.q;
+
+            // A = Kd Ki^T (warp 6) and P = Qd Ki^T (warp 7) on warp-level MMA
+            if (mw == 0 || OUT) {
+                const unsigned char *Aop = mw == 0 ? Kd : Qd;
                 float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int kk = 0; kk < DK / 16; ++kk) {
                     uint32_t a[4], b[4];
-                    ldsm4(a, &Aop[((lane & 7) + ((lane >> 3) & 1) * 8) * LK + 16 * kk + (lane >> 4) * 8]);
-                    ldsm4(b, &Ki[((lane & 7) + (lane >> 4) * 8) * LK + 16 * kk + ((lane >> 3) & 1) * 8]);
+                    ldsm4(a, Aop + sw128((lane & 7) + ((lane >> 3) & 1) * 8, 16 * kk + (lane >> 4) * 8));
+                    ldsm4(b, Ki + sw128((lane & 7) + (lane >> 4) * 8, 16 * kk + ((lane >> 3) & 1) * 8));
                     mma16816(acc0, a, b[0], b[1]);
                     mma16816(acc1, a, b[2], b[3]);
                 }
                 const int r0 = lane >> 2, c0 = 2 * (lane & 3);
-                if (which == 0) {
+                if (mw == 0) {
                     // AT[s][r] = beta_r A[r][s] for s < r (the solve's column sweeps)
                     const float vals[8] = {acc0[0], acc0[1], acc0[2], acc0[3],
                                            acc1[0], acc1[1], acc1[2], acc1[3]};
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int r = r0 + ((e & 2) ? 8 : 0);
-                        const int sc = c0 + (e & 1) + ((e & 4) ? 8 : 0);
-                        pr.AT[sc * 16 + r] = sc < r ? pr.beta[r] * vals[e] : 0.f;
+                    for (int e2 = 0; e2 < 8; ++e2) {
+                        const int r = r0 + ((e2 & 2) ? 8 : 0);
+                        const int sc = c0 + (e2 & 1) + ((e2 & 4) ? 8 : 0);
+                        pr.AT[sc * 16 + r] = sc < r ? bet[r] * vals[e2] : 0.f;
                     }
                 } else {
                     auto pv = [&](float x, int r, int sc) { return sc <= r ? x : 0.f; };
@@ -543,44 +618,58 @@ __device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const 
                 }
             }
             __syncwarp();
+            bar_sync(BAR_MPAIR, kPair);             // AT and P are written
+            KDA_MARK(m == 0 && c < 128, 2048 + c * 8 + 6);
 
-            KDA_MARK(lane == 0 && c < 128, 2048 + c * 8 + 4);
-            // 3. Tb = (I + Diag(beta) A)^-1 Diag(beta); lane j < 16 owns column j.
-            //    After row r is final it is pushed into every later row.
-            if (lane < 16) {
-                const int jj = lane;
-                float col[16];
+            // Tb = (I + Diag(beta) A)^-1 Diag(beta): lane j < 16 of warp 6 owns
+            // column j, and after row r is final it is pushed into every later
+            // row.  Meanwhile warp 7 copies Qd into rows 16-31 of [-W | Qd].
+            if (mw == 0) {
+                if (lane < 16) {
+                    const int jj = lane;
+                    float col[16];
 #pragma unroll
-                for (int r = 0; r < 16; ++r) col[r] = (r == jj) ? 1.f : 0.f;
+                    for (int r = 0; r < 16; ++r) col[r] = (r == jj) ? 1.f : 0.f;
 #pragma unroll
-                for (int r = 0; r < 15; ++r) {
-                    float at[16];
+                    for (int r = 0; r < 15; ++r) {
+                        float at[16];
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        const float4 a4 = *reinterpret_cast<const float4 *>(&pr.AT[r * 16 + 4 * q4]);
-                        at[4 * q4 + 0] = a4.x; at[4 * q4 + 1] = a4.y;
-                        at[4 * q4 + 2] = a4.z; at[4 * q4 + 3] = a4.w;
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            const float4 a4 = *reinterpret_cast<const float4 *>(&pr.AT[r * 16 + 4 * q4]);
+                            at[4 * q4 + 0] = a4.x; at[4 * q4 + 1] = a4.y;
+                            at[4 * q4 + 2] = a4.z; at[4 * q4 + 3] = a4.w;
+                        }
+#pragma unroll
+                        for (int r2 = r + 1; r2 < 16; ++r2) col[r2] = fmaf(-at[r2], col[r], col[r2]);
                     }
+                    const float bj = bet[jj];
 #pragma unroll
-                    for (int r2 = r + 1; r2 < 16; ++r2) col[r2] = fmaf(-at[r2], col[r], col[r2]);
+                    for (int r = 0; r < 16; ++r)
+                        *at_bytes(St.b0, kmaj(r, jj, 16)) = __float2bfloat16_rn(col[r] * bj);
                 }
-                const float bj = pr.beta[jj];
+            } else if (OUT) {
 #pragma unroll
-                for (int r = 0; r < 16; ++r)
-                    *at_bytes(St.b0, kmaj(r, jj, 16)) = __float2bfloat16_rn(col[r] * bj);
+                for (int it = 0; it < DK / 16; ++it) {
+                    const int x = lane + 32 * it;
+                    const int r = x & 15, kc = x >> 4;
+                    *reinterpret_cast<uint4 *>(at_bytes(St.b1, kmaj(16 + r, 8 * kc, DK))) =
+                        *reinterpret_cast<const uint4 *>(Qd + sw128(r, 8 * kc));
+                }
             }
             __syncwarp();
+            bar_sync(BAR_MPAIR, kPair);             // Tb is written
+            KDA_MARK(m == 0 && c < 128, 2048 + c * 8 + 7);
 
-            KDA_MARK(lane == 0 && c < 128, 2048 + c * 8 + 5);
-            // 4. W = Tb Kd -> rows 0-15 of the [-W | Qd] operand hold -W
+            // W = Tb Kd -> rows 0-15 of the [-W | Qd] operand hold -W; warp mw
+            // covers key channels [DK/2 mw, DK/2 (mw + 1))
             {
                 uint32_t a[4];
                 ldsm4(a, at_bytes(St.b0, kmaj((lane & 7) + ((lane >> 3) & 1) * 8, (lane >> 4) * 8, 16)));
 #pragma unroll
-                for (int np = 0; np < DK / 16; ++np) {
+                for (int np = mw * (DK / 32); np < (mw + 1) * (DK / 32); ++np) {
                     const int n0 = 16 * np;
                     uint32_t b[4];
-                    ldsm4t(b, &Kd[((lane & 7) + ((lane >> 3) & 1) * 8) * LK + n0 + (lane >> 4) * 8]);
+                    ldsm4t(b, Kd + sw128((lane & 7) + ((lane >> 3) & 1) * 8, n0 + (lane >> 4) * 8));
                     float w0[4] = {0.f, 0.f, 0.f, 0.f}, w1[4] = {0.f, 0.f, 0.f, 0.f};
                     mma16816(w0, a, b[0], b[1]);
                     mma16816(w1, a, b[2], b[3]);
@@ -591,18 +680,14 @@ __device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const 
                     *reinterpret_cast<uint32_t *>(at_bytes(St.b1, kmaj(r + 8, cc + 8, DK))) = pack_bf16(-w1[2], -w1[3]);
                 }
             }
-            __syncwarp();
-            KDA_MARK(lane == 0 && c < 128, 2048 + c * 8 + 6);
-            cp_async_wait<0>();  // v of chunk c (the only group in flight)
-            // generic-proxy writes of the stage must be visible to the tensor core
+            // the stage's generic writes become visible to the tensor core; the
+            // raw tile is no longer read by either pair: refill it
             fence_async_smem();
             __syncwarp();
-            KDA_MARK(lane == 0 && c < 128, 2048 + c * 8 + 7);
-            bar_arrive(BAR_FULL + pw, kBarCount);
-            // the work buffers are free: fetch this warp's next chunk
-            if (c + kPrepWarps < nchunks) issue_raw(c + kPrepWarps);
+            bar_sync(BAR_MPAIR, kPair);
+            if (m == 0 && c + kRaw < nchunks) issue_raw(c + kRaw);
+            bar_arrive(BAR_FULL + stg, kBarCount);
         }
-        if (pw < nchunks) bar_sync(BAR_EMPTY + pw, kBarCount);
     }
 
     // ---- tear-down: every TMEM access of the CTA is complete
@@ -614,8 +699,8 @@ __device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const 
                      : "memory");
 }
 
-template <int DK>
-__global__ void __launch_bounds__(kThreads, kBlocksPerSM) summary_kernel(PrefillParams p) {
+template <int DK, bool L2N>
+__global__ void __launch_bounds__(kThreads, kBlocksPerSM) summary_kernel(PrefillParams p, const __grid_constant__ TmaMaps maps) {
     extern __shared__ __align__(128) unsigned char smem[];
     // (piece, head) pairs with the head fastest: co-resident CTAs cover all
     // heads of a few pieces, spreading their rows over every memory channel
@@ -630,15 +715,15 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSM) summary_kernel(Prefill
         const float *init = (j == 0 && p.initial_state)
                                 ? p.initial_state + ((size_t)n * p.H + h) * DK * NC
                                 : nullptr;
-        run_piece<DK, false, true>(p, pc.y, pc.z, h, init, false, p.Szero + ph * DK * NC, smem);
+        run_piece<DK, false, true, L2N>(p, maps, pc.y, pc.z, h, init, false, p.Szero + ph * DK * NC, smem);
     } else {
         if (j == 0) return;
-        run_piece<DK, false, false>(p, pc.y, pc.z, h, nullptr, true, p.M + ph * DK * DK, smem);
+        run_piece<DK, false, false, L2N>(p, maps, pc.y, pc.z, h, nullptr, true, p.M + ph * DK * DK, smem);
     }
 }
 
-template <int DK>
-__global__ void __launch_bounds__(kThreads, kBlocksPerSM) output_kernel(PrefillParams p) {
+template <int DK, bool L2N>
+__global__ void __launch_bounds__(kThreads, kBlocksPerSM) output_kernel(PrefillParams p, const __grid_constant__ TmaMaps maps) {
     extern __shared__ __align__(128) unsigned char smem[];
     // (piece, head) pairs with the head fastest: co-resident CTAs cover all
     // heads of a few pieces, spreading their rows over every memory channel
@@ -651,28 +736,68 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSM) output_kernel(PrefillP
     const float *init = (np == 1) ? (p.initial_state ? p.initial_state + nh * DK * NC : nullptr)
                                   : p.Sin + ((size_t)pi * p.H + h) * DK * NC;
     float *fin = (j == np - 1 && p.final_state) ? p.final_state + nh * DK * NC : nullptr;
-    run_piece<DK, true, true>(p, pc.y, pc.z, h, init, false, fin, smem);
+    run_piece<DK, true, true, L2N>(p, maps, pc.y, pc.z, h, init, false, fin, smem);
 }
 
 }  // namespace tc5
 
 // dk = dv = 128 only (one state column per TMEM lane; the transition part has
 // dk columns too).
-cudaError_t launch_prefill_tc5(const PrefillParams &p, bool summaries, cudaStream_t st) {
+namespace {
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against the driver library); null when the driver does not provide it.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return (PFN_cuTensorMapEncodeTiled_v12000) nullptr;
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }();
+    return fn;
+}
+
+// [T][H][128] bf16 as a 3-D tensor (channel, head, token); box 64 x 1 x 16.
+bool encode_rows(CUtensorMap *m, const void *base, int T, int H) {
+    const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {128, (cuuint64_t)H, (cuuint64_t)T};
+    const cuuint64_t strides[2] = {256, (cuuint64_t)H * 256};
+    const cuuint32_t box[3] = {64, 1, 16};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool L2N>
+cudaError_t launch_tc5(const PrefillParams &p, bool summaries, cudaStream_t st) {
     const size_t sm = tc5::Layout<128>::bytes;
     cudaError_t e;
+    tc5::TmaMaps maps;
+    memset(&maps, 0, sizeof(maps));
+    if (p.total_tokens > 0 &&
+        (!encode_rows(&maps.q, p.q, p.total_tokens, p.H) || !encode_rows(&maps.k, p.k, p.total_tokens, p.H) ||
+         !encode_rows(&maps.g, p.g, p.total_tokens, p.H)))
+        return cudaErrorInvalidValue;
     if (summaries) {
-        e = cudaFuncSetAttribute(tc5::summary_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)sm);
+        e = cudaFuncSetAttribute(tc5::summary_kernel<128, L2N>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
         if (e != cudaSuccess) return e;
-        tc5::summary_kernel<128><<<dim3((unsigned)(p.P_max * p.H), 2), tc5::kThreads, sm, st>>>(p);
+        tc5::summary_kernel<128, L2N><<<dim3((unsigned)(p.P_max * p.H), 2), tc5::kThreads, sm, st>>>(p, maps);
         return cudaGetLastError();
     }
-    e = cudaFuncSetAttribute(tc5::output_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(tc5::output_kernel<128, L2N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)sm);
     if (e != cudaSuccess) return e;
-    tc5::output_kernel<128><<<dim3((unsigned)(p.P_max * p.H)), tc5::kThreads, sm, st>>>(p);
+    tc5::output_kernel<128, L2N><<<dim3((unsigned)(p.P_max * p.H)), tc5::kThreads, sm, st>>>(p, maps);
     return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_prefill_tc5(const PrefillParams &p, bool summaries, cudaStream_t st) {
+    return p.qk_l2norm ? launch_tc5<true>(p, summaries, st) : launch_tc5<false>(p, summaries, st);
 }
 
 }  // namespace kda

@@ -120,6 +120,16 @@ KDA_DEVICE void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uin
         "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// One lane of the (converged, full) warp is elected; the compiler then keeps
+// the MMA operands of the elected lane in the uniform datapath, which halves
+// the issue cost of a tcgen05.mma sequence against a plain lane-0 branch.
+KDA_DEVICE bool elect_one_sync() {
+    uint32_t pred = 0;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.b32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(pred));
+    return pred != 0;
+}
 KDA_DEVICE void tc_commit(uint32_t mbar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
                  : "memory");
@@ -190,6 +200,20 @@ KDA_DEVICE bool mbar_try_wait(uint32_t mbar, uint32_t parity) {
         : "r"(mbar), "r"(parity)
         : "memory");
     return ok != 0;
+}
+// Arrive on the mbarrier and add `bytes` to the transaction count its current
+// phase waits for (the issuing thread of a TMA load).
+KDA_DEVICE void mbar_arrive_expect_tx(uint32_t mbar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mbar), "r"(bytes) : "memory");
+}
+// Tiled TMA load of one box of a 3-D tensor map into this CTA's shared
+// memory; completion is counted in bytes on `mbar`.  The innermost coordinate
+// times the element size must be a multiple of 16 bytes.
+KDA_DEVICE void tma_load_3d(uint32_t dst, const void *tmap, int c0, int c1, int c2, uint32_t mbar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+        "l"(tmap), "r"(mbar), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
 }
 // Bounded wait on an mbarrier phase: gives up after ~2 s of wall time.
 KDA_DEVICE bool mbar_wait(uint32_t mbar, uint32_t parity) {
