@@ -170,6 +170,58 @@ int kda_decode_step(const void *q, const void *k, const void *v, const void *g, 
                     int32_t dk, int32_t dv, kda_dtype dtype, float scale, int32_t qk_l2norm,
                     kda_stream_t stream);
 
+/*
+ * Flags of the extended entry points (kda_chunk_fwd_ex, kda_decode_step_ex).
+ * The preprocessing that the FlashKDA preparation stage folds into its kernel
+ * (affta.cn page, section "FlashKDA ，让线性计算也能沾上并行的光"): q/k
+ * normalisation, the squashing of the write strength and of the output gate,
+ * and the decay floor of the forget gate (affta.cn page, section
+ * "第一关：KDA 解决算得动": at least about 0.67% of the state survives a step).
+ */
+#define KDA_FLAG_QK_L2NORM 1    /* q_t, k_t divided by sqrt(sum x^2 + 1e-6) (= qk_l2norm) */
+#define KDA_FLAG_BETA_LOGITS 2  /* beta holds logits: beta = 1 / (1 + exp(-x)) */
+#define KDA_FLAG_GATE_LOGITS 4  /* gate holds logits: gate = 1 / (1 + exp(-x)) (when not NULL) */
+#define KDA_FLAG_CLAMP_DECAY 8  /* g = max(g, ln 0.0067) per element */
+
+/*
+ * kda_chunk_fwd with a flags word instead of qk_l2norm, and optional state
+ * snapshots (prefix caching at block granularity: the state at fixed token
+ * boundaries of each sequence, so that a later call can resume from any of
+ * them -- prism.simon-ai.net page, section "推理瓶颈与Kimi K3的针对性优化").
+ *
+ *   flags             any OR of the KDA_FLAG_* bits; other bits ->
+ *                     KDA_ERR_INVALID_ARG.
+ *   snapshot_tokens   0 = no snapshots.  Otherwise a multiple of 16: for
+ *                     each sequence n of length L_n the state after tokens
+ *                     m * snapshot_tokens, m = 1 .. (L_n - 1) / snapshot_tokens
+ *                     (the state at L_n itself is the final state), is
+ *                     written to
+ *                     snapshots[((snapshot_offsets[n] + m - 1) * H + h) * dk * dv],
+ *                     laid out [dk][dv] like the states.  Not a multiple of 16,
+ *                     or negative -> KDA_ERR_INVALID_ARG.
+ *   snapshots         device fp32, 16-byte aligned, at least
+ *                     snapshot_offsets[num_seqs] * H * dk * dv floats; must not
+ *                     overlap any other argument.  Required when
+ *                     snapshot_tokens > 0.
+ *   snapshot_offsets  device int32 [num_seqs + 1]: the caller's running sums
+ *                     of (L_n - 1) / snapshot_tokens (0 for empty sequences).
+ *                     Required when snapshot_tokens > 0.
+ * Everything else as kda_chunk_fwd (same workspace size).
+ */
+int kda_chunk_fwd_ex(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                     const void *gate, void *out, const int32_t *cu_seqlens,
+                     const int32_t *cu_seqlens_host, int32_t num_seqs, int32_t total_tokens,
+                     int32_t H, int32_t dk, int32_t dv, kda_dtype dtype, float scale, int32_t flags,
+                     const float *initial_state, float *final_state, int32_t snapshot_tokens,
+                     float *snapshots, const int32_t *snapshot_offsets, void *workspace,
+                     size_t workspace_bytes, kda_stream_t stream);
+
+/* kda_decode_step with a flags word (KDA_FLAG_*) instead of qk_l2norm. */
+int kda_decode_step_ex(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                       const void *gate, void *out, float *state, int32_t num_seqs, int32_t H,
+                       int32_t dk, int32_t dv, kda_dtype dtype, float scale, int32_t flags,
+                       kda_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

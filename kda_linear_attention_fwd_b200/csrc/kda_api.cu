@@ -85,17 +85,23 @@ int kda_chunk_fwd_plan(int32_t total_tokens, int32_t num_seqs, int32_t H, int32_
     return KDA_OK;
 }
 
-int kda_chunk_fwd(const void *q, const void *k, const void *v, const void *g, const void *beta,
-                  const void *gate, void *out, const int32_t *cu_seqlens,
-                  const int32_t *cu_seqlens_host, int32_t num_seqs, int32_t total_tokens,
-                  int32_t H, int32_t dk, int32_t dv, kda_dtype dtype, float scale,
-                  int32_t qk_l2norm, const float *initial_state, float *final_state,
-                  void *workspace, size_t workspace_bytes, kda_stream_t stream_) {
+int kda_chunk_fwd_ex(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                     const void *gate, void *out, const int32_t *cu_seqlens,
+                     const int32_t *cu_seqlens_host, int32_t num_seqs, int32_t total_tokens,
+                     int32_t H, int32_t dk, int32_t dv, kda_dtype dtype, float scale, int32_t flags,
+                     const float *initial_state, float *final_state, int32_t snapshot_tokens,
+                     float *snapshots, const int32_t *snapshot_offsets, void *workspace,
+                     size_t workspace_bytes, kda_stream_t stream_) {
     cudaStream_t stream = (cudaStream_t)stream_;
     if (num_seqs < 0 || total_tokens < 0 || H < 1) return KDA_ERR_INVALID_ARG;
     if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
     if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_UNSUPPORTED;
-    if (qk_l2norm != 0 && qk_l2norm != 1) return KDA_ERR_INVALID_ARG;
+    if (flags & ~kda::FLAG_ALL) return KDA_ERR_INVALID_ARG;
+    if (snapshot_tokens < 0 || snapshot_tokens % 16 != 0) return KDA_ERR_INVALID_ARG;
+    if (snapshot_tokens > 0) {
+        if (!snapshots || !snapshot_offsets) return KDA_ERR_INVALID_ARG;
+        if (!aligned(snapshots, 16) || !aligned(snapshot_offsets, 4)) return KDA_ERR_ALIGNMENT;
+    }
     if (num_seqs == 0) return total_tokens == 0 ? KDA_OK : KDA_ERR_INVALID_ARG;
     if (!cu_seqlens) return KDA_ERR_INVALID_ARG;
     if (total_tokens > 0 && (!q || !k || !v || !g || !beta || !out)) return KDA_ERR_INVALID_ARG;
@@ -141,8 +147,11 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const void *g, co
     p.H = H;
     p.P_max = (int)P_max;
     p.scale = scale;
-    p.qk_l2norm = qk_l2norm;
+    p.flags = flags;
     p.total_tokens = total_tokens;
+    p.snap_tokens = snapshot_tokens;
+    p.snapshots = snapshot_tokens > 0 ? snapshots : nullptr;
+    p.snap_offsets = snapshot_tokens > 0 ? snapshot_offsets : nullptr;
 
     const bool bf16 = dtype == KDA_DTYPE_BF16;
     cudaError_t e = kda::launch_plan(cu_seqlens, num_seqs, total_tokens, L, (int)P_max,
@@ -162,14 +171,26 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const void *g, co
     return KDA_OK;
 }
 
-int kda_decode_step(const void *q, const void *k, const void *v, const void *g, const void *beta,
-                    const void *gate, void *out, float *state, int32_t num_seqs, int32_t H,
-                    int32_t dk, int32_t dv, kda_dtype dtype, float scale, int32_t qk_l2norm,
-                    kda_stream_t stream) {
+int kda_chunk_fwd(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                  const void *gate, void *out, const int32_t *cu_seqlens,
+                  const int32_t *cu_seqlens_host, int32_t num_seqs, int32_t total_tokens,
+                  int32_t H, int32_t dk, int32_t dv, kda_dtype dtype, float scale,
+                  int32_t qk_l2norm, const float *initial_state, float *final_state,
+                  void *workspace, size_t workspace_bytes, kda_stream_t stream) {
+    if (qk_l2norm != 0 && qk_l2norm != 1) return KDA_ERR_INVALID_ARG;
+    return kda_chunk_fwd_ex(q, k, v, g, beta, gate, out, cu_seqlens, cu_seqlens_host, num_seqs,
+                            total_tokens, H, dk, dv, dtype, scale, qk_l2norm, initial_state,
+                            final_state, 0, nullptr, nullptr, workspace, workspace_bytes, stream);
+}
+
+int kda_decode_step_ex(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                       const void *gate, void *out, float *state, int32_t num_seqs, int32_t H,
+                       int32_t dk, int32_t dv, kda_dtype dtype, float scale, int32_t flags,
+                       kda_stream_t stream) {
     if (num_seqs < 0 || H < 1) return KDA_ERR_INVALID_ARG;
     if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
     if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_UNSUPPORTED;
-    if (qk_l2norm != 0 && qk_l2norm != 1) return KDA_ERR_INVALID_ARG;
+    if (flags & ~kda::FLAG_ALL) return KDA_ERR_INVALID_ARG;
     if (num_seqs == 0) return KDA_OK;
     if (!q || !k || !v || !g || !beta || !out || !state) return KDA_ERR_INVALID_ARG;
     const size_t esz = dtype == KDA_DTYPE_BF16 ? 2 : 4;
@@ -180,9 +201,18 @@ int kda_decode_step(const void *q, const void *k, const void *v, const void *g, 
     const long nh = (long)num_seqs * H;
     if (nh > 0x7fffffffL) return KDA_ERR_UNSUPPORTED;
     const cudaError_t e = kda::launch_decode(dtype == KDA_DTYPE_BF16, dk, dv, q, k, v, g, beta,
-                                             gate, out, state, nh, scale, qk_l2norm,
+                                             gate, out, state, nh, scale, flags,
                                              (cudaStream_t)stream);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+int kda_decode_step(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                    const void *gate, void *out, float *state, int32_t num_seqs, int32_t H,
+                    int32_t dk, int32_t dv, kda_dtype dtype, float scale, int32_t qk_l2norm,
+                    kda_stream_t stream) {
+    if (qk_l2norm != 0 && qk_l2norm != 1) return KDA_ERR_INVALID_ARG;
+    return kda_decode_step_ex(q, k, v, g, beta, gate, out, state, num_seqs, H, dk, dv, dtype, scale,
+                              qk_l2norm, stream);
 }
 
 }  // extern "C"

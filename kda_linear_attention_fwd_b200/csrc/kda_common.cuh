@@ -27,6 +27,22 @@ template <typename T> KDA_DEVICE void st(T *p, float x) { Elem<T>::store(p, x); 
 KDA_DEVICE float4 ld_stream(const float4 *p) { return __ldcs(p); }
 KDA_DEVICE void st_stream(float4 *p, float4 v) { __stcs(p, v); }
 
+// Bits of the flags word of the extended entry points (bit 0 is the
+// qk_l2norm switch of the plain ones).
+constexpr int FLAG_L2NORM = 1;       // q, k divided by their L2 norms (+1e-6 under the root)
+constexpr int FLAG_BETA_LOGITS = 2;  // beta given as logits: sigmoid applied on load
+constexpr int FLAG_GATE_LOGITS = 4;  // gate given as logits: sigmoid applied on load
+constexpr int FLAG_CLAMP_G = 8;      // log-decay clamped from below at ln(0.0067)
+constexpr int FLAG_ALL = 15;
+
+// ln(0.0067): the smallest single-step retention of the forget gate
+constexpr float kLogDecayFloor = -5.005647752585217f;
+
+KDA_DEVICE float sigmoid_f(float x) { return 1.f / (1.f + __expf(-x)); }
+KDA_DEVICE float beta_in(float x, int flags) { return (flags & FLAG_BETA_LOGITS) ? sigmoid_f(x) : x; }
+KDA_DEVICE float gate_in(float x, int flags) { return (flags & FLAG_GATE_LOGITS) ? sigmoid_f(x) : x; }
+KDA_DEVICE float g_in(float x, int flags) { return (flags & FLAG_CLAMP_G) ? fmaxf(x, kLogDecayFloor) : x; }
+
 KDA_DEVICE float warp_sum(float x) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);

@@ -26,7 +26,7 @@ __global__ void __launch_bounds__(256, 2)
     decode_step_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                        const T *__restrict__ g, const T *__restrict__ beta,
                        const T *__restrict__ gate, T *__restrict__ out, float *state, float scale,
-                       int qk_l2norm) {
+                       int flags) {
     constexpr int NT = 256;
     constexpr int COLG = DV / 4;       // float4 groups per state row
     constexpr int RPP = NT / COLG;     // rows covered by one pass of the CTA
@@ -54,11 +54,11 @@ __global__ void __launch_bounds__(256, 2)
     for (int i = tid; i < DK; i += NT) {
         sk[i] = ld(k + w * DK + i);
         sq[i] = ld(q + w * DK + i);
-        salpha[i] = __expf(ld(g + w * DK + i));
+        salpha[i] = __expf(g_in(ld(g + w * DK + i), flags));
     }
     for (int j = tid; j < DV; j += NT) {
         sv[j] = ld(v + w * DV + j);
-        sgate[j] = gate ? ld(gate + w * DV + j) : 1.0f;
+        sgate[j] = gate ? gate_in(ld(gate + w * DV + j), flags) : 1.0f;
     }
     __syncthreads();
     if (tid < 32) {
@@ -73,8 +73,8 @@ __global__ void __launch_bounds__(256, 2)
         qq = warp_sum(qq);
         kk = warp_sum(kk);
         if (tid == 0) {
-            const float rq = qk_l2norm ? rsqrtf(qq + 1e-6f) : 1.0f;
-            const float rk = qk_l2norm ? rsqrtf(kk + 1e-6f) : 1.0f;
+            const float rq = (flags & FLAG_L2NORM) ? rsqrtf(qq + 1e-6f) : 1.0f;
+            const float rk = (flags & FLAG_L2NORM) ? rsqrtf(kk + 1e-6f) : 1.0f;
             snorm[0] = rq;
             snorm[1] = rk;
             snorm[2] = kq * rq * rk;
@@ -104,7 +104,7 @@ __global__ void __launch_bounds__(256, 2)
             a += red_a[r][j];
             b += red_b[r][j];
         }
-        const float bt = ld(beta + w);
+        const float bt = beta_in(ld(beta + w), flags);
         const float u = bt * (sv[j] - a * rk);
         const float o = scale * (b * rq + kq * u);
         st(out + w * DV + j, sgate[j] * o);
@@ -126,33 +126,33 @@ __global__ void __launch_bounds__(256, 2)
 template <int DK, int DV, typename T>
 static cudaError_t launch_decode_t(const void *q, const void *k, const void *v, const void *g,
                                    const void *beta, const void *gate, void *out, float *state,
-                                   long nh, float scale, int l2, cudaStream_t st) {
+                                   long nh, float scale, int flags, cudaStream_t st) {
     decode_step_kernel<DK, DV, T><<<(unsigned)nh, 256, 0, st>>>(
         (const T *)q, (const T *)k, (const T *)v, (const T *)g, (const T *)beta, (const T *)gate,
-        (T *)out, state, scale, l2);
+        (T *)out, state, scale, flags);
     return cudaGetLastError();
 }
 
 template <typename T>
 static cudaError_t launch_decode_dt(int dk, int dv, const void *q, const void *k, const void *v,
                                     const void *g, const void *beta, const void *gate, void *out,
-                                    float *state, long nh, float scale, int l2, cudaStream_t st) {
+                                    float *state, long nh, float scale, int flags, cudaStream_t st) {
     if (dk == 128 && dv == 128)
-        return launch_decode_t<128, 128, T>(q, k, v, g, beta, gate, out, state, nh, scale, l2, st);
+        return launch_decode_t<128, 128, T>(q, k, v, g, beta, gate, out, state, nh, scale, flags, st);
     if (dk == 128 && dv == 64)
-        return launch_decode_t<128, 64, T>(q, k, v, g, beta, gate, out, state, nh, scale, l2, st);
+        return launch_decode_t<128, 64, T>(q, k, v, g, beta, gate, out, state, nh, scale, flags, st);
     if (dk == 64 && dv == 128)
-        return launch_decode_t<64, 128, T>(q, k, v, g, beta, gate, out, state, nh, scale, l2, st);
-    return launch_decode_t<64, 64, T>(q, k, v, g, beta, gate, out, state, nh, scale, l2, st);
+        return launch_decode_t<64, 128, T>(q, k, v, g, beta, gate, out, state, nh, scale, flags, st);
+    return launch_decode_t<64, 64, T>(q, k, v, g, beta, gate, out, state, nh, scale, flags, st);
 }
 
 cudaError_t launch_decode(bool bf16, int dk, int dv, const void *q, const void *k, const void *v,
                           const void *g, const void *beta, const void *gate, void *out,
-                          float *state, long nh, float scale, int l2, cudaStream_t st) {
+                          float *state, long nh, float scale, int flags, cudaStream_t st) {
     if (bf16)
         return launch_decode_dt<__nv_bfloat16>(dk, dv, q, k, v, g, beta, gate, out, state, nh,
-                                               scale, l2, st);
-    return launch_decode_dt<float>(dk, dv, q, k, v, g, beta, gate, out, state, nh, scale, l2, st);
+                                               scale, flags, st);
+    return launch_decode_dt<float>(dk, dv, q, k, v, g, beta, gate, out, state, nh, scale, flags, st);
 }
 
 }  // namespace kda

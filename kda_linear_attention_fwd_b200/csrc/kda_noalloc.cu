@@ -155,7 +155,10 @@ extern "C" int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v
     p.H = H;
     p.P_max = (int)P_max;
     p.scale = scale;
-    p.qk_l2norm = qk_l2norm;
+    p.flags = qk_l2norm;
+    p.snap_tokens = 0;
+    p.snapshots = nullptr;
+    p.snap_offsets = nullptr;
     p.total_tokens = total_tokens;
 
     const bool bf16 = dtype == KDA_DTYPE_BF16;

@@ -143,7 +143,39 @@ struct PrefillParams {
     int num_seqs, H, P_max;
     int total_tokens;
     float scale;
-    int qk_l2norm;
+    int flags;                    // FLAG_* bits (kda_common.cuh)
+    // state snapshots after every snap_tokens tokens of a sequence (0 = none):
+    // snapshot m (m = 1, 2, ... while m * snap_tokens < length) of sequence n
+    // and head h at snapshots[((snap_offsets[n] + m - 1) * H + h) * dk * dv]
+    int snap_tokens;
+    float *snapshots;
+    const int32_t *snap_offsets;
 };
+
+// Where the output pass of one (piece, head) writes state snapshots.
+struct Snap {
+    float *base = nullptr;  // first snapshot of this (sequence, head); null = none
+    size_t stride = 0;      // floats between consecutive snapshots of it
+    int pos0 = 0;           // position of the piece's first token in its sequence
+    int len = 0;            // sequence length
+    int every = 0;          // snapshot interval in tokens (a multiple of 16)
+    // The state after position pos_end - 1 goes here, or nowhere (null).
+    __device__ __forceinline__ float *at(int pos_end) const {
+        if (!base || pos_end % every != 0 || pos_end >= len) return nullptr;
+        return base + (size_t)(pos_end / every - 1) * stride;
+    }
+};
+__device__ __forceinline__ Snap make_snap(const PrefillParams &p, int n, int h, int t0, size_t dkdv) {
+    Snap sn;
+    if (p.snap_tokens > 0 && p.snapshots && p.snap_offsets) {
+        const int a = p.cu_seqlens[n], b = p.cu_seqlens[n + 1];
+        sn.base = p.snapshots + ((size_t)p.snap_offsets[n] * p.H + h) * dkdv;
+        sn.stride = (size_t)p.H * dkdv;
+        sn.pos0 = t0 - a;
+        sn.len = b - a;
+        sn.every = p.snap_tokens;
+    }
+    return sn;
+}
 
 }  // namespace kda

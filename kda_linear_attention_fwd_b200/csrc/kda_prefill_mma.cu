@@ -136,7 +136,8 @@ struct Layout {
 // identity, a copy of s_init ([DK][NC] fp32) or zeros and is written to s_out.
 template <int DK, int NC, bool OUT, bool USE_V>
 __device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const float *s_init,
-                          bool identity, float *s_out, unsigned char *smem_raw) {
+                          bool identity, float *s_out, unsigned char *smem_raw,
+                          const Snap &snap = Snap()) {
     using Lay = Layout<DK, NC>;
     constexpr int LK = Lay::LK, LC = Lay::LC, MT = Lay::MT, CW = Lay::CW, LY = Lay::LY;
     typename Lay::All &sm = *reinterpret_cast<typename Lay::All *>(smem_raw);
@@ -161,6 +162,7 @@ __device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const 
                                            : (s_init ? s_init[(size_t)i * NC + j] : 0.f);
                 }
         bf16 *out = (bf16 *)p.out;
+        const bool gate_logits = p.gate && (p.flags & FLAG_GATE_LOGITS);
         for (int c = 0; c < nchunks; ++c) {
             const int stg = c & (kStages - 1);
             bar_sync(BAR_FULL + stg, kBarCount);
@@ -241,6 +243,18 @@ __device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const 
                     mma16816(s[m][2 * np + 1], ua[m], bk[2], bk[3]);
                 }
             }
+            if (float *sp = snap.at(snap.pos0 + 16 * (c + 1))) {  // state snapshot after chunk c
+#pragma unroll
+                for (int m = 0; m < MT; ++m)
+#pragma unroll
+                    for (int nt = 0; nt < DK / 8; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int j = jb + 16 * m + g8 + (e >= 2 ? 8 : 0);
+                            const int i = 8 * nt + 2 * q4 + (e & 1);
+                            sp[(size_t)i * NC + j] = s[m][nt][e];
+                        }
+            }
             if (OUT) {
                 float *ys = sm.ys[warp];
 #pragma unroll
@@ -270,7 +284,8 @@ __device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const 
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const int jl = jl0 + 8 * v8 + 2 * e;
-                            const float2 gg = unpack_bf16(gw[e]);
+                            float2 gg = unpack_bf16(gw[e]);
+                            if (gate_logits) gg = make_float2(sigmoid_f(gg.x), sigmoid_f(gg.y));
                             pk[e] = pack_bf16(gg.x * ys[r * LY + jl], gg.y * ys[r * LY + jl + 1]);
                         }
                         *reinterpret_cast<uint4 *>(dst + 8 * v8) =
@@ -321,7 +336,7 @@ __device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const 
             if (OUT) cp_async16(&R.q[r * DK + cc * 8], q + off, ok);
         }
         cp_async_commit();
-        beta_next = lane < rows ? __bfloat162float(beta[(size_t)(tc + lane) * H + h]) : 0.f;
+        beta_next = lane < rows ? beta_in(__bfloat162float(beta[(size_t)(tc + lane) * H + h]), p.flags) : 0.f;
     };
     // v and gate of chunk c -> the stage itself (padded rows)
     auto issue_vg = [&](int c) {
@@ -347,7 +362,7 @@ __device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const 
         cp_async_wait<1>();  // raw q, k, g of chunk c have landed
         __syncwarp();
 
-        if (p.qk_l2norm) {  // 1/|q_r|, 1/|k_r| over the head dimension
+        if (p.flags & FLAG_L2NORM) {  // 1/|q_r|, 1/|k_r| over the head dimension
             for (int r = 0; r < 16; ++r) {
                 float kk = 0.f, qq = 0.f;
                 for (int i = lane; i < DK; i += 32) {
@@ -377,7 +392,7 @@ __device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const 
 #pragma unroll
             for (int r = 0; r < 16; ++r) {
                 const float2 gg = unpack_bf16(*reinterpret_cast<const uint32_t *>(&R.g[r * DK + i]));
-                e[r] = make_float2(__expf(gg.x), __expf(gg.y));
+                e[r] = make_float2(__expf(g_in(gg.x, p.flags)), __expf(g_in(gg.y, p.flags)));
             }
             float2 acc = make_float2(1.f, 1.f);
 #pragma unroll
@@ -392,7 +407,7 @@ __device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const 
 #pragma unroll
             for (int r = 15; r >= 0; --r) {
                 float2 kv = unpack_bf16(*reinterpret_cast<const uint32_t *>(&R.k[r * DK + i]));
-                if (p.qk_l2norm) { kv.x *= pr.rk[r]; kv.y *= pr.rk[r]; }
+                if (p.flags & FLAG_L2NORM) { kv.x *= pr.rk[r]; kv.y *= pr.rk[r]; }
                 *reinterpret_cast<uint32_t *>(&pr.kd[r * LK + i]) = pack_bf16(kv.x * E[r].x, kv.y * E[r].y);
                 *reinterpret_cast<uint32_t *>(&pr.ki[r * LK + i]) =
                     pack_bf16(kv.x * (F.x * invEl.x), kv.y * (F.y * invEl.y));
@@ -400,7 +415,7 @@ __device__ void run_piece(const PrefillParams &p, int t0, int len, int h, const 
                 if (OUT) {
                     float2 qv = unpack_bf16(*reinterpret_cast<const uint32_t *>(&R.q[r * DK + i]));
                     float sc = p.scale;
-                    if (p.qk_l2norm) sc *= pr.rq[r];
+                    if (p.flags & FLAG_L2NORM) sc *= pr.rq[r];
                     *reinterpret_cast<uint32_t *>(&S.qd[r * LK + i]) =
                         pack_bf16(qv.x * sc * E[r].x, qv.y * sc * E[r].y);
                 }
@@ -533,7 +548,8 @@ __global__ void __launch_bounds__(kThreads, 1) output_kernel(PrefillParams p) {
     const float *init = (np == 1) ? (p.initial_state ? p.initial_state + nh * DK * DV : nullptr)
                                   : p.Sin + ((size_t)pi * p.H + h) * DK * DV;
     float *fin = (j == np - 1 && p.final_state) ? p.final_state + nh * DK * DV : nullptr;
-    run_piece<DK, DV, true, true>(p, pc.y, pc.z, h, init, false, fin, smem);
+    run_piece<DK, DV, true, true>(p, pc.y, pc.z, h, init, false, fin, smem,
+                                  make_snap(p, n, h, pc.y, (size_t)DK * DV));
 }
 
 template <int DK, int DV>

@@ -41,7 +41,7 @@ struct SimtSmem {
 // zeros, and is written to s_out (if not null) at the end.
 template <int DK, int NC, bool OUT, bool USE_V, typename T>
 __device__ void simt_piece(const PrefillParams &p, int t0, int len, int h, const float *s_init,
-                           bool identity, float *s_out, float *smem) {
+                           bool identity, float *s_out, float *smem, const Snap &snap = Snap()) {
     constexpr int NT = 256;
     using L = SimtSmem<DK, NC>;
     constexpr int LDK = L::LDK, L16 = L::L16;
@@ -82,7 +82,7 @@ __device__ void simt_piece(const PrefillParams &p, int t0, int len, int h, const
             const bool ok = r < rows;
             const size_t o = ((size_t)(t0 + c0 + r) * H + h) * DK + i;
             Kd[r * LDK + i] = ok ? ld(k + o) : 0.f;
-            Gs[r * DK + i] = ok ? ld(g + o) : 0.f;
+            Gs[r * DK + i] = ok ? g_in(ld(g + o), p.flags) : 0.f;
             if (OUT) Qd[r * LDK + i] = ok ? ld(q + o) : 0.f;
         }
         constexpr int DV = NC;
@@ -91,11 +91,11 @@ __device__ void simt_piece(const PrefillParams &p, int t0, int len, int h, const
             const bool ok = r < rows;
             const size_t o = ((size_t)(t0 + c0 + r) * H + h) * DV + c;
             if (USE_V) V[idx] = ok ? ld(v + o) : 0.f;
-            if (OUT) GT[idx] = ok ? (gate ? ld(gate + o) : 1.f) : 0.f;
+            if (OUT) GT[idx] = ok ? (gate ? gate_in(ld(gate + o), p.flags) : 1.f) : 0.f;
         }
-        if (tid < 16) bet[tid] = tid < rows ? ld(beta + (size_t)(t0 + c0 + tid) * H + h) : 0.f;
+        if (tid < 16) bet[tid] = tid < rows ? beta_in(ld(beta + (size_t)(t0 + c0 + tid) * H + h), p.flags) : 0.f;
         __syncthreads();
-        if (p.qk_l2norm) {
+        if (p.flags & FLAG_L2NORM) {
             // warp w: rows 2w and 2w+1 -> rn[r] = 1/|q_r|, rn[16 + r] = 1/|k_r|
             const int lane = tid & 31, w = tid >> 5;
             for (int rr = 0; rr < 2; ++rr) {
@@ -130,12 +130,12 @@ __device__ void simt_piece(const PrefillParams &p, int t0, int len, int h, const
             for (int r = 0; r < 16; ++r) {
                 const float Gr = Gs[r * DK + i];
                 const float eG = expf(Gr), eN = expf(-Gr), eB = expf(Gl - Gr);
-                const float kv = Kd[r * LDK + i] * (p.qk_l2norm ? rn[16 + r] : 1.f);
+                const float kv = Kd[r * LDK + i] * ((p.flags & FLAG_L2NORM) ? rn[16 + r] : 1.f);
                 Kd[r * LDK + i] = kv * eG;
                 Ki[r * LDK + i] = kv * eN;
                 Kb[r * LDK + i] = kv * eB;
                 if (OUT) {
-                    const float qv = Qd[r * LDK + i] * (p.qk_l2norm ? rn[r] : 1.f) * p.scale;
+                    const float qv = Qd[r * LDK + i] * ((p.flags & FLAG_L2NORM) ? rn[r] : 1.f) * p.scale;
                     Qd[r * LDK + i] = qv * eG;
                 }
             }
@@ -204,6 +204,8 @@ __device__ void simt_piece(const PrefillParams &p, int t0, int len, int h, const
             for (int s = 0; s < 16; ++s) sv += Kb[s * LDK + i] * U[s * NC + c];
             S[idx] = sv;
         }
+        if (float *sp = snap.at(snap.pos0 + c0 + 16))  // same element mapping as the update
+            for (int idx = tid; idx < DK * NC; idx += NT) sp[idx] = S[idx];
         if (OUT) {
             for (int idx = tid; idx < 16 * NC; idx += NT) {
                 const int r = idx / NC, c = idx % NC;
@@ -256,7 +258,8 @@ __global__ void __launch_bounds__(256) simt_output_kernel(PrefillParams p) {
     const float *init = (np == 1) ? (p.initial_state ? p.initial_state + nh * DK * DV : nullptr)
                                   : p.Sin + ((size_t)pi * p.H + h) * DK * DV;
     float *fin = (j == np - 1 && p.final_state) ? p.final_state + nh * DK * DV : nullptr;
-    simt_piece<DK, DV, true, true, T>(p, pc.y, pc.z, h, init, false, fin, smem);
+    simt_piece<DK, DV, true, true, T>(p, pc.y, pc.z, h, init, false, fin, smem,
+                                      make_snap(p, n, h, pc.y, (size_t)DK * DV));
 }
 
 template <int DK, int DV, typename T>

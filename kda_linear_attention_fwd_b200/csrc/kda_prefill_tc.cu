@@ -154,7 +154,8 @@ KDA_DEVICE T *at_bytes(T *base, uint32_t off) {
 // is written to s_out.  The fp32 state lives in tensor memory.
 template <int DK, bool OUT, bool USE_V, bool L2N>
 __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, int len, int h,
-                          const float *s_init, bool identity, float *s_out, unsigned char *smem_raw) {
+                          const float *s_init, bool identity, float *s_out, unsigned char *smem_raw,
+                          const Snap &snap = Snap()) {
     using Lay = Layout<DK>;
     typename Lay::All &sm = *reinterpret_cast<typename Lay::All *>(
         smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
@@ -196,6 +197,7 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
         constexpr uint32_t ID_UP = idesc_bf16(128, 16, 0, 0);
         const bf16 *gate = (const bf16 *)p.gate;
         bf16 *out = (bf16 *)p.out;
+        const bool gate_logits = gate && (p.flags & FLAG_GATE_LOGITS);
 
         bool ok = true;
         // gate of this thread's column for the chunk whose output is pending;
@@ -226,8 +228,11 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
                 tmem_ld16_wait(t_d1 + 32 * (c & 1) + 16, o);
                 bf16 *tile = sm.io[c & 1];
 #pragma unroll
-                for (int t = 0; t < 16; ++t)
-                    tile[t * NC + j] = __float2bfloat16_rn(__bfloat162float(tile[t * NC + j]) * __uint_as_float(o[t]));
+                for (int t = 0; t < 16; ++t) {
+                    float gv = __bfloat162float(tile[t * NC + j]);
+                    if (gate_logits) gv = sigmoid_f(gv);
+                    tile[t * NC + j] = __float2bfloat16_rn(gv * __uint_as_float(o[t]));
+                }
             }
         };
         // the y tile of chunk c -> global (after a warpgroup barrier)
@@ -248,7 +253,7 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
         // a next chunk exists, the state is pre-scaled by that chunk's
         // exp(G_C) so that its MMA 3 can accumulate U^T Kb straight into it.
         // src: nullptr = read the state from TMEM; else an initial state.
-        auto state_pass = [&](const float *gam_next, bool from_init) {
+        auto state_pass = [&](const float *gam_next, bool from_init, float *snap_out) {
 #pragma unroll 1
             for (int cb = 0; cb < DK / 32; ++cb) {
                 uint32_t d[32];
@@ -261,6 +266,10 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
                     }
                 } else {
                     tmem_ld32_wait(t_s + 32 * cb, d);
+                    if (snap_out) {  // a state snapshot after this chunk
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) snap_out[(size_t)(32 * cb + e) * NC + j] = __uint_as_float(d[e]);
+                    }
                 }
                 uint32_t pk[16];
 #pragma unroll
@@ -303,7 +312,7 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
             }
         } else {
             bar_sync(BAR_FULL + 0, kBarCount);  // stage of chunk 0: its exp(G_C)
-            state_pass(sm.st[0].gam, true);
+            state_pass(sm.st[0].gam, true, nullptr);
         }
         // MMA operand descriptors of stage 0; stages are contiguous, so stage s
         // adds s * sizeof(Stage) / 16 to the start-address field (all of shared
@@ -385,7 +394,8 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
             bar_arrive(BAR_EMPTY + stg, kBarCount);  // every reader of this stage is done
             KDA_MARK(tid == 0 && c < 128, c * 16 + 10);
             if (ok) {
-                state_pass(has_next ? sm.st[(c + 1) % kStages].gam : nullptr, false);
+                state_pass(has_next ? sm.st[(c + 1) % kStages].gam : nullptr, false,
+                           snap.at(snap.pos0 + 16 * (c + 1)));
             } else {
                 tc_fence_before();
             }
@@ -460,7 +470,7 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
                     }
                 }
             }
-            if (d < 16) pr.beta[stg][d] = __bfloat162float(__ushort_as_bfloat16(bq0));
+            if (d < 16) pr.beta[stg][d] = beta_in(__bfloat162float(__ushort_as_bfloat16(bq0)), p.flags);
             __syncwarp();
             bar_sync(BAR_DPAIR, kPair);             // the tiles (with cleared rows) are visible
             KDA_MARK(d == 0 && c < 128, 2048 + c * 8 + 2);
@@ -490,7 +500,7 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
 #pragma unroll
             for (int r = 0; r < 16; ++r) {
                 const float2 gg = unpack_bf16(*reinterpret_cast<const uint32_t *>(Wk.g + sw128(r, ip)));
-                e[r] = make_float2(__expf(gg.x), __expf(gg.y));
+                e[r] = make_float2(__expf(g_in(gg.x, p.flags)), __expf(g_in(gg.y, p.flags)));
             }
             {
                 float2 acc = make_float2(1.f, 1.f);
@@ -736,7 +746,8 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSM) output_kernel(PrefillP
     const float *init = (np == 1) ? (p.initial_state ? p.initial_state + nh * DK * NC : nullptr)
                                   : p.Sin + ((size_t)pi * p.H + h) * DK * NC;
     float *fin = (j == np - 1 && p.final_state) ? p.final_state + nh * DK * NC : nullptr;
-    run_piece<DK, true, true, L2N>(p, maps, pc.y, pc.z, h, init, false, fin, smem);
+    run_piece<DK, true, true, L2N>(p, maps, pc.y, pc.z, h, init, false, fin, smem,
+                                   make_snap(p, n, h, pc.y, (size_t)DK * NC));
 }
 
 }  // namespace tc5
@@ -797,7 +808,7 @@ cudaError_t launch_tc5(const PrefillParams &p, bool summaries, cudaStream_t st) 
 }  // namespace
 
 cudaError_t launch_prefill_tc5(const PrefillParams &p, bool summaries, cudaStream_t st) {
-    return p.qk_l2norm ? launch_tc5<true>(p, summaries, st) : launch_tc5<false>(p, summaries, st);
+    return (p.flags & FLAG_L2NORM) ? launch_tc5<true>(p, summaries, st) : launch_tc5<false>(p, summaries, st);
 }
 
 }  // namespace kda

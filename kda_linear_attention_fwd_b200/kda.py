@@ -19,7 +19,10 @@ KDA_DTYPE_F32 = 0
 KDA_DTYPE_BF16 = 1
 
 EXPORTS = ("kda_status_string", "kda_chunk_fwd_workspace_size", "kda_chunk_fwd_plan",
-           "kda_chunk_fwd", "kda_decode_step")
+           "kda_chunk_fwd", "kda_decode_step", "kda_chunk_fwd_ex", "kda_decode_step_ex")
+
+# flags of the extended entry points (include/kda.h)
+FLAG_QK_L2NORM, FLAG_BETA_LOGITS, FLAG_GATE_LOGITS, FLAG_CLAMP_DECAY = 1, 2, 4, 8
 
 _lib = None
 
@@ -52,6 +55,12 @@ def load(path: str = LIB_PATH):
     lib.kda_decode_step.argtypes = [P, P, P, P, P, P, P, P, i32, i32, i32, i32, ctypes.c_int,
                                     f32, i32, P]
     lib.kda_decode_step.restype = ctypes.c_int
+    lib.kda_chunk_fwd_ex.argtypes = [P, P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32,
+                                     ctypes.c_int, f32, i32, P, P, i32, P, P, P, sz, P]
+    lib.kda_chunk_fwd_ex.restype = ctypes.c_int
+    lib.kda_decode_step_ex.argtypes = [P, P, P, P, P, P, P, P, i32, i32, i32, i32, ctypes.c_int,
+                                       f32, i32, P]
+    lib.kda_decode_step_ex.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -101,11 +110,28 @@ def plan(total_tokens, num_seqs, H) -> dict:
     return dict(piece_len=L.value, max_pieces=P.value, launches=n.value)
 
 
+def _flags(qk_l2norm, beta_logits, gate_logits, clamp_decay):
+    return ((FLAG_QK_L2NORM if qk_l2norm else 0) | (FLAG_BETA_LOGITS if beta_logits else 0) |
+            (FLAG_GATE_LOGITS if gate_logits else 0) | (FLAG_CLAMP_DECAY if clamp_decay else 0))
+
+
+def snapshot_offsets(lengths, snapshot_tokens):
+    """Running sums of the per-sequence snapshot counts (L - 1) // B."""
+    offs = [0]
+    for L in lengths:
+        offs.append(offs[-1] + (max(int(L), 1) - 1) // snapshot_tokens)
+    return offs
+
+
 def chunk_fwd(q, k, v, g, beta, gate, cu_seqlens, *, scale=1.0, qk_l2norm=False,
               initial_state=None, final_state=None, out=None, workspace=None,
-              cu_seqlens_host=None, output_final_state=True, stream=None):
+              cu_seqlens_host=None, output_final_state=True, stream=None,
+              beta_logits=False, gate_logits=False, clamp_decay=False, snapshot_tokens=0):
     """Prefill over packed sequences.  q, k, g [T, H, dk]; v, gate [T, H, dv];
-    beta [T, H]; cu_seqlens int32 [N+1] (device).  Returns (out, final_state)."""
+    beta [T, H]; cu_seqlens int32 [N+1] (device).  Returns (out, final_state),
+    plus the snapshots [count, H, dk, dv] fp32 when snapshot_tokens > 0 (the
+    state after every snapshot_tokens tokens of each sequence, sequence-major;
+    needs the offsets on the host: cu_seqlens_host, else one device read)."""
     lib = load()
     _require_cuda(q, k, v, g, beta, gate, cu_seqlens, initial_state, final_state, out, workspace)
     T, H, dk = q.shape
@@ -123,17 +149,34 @@ def chunk_fwd(q, k, v, g, beta, gate, cu_seqlens, *, scale=1.0, qk_l2norm=False,
     if cu_seqlens_host is not None:
         host_arr = (ctypes.c_int32 * len(cu_seqlens_host))(*[int(x) for x in cu_seqlens_host])
         host = ctypes.cast(host_arr, ctypes.c_void_p)
-    st = lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(gate), _ptr(out),
-                           _ptr(cu_seqlens), host, N, T, H, dk, dv, code, float(scale),
-                           int(bool(qk_l2norm)), _ptr(initial_state), _ptr(final_state),
-                           _ptr(workspace), workspace.numel() * workspace.element_size(),
-                           _stream(stream))
-    _check("kda_chunk_fwd", st)
+    flags = _flags(qk_l2norm, beta_logits, gate_logits, clamp_decay)
+    if flags & ~FLAG_QK_L2NORM == 0 and not snapshot_tokens:
+        st = lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(gate),
+                               _ptr(out), _ptr(cu_seqlens), host, N, T, H, dk, dv, code,
+                               float(scale), flags, _ptr(initial_state), _ptr(final_state),
+                               _ptr(workspace), workspace.numel() * workspace.element_size(),
+                               _stream(stream))
+        _check("kda_chunk_fwd", st)
+        return out, final_state
+    snaps = offs_dev = None
+    if snapshot_tokens:
+        cu = list(cu_seqlens_host) if cu_seqlens_host is not None else cu_seqlens.tolist()
+        offs = snapshot_offsets([cu[i + 1] - cu[i] for i in range(N)], snapshot_tokens)
+        offs_dev = torch.tensor(offs, dtype=torch.int32, device=q.device)
+        snaps = torch.empty(max(offs[-1], 1), H, dk, dv, dtype=torch.float32, device=q.device)
+    st = lib.kda_chunk_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(gate),
+                              _ptr(out), _ptr(cu_seqlens), host, N, T, H, dk, dv, code,
+                              float(scale), flags, _ptr(initial_state), _ptr(final_state),
+                              int(snapshot_tokens), _ptr(snaps), _ptr(offs_dev), _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("kda_chunk_fwd_ex", st)
+    if snapshot_tokens:
+        return out, final_state, snaps[:offs[-1]]
     return out, final_state
 
 
 def decode_step(q, k, v, g, beta, gate, state, *, scale=1.0, qk_l2norm=False, out=None,
-                stream=None):
+                stream=None, beta_logits=False, gate_logits=False, clamp_decay=False):
     """One token per sequence.  q, k, g [N, H, dk]; v, gate [N, H, dv]; beta
     [N, H]; state [N, H, dk, dv] fp32, updated in place.  Returns out."""
     lib = load()
@@ -142,8 +185,9 @@ def decode_step(q, k, v, g, beta, gate, state, *, scale=1.0, qk_l2norm=False, ou
     dv = v.shape[-1]
     if out is None:
         out = torch.empty(N, H, dv, dtype=q.dtype, device=q.device)
-    st = lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(gate),
-                             _ptr(out), _ptr(state), N, H, dk, dv, _dtype_code(q), float(scale),
-                             int(bool(qk_l2norm)), _stream(stream))
-    _check("kda_decode_step", st)
+    st = lib.kda_decode_step_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(gate),
+                                _ptr(out), _ptr(state), N, H, dk, dv, _dtype_code(q),
+                                float(scale), _flags(qk_l2norm, beta_logits, gate_logits,
+                                                     clamp_decay), _stream(stream))
+    _check("kda_decode_step_ex", st)
     return out

@@ -150,3 +150,44 @@ def test_binding_refuses_cpu_tensors():
     with pytest.raises((ValueError, RuntimeError)):
         kda.chunk_fwd(x, x, x, x, torch.zeros(16, 1, dtype=torch.bfloat16), None,
                       torch.tensor([0, 16], dtype=torch.int32))
+
+
+def call_fwd_ex(lib, **kw):
+    a = dict(q=A, k=A, v=A, g=A, beta=A, gate=None, out=A, cu=A, cu_host=None, N=1, T=16, H=1,
+             dk=64, dv=64, dtype=BF16, scale=1.0, flags=0, s0=None, s1=None, snap_tokens=0,
+             snaps=None, snap_offs=None, ws=A, ws_bytes=1 << 40, stream=None)
+    a.update(kw)
+    return lib.kda_chunk_fwd_ex(a["q"], a["k"], a["v"], a["g"], a["beta"], a["gate"], a["out"],
+                                a["cu"], a["cu_host"], a["N"], a["T"], a["H"], a["dk"], a["dv"],
+                                a["dtype"], a["scale"], a["flags"], a["s0"], a["s1"],
+                                a["snap_tokens"], a["snaps"], a["snap_offs"], a["ws"],
+                                a["ws_bytes"], a["stream"])
+
+
+def test_chunk_fwd_ex_validation(lib):
+    assert call_fwd_ex(lib, N=0, T=0) == OK
+    assert call_fwd_ex(lib, N=0, T=0, flags=15) == OK
+    assert call_fwd_ex(lib, flags=16) == INVALID
+    assert call_fwd_ex(lib, flags=-1) == INVALID
+    assert call_fwd_ex(lib, snap_tokens=8, snaps=A, snap_offs=A) == INVALID
+    assert call_fwd_ex(lib, snap_tokens=-16, snaps=A, snap_offs=A) == INVALID
+    assert call_fwd_ex(lib, snap_tokens=64) == INVALID          # no buffers
+    assert call_fwd_ex(lib, snap_tokens=64, snaps=A) == INVALID  # no offsets
+    assert call_fwd_ex(lib, snap_tokens=64, snaps=A + 8, snap_offs=A) == ALIGN
+    assert call_fwd_ex(lib, snap_tokens=64, snaps=A, snap_offs=A + 2) == ALIGN
+    assert call_fwd_ex(lib, flags=15, ws=None) == WORKSPACE     # flags accepted, then workspace
+    # the plain entry point still accepts only 0 / 1 for qk_l2norm
+    assert call_fwd(lib, l2=2) == INVALID
+
+
+def test_decode_ex_validation(lib):
+    f = lib.kda_decode_step_ex
+    args = [A, A, A, A, A, None, A, A, 4, 2, 128, 128, BF16, 1.0]
+    assert f(*args[:8], 0, 2, 128, 128, BF16, 1.0, 15, None) == OK  # no sequences
+    assert f(*args, 16, None) == INVALID
+    assert f(*args[:2], A + 2, *args[3:], 3, None) == ALIGN
+
+
+def test_snapshot_offsets_host_helper():
+    assert kda.snapshot_offsets([0, 5, 64, 300, 701], 64) == [0, 0, 0, 0, 4, 14]
+    assert kda.snapshot_offsets([65, 128, 129], 64) == [0, 1, 2, 4]
