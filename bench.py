@@ -230,6 +230,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-ex", action="store_true",
+                    help="skip the extended-path measurement (flags + state snapshots)")
     ap.add_argument("--out-dir", default=os.path.join(ROOT, "gpurun_out"))
     ap.add_argument("--ref-tokens", type=int, default=0,
                     help="reference arm: tokens per step sample (0 = scale with cores)")
@@ -300,6 +302,46 @@ def main():
                 "tensor_frac_of_peak": pflops / (ms / 1e3) / 1e12 / pk["bf16_tflops"],
                 "roofline_model_frac": max(pbytes / (hbm * 1e9),
                                            pflops / (pk["bf16_tflops"] * 1e12)) / (ms / 1e3)}
+
+    # ------- extended path: in-kernel preprocessing + snapshots, same inputs -------
+    exm = None
+    if not args.no_ex:
+        B = 8192  # a state snapshot every 8192 tokens of each sequence
+        offs = kda.snapshot_offsets([cu_host[i + 1] - cu_host[i] for i in range(N)], B)
+        offs_dev = torch.tensor(offs, dtype=torch.int32, device=dev)
+        snaps = torch.empty(max(offs[-1], 1), w.H, w.dk, w.dv, dtype=torch.float32, device=dev)
+        P = ctypes.c_void_p
+        ptr = lambda t: P(t.data_ptr())
+        cu_arr = (ctypes.c_int32 * len(cu_host))(*cu_host)
+        ex_args = (ptr(inp["q"]), ptr(inp["k"]), ptr(inp["v"]), ptr(inp["g"]), ptr(inp["beta"]),
+                   ptr(inp["gate"]), ptr(out), ptr(inp["cu_seqlens"]), ctypes.cast(cu_arr, P),
+                   N, T, w.H, w.dk, w.dv, kda._dtype_code(inp["q"]), 1.0, 15,
+                   None if inp["initial_state"] is None else ptr(inp["initial_state"]), ptr(fin),
+                   B, ptr(snaps), ptr(offs_dev), ptr(wsp), ws_bytes, P(stream.cuda_stream))
+
+        def ex_call():
+            rc = lib.kda_chunk_fwd_ex(*ex_args)
+            if rc != 0:
+                raise RuntimeError(kda.status_string(rc))
+
+        for _ in range(args.warmup):
+            ex_call()
+        torch.cuda.synchronize()
+        barrier(ws)
+        x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        x0.record(stream)
+        for _ in range(args.steps):
+            ex_call()
+        x1.record(stream)
+        torch.cuda.synchronize()
+        barrier(ws)
+        xms = reduce_max(x0.elapsed_time(x1), ws) / args.steps
+        exm = {"value": ws * T / (xms / 1e3), "unit": "tokens/s", "ms_per_step": xms,
+               "vs_plain_time": xms / ms, "flags": "qk_l2norm|beta_logits|gate_logits|clamp_decay",
+               "snapshot_tokens": B, "snapshots_per_head": offs[-1],
+               "snapshot_bytes": offs[-1] * w.H * w.dk * w.dv * 4,
+               "gpu_launches": plan["launches"] * args.steps}
+        del snaps, offs_dev
 
     # ---------------- decode ----------------
     dec = None
@@ -399,7 +441,8 @@ def main():
                            "l2": "inputs larger than L2 (%.1f GB per step)" % (pbytes / 1e9),
                            "piece_len": plan["piece_len"]},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": plan["launches"] * args.steps, "clocks": clk, "decode": dec}
+                "gpu_launches": plan["launches"] * args.steps, "clocks": clk, "decode": dec,
+                "extended": exm}
         print(json.dumps(line), flush=True)
     if ws > 1:
         import torch.distributed as dist

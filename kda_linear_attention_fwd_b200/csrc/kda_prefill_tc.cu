@@ -128,6 +128,7 @@ struct Layout {
         alignas(16) float AT[16 * 16];  // AT[s][r] = beta_r A[r][s], r > s (matrix pair)
         float beta[kStages][16];        // beta of the chunk in each stage
         float nk[2][16], nq[2][16];     // per decay warp and row: partial sums of k^2, q^2
+        float rk[16], rq[16];           // 1/|k_r| and scale/|q_r| of the chunk being decayed
     };
     struct All {
         Raw raw[kRaw];
@@ -230,7 +231,7 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
 #pragma unroll
                 for (int t = 0; t < 16; ++t) {
                     float gv = __bfloat162float(tile[t * NC + j]);
-                    if (gate_logits) gv = sigmoid_f(gv);
+                    if (gate_logits) gv = sigmoid_fast(gv);
                     tile[t * NC + j] = __float2bfloat16_rn(gv * __uint_as_float(o[t]));
                 }
             }
@@ -475,20 +476,30 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
             bar_sync(BAR_DPAIR, kPair);             // the tiles (with cleared rows) are visible
             KDA_MARK(d == 0 && c < 128, 2048 + c * 8 + 2);
             if (L2N) {  // row norms of k and q: the two warps cover all channels
+                float sk[16], sq[16];
 #pragma unroll
                 for (int r = 0; r < 16; ++r) {
                     const float2 kv = unpack_bf16(*reinterpret_cast<const uint32_t *>(Wk.k + sw128(r, ip)));
-                    float sk = kv.x * kv.x + kv.y * kv.y, sq = 0.f;
+                    sk[r] = kv.x * kv.x + kv.y * kv.y;
+                    sq[r] = 0.f;
                     if (OUT) {
                         const float2 qv = unpack_bf16(*reinterpret_cast<const uint32_t *>(Wk.q + sw128(r, ip)));
-                        sq = qv.x * qv.x + qv.y * qv.y;
+                        sq[r] = qv.x * qv.x + qv.y * qv.y;
                     }
-                    sk = warp_sum(sk);
-                    sq = warp_sum(sq);
-                    if (lane == 0) {
-                        pr.nk[dw][r] = sk;
-                        pr.nq[dw][r] = sq;
-                    }
+                }
+                const float tk = warp_sum16_scatter(sk, lane);
+                const float tq = OUT ? warp_sum16_scatter(sq, lane) : 0.f;
+                if (!(lane & 1)) {
+                    pr.nk[dw][row_of_lane(lane)] = tk;
+                    pr.nq[dw][row_of_lane(lane)] = tq;
+                }
+                __syncwarp();
+                bar_sync(BAR_DPAIR, kPair);
+                if (d < 32) {  // 1/|k_r| and scale/|q_r|, once per row
+                    const int r = d & 15;
+                    float *dst = d < 16 ? pr.rk : pr.rq;
+                    const float (*src)[16] = d < 16 ? pr.nk : pr.nq;
+                    dst[r] = rsqrtf(src[0][r] + src[1][r] + 1e-6f) * (d < 16 ? 1.f : p.scale);
                 }
                 __syncwarp();
                 bar_sync(BAR_DPAIR, kPair);
@@ -521,9 +532,9 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
                 float2 kv = unpack_bf16(*reinterpret_cast<const uint32_t *>(Wk.k + sw128(r, ip)));
                 float sc = p.scale;
                 if (L2N) {
-                    const float rk = rsqrtf(pr.nk[0][r] + pr.nk[1][r] + 1e-6f);
+                    const float rk = pr.rk[r];
                     kv = f2mul(kv, make_float2(rk, rk));
-                    sc *= rsqrtf(pr.nq[0][r] + pr.nq[1][r] + 1e-6f);
+                    sc = pr.rq[r];
                 }
                 *reinterpret_cast<uint32_t *>(Wk.k + sw128(r, ip)) = pack_bf16(f2mul(kv, E[r]));
                 *reinterpret_cast<uint32_t *>(Wk.g + sw128(r, ip)) = pack_bf16(f2mul(kv, f2mul(F, invEl)));

@@ -46,6 +46,35 @@ KDA_DEVICE float2 f2fma(float2 a, float2 b, float2 c) {
 }
 KDA_DEVICE uint32_t pack_bf16(float2 v) { return pack_bf16(v.x, v.y); }
 
+// Sixteen per-lane values summed over the warp, element i landing in the
+// lanes whose bits 4..1 spell i (lanes 2i' and 2i'+1 with i' the bit-reversed
+// index below): each halving step keeps half of the values and adds the
+// partner's other half, 8 + 4 + 2 + 1 + 1 shuffles in all.  Returns the sum of
+// element row_of_lane(lane).
+KDA_DEVICE int row_of_lane(int lane) {
+    return ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
+}
+KDA_DEVICE float warp_sum16_scatter(float (&v)[16], int lane) {
+#pragma unroll
+    for (int w = 8, m = 16; w >= 1; w >>= 1, m >>= 1) {
+        const bool up = lane & m;  // this lane keeps the upper half of the live values
+#pragma unroll
+        for (int i = 0; i < w; ++i) {
+            const float keep = up ? v[i + w] : v[i];
+            const float give = up ? v[i] : v[i + w];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, give, m);
+        }
+    }
+    return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
+}
+// 1 / (1 + exp(-x)) as 0.5 + 0.5 tanh(x / 2) with the hardware tanh
+// approximation (one special-function instruction).
+KDA_DEVICE float sigmoid_fast(float x) {
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
+    return fmaf(0.5f, t, 0.5f);
+}
+
 // ---- warp-level MMA (m16n8k16, bf16 in, fp32 accumulate) and ldmatrix
 KDA_DEVICE void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
     asm volatile(
