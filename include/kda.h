@@ -222,6 +222,46 @@ int kda_decode_step_ex(const void *q, const void *k, const void *v, const void *
                        int32_t dk, int32_t dv, kda_dtype dtype, float scale, int32_t flags,
                        kda_stream_t stream);
 
+/*
+ * Context parallelism (affta.cn page, section "KDA 上下文并行，让上下文的交接变薄";
+ * prism.simon-ai.net page, section "Linear Attention 的分层 Chunking 策略"):
+ * the tokens of a sequence segment act on an incoming state as one affine
+ * map S -> transition * S + zero_state, of fixed size whatever the segment's
+ * length.  A sequence split over devices exchanges only these maps; each
+ * device folds the maps of the segments before its own into its incoming
+ * state (kda_state_compose) and runs kda_chunk_fwd from there.
+ *
+ * kda_chunk_fwd_summary: the map of every sequence of a packed batch.
+ *   k, v, g, beta, cu_seqlens, cu_seqlens_host, sizes, dtype: as kda_chunk_fwd
+ *                 (q and gate are not needed: the map does not depend on them).
+ *   flags         KDA_FLAG_* (the gate flag has no effect here).
+ *   transition    device fp32 [num_seqs][H][dk][dk], written.
+ *   zero_state    device fp32 [num_seqs][H][dk][dv], written: the state the
+ *                 sequence's tokens produce from zero.
+ *   workspace     >= kda_chunk_fwd_workspace_size(total_tokens, num_seqs, H,
+ *                 dk, dv, dtype) bytes.
+ * An empty sequence has the identity map.  Errors as kda_chunk_fwd.
+ */
+int kda_chunk_fwd_summary(const void *k, const void *v, const void *g, const void *beta,
+                          const int32_t *cu_seqlens, const int32_t *cu_seqlens_host,
+                          int32_t num_seqs, int32_t total_tokens, int32_t H, int32_t dk, int32_t dv,
+                          kda_dtype dtype, int32_t flags, float *transition, float *zero_state,
+                          void *workspace, size_t workspace_bytes, kda_stream_t stream);
+
+/*
+ * kda_state_compose: state_out = map[count-1]( ... map[0](state_in) ...) for
+ * every (sequence, head), map[i](S) = transitions[i] S + zero_states[i], fp32.
+ *   transitions   device fp32 [count][num_seqs][H][dk][dk].
+ *   zero_states   device fp32 [count][num_seqs][H][dk][dv].
+ *   state_in      device fp32 [num_seqs][H][dk][dv]; NULL = zeros.
+ *   state_out     device fp32 [num_seqs][H][dk][dv]; may alias state_in
+ *                 exactly, no partial overlap (KDA_ERR_INVALID_ARG).
+ * count = 0 copies state_in (or writes zeros).  All pointers 16-byte aligned.
+ */
+int kda_state_compose(const float *transitions, const float *zero_states, int32_t count,
+                      const float *state_in, float *state_out, int32_t num_seqs, int32_t H,
+                      int32_t dk, int32_t dv, kda_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -131,7 +131,7 @@ int kda_chunk_fwd_ex(const void *q, const void *k, const void *v, const void *g,
     if (!workspace || workspace_bytes < WL.total) return KDA_ERR_WORKSPACE;
 
     char *ws = (char *)workspace;
-    kda::PrefillParams p;
+    kda::PrefillParams p{};
     p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.gate = gate; p.out = out;
     p.cu_seqlens = cu_seqlens;
     p.header = (const int32_t *)(ws + WL.off_header);

@@ -139,7 +139,7 @@ extern "C" int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v
     if (rc != KDA_OK) return rc;
     char *ws = (char *)scratch;
 
-    kda::PrefillParams p;
+    kda::PrefillParams p{};
     p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.gate = gate; p.out = out;
     p.cu_seqlens = cu_seqlens;
     p.header = (const int32_t *)(ws + WL.off_header);

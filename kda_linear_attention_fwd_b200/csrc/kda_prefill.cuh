@@ -150,6 +150,9 @@ struct PrefillParams {
     int snap_tokens;
     float *snapshots;
     const int32_t *snap_offsets;
+    // summary pass over every piece (both parts), for the per-sequence affine
+    // map of kda_chunk_fwd_summary; 0 = the prefill's own summary pass
+    int summarize_all;
 };
 
 // Where the output pass of one (piece, head) writes state snapshots.

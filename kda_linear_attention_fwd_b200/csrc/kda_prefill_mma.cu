@@ -521,7 +521,7 @@ __global__ void __launch_bounds__(kThreads, 1) summary_kernel(PrefillParams p) {
     if (pc.x < 0) return;
     const int n = pc.x, j = pc.w;
     const int np = p.seq_first[n + 1] - p.seq_first[n];
-    if (j >= np - 1) return;
+    if (!p.summarize_all && j >= np - 1) return;
     const size_t ph = (size_t)pi * p.H + h;
     if (blockIdx.y == 0) {
         const float *init = (j == 0 && p.initial_state)
@@ -529,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1) summary_kernel(PrefillParams p) {
                                 : nullptr;
         run_piece<DK, DV, false, true>(p, pc.y, pc.z, h, init, false, p.Szero + ph * DK * DV, smem);
     } else {
-        if (j == 0) return;
+        if (!p.summarize_all && j == 0) return;
         run_piece<DK, DK, false, false>(p, pc.y, pc.z, h, nullptr, true, p.M + ph * DK * DK, smem);
     }
 }

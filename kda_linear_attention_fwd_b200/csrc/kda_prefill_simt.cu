@@ -229,7 +229,7 @@ __global__ void __launch_bounds__(256) simt_summary_kernel(PrefillParams p) {
     if (pc.x < 0) return;
     const int n = pc.x, j = pc.w;
     const int np = p.seq_first[n + 1] - p.seq_first[n];
-    if (j >= np - 1) return;
+    if (!p.summarize_all && j >= np - 1) return;
     const size_t ph = (size_t)pi * p.H + h;
     if (blockIdx.y == 0) {
         const float *init = (j == 0 && p.initial_state)
@@ -238,7 +238,7 @@ __global__ void __launch_bounds__(256) simt_summary_kernel(PrefillParams p) {
         simt_piece<DK, DV, false, true, T>(p, pc.y, pc.z, h, init, false,
                                            p.Szero + ph * DK * DV, smem);
     } else {
-        if (j == 0) return;
+        if (!p.summarize_all && j == 0) return;
         simt_piece<DK, DK, false, false, T>(p, pc.y, pc.z, h, nullptr, true, p.M + ph * DK * DK,
                                             smem);
     }

@@ -730,7 +730,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSM) summary_kernel(Prefill
     if (pc.x < 0) return;
     const int n = pc.x, j = pc.w;
     const int np = p.seq_first[n + 1] - p.seq_first[n];
-    if (j >= np - 1) return;
+    if (!p.summarize_all && j >= np - 1) return;
     const size_t ph = (size_t)pi * p.H + h;
     if (blockIdx.y == 0) {
         const float *init = (j == 0 && p.initial_state)
@@ -738,7 +738,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSM) summary_kernel(Prefill
                                 : nullptr;
         run_piece<DK, false, true, L2N>(p, maps, pc.y, pc.z, h, init, false, p.Szero + ph * DK * NC, smem);
     } else {
-        if (j == 0) return;
+        if (!p.summarize_all && j == 0) return;
         run_piece<DK, false, false, L2N>(p, maps, pc.y, pc.z, h, nullptr, true, p.M + ph * DK * DK, smem);
     }
 }

@@ -19,7 +19,8 @@ KDA_DTYPE_F32 = 0
 KDA_DTYPE_BF16 = 1
 
 EXPORTS = ("kda_status_string", "kda_chunk_fwd_workspace_size", "kda_chunk_fwd_plan",
-           "kda_chunk_fwd", "kda_decode_step", "kda_chunk_fwd_ex", "kda_decode_step_ex")
+           "kda_chunk_fwd", "kda_decode_step", "kda_chunk_fwd_ex", "kda_decode_step_ex",
+           "kda_chunk_fwd_summary", "kda_state_compose")
 
 # flags of the extended entry points (include/kda.h)
 FLAG_QK_L2NORM, FLAG_BETA_LOGITS, FLAG_GATE_LOGITS, FLAG_CLAMP_DECAY = 1, 2, 4, 8
@@ -61,6 +62,11 @@ def load(path: str = LIB_PATH):
     lib.kda_decode_step_ex.argtypes = [P, P, P, P, P, P, P, P, i32, i32, i32, i32, ctypes.c_int,
                                        f32, i32, P]
     lib.kda_decode_step_ex.restype = ctypes.c_int
+    lib.kda_chunk_fwd_summary.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, ctypes.c_int,
+                                          i32, P, P, P, sz, P]
+    lib.kda_chunk_fwd_summary.restype = ctypes.c_int
+    lib.kda_state_compose.argtypes = [P, P, i32, P, P, i32, i32, i32, i32, P]
+    lib.kda_state_compose.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -190,4 +196,48 @@ def decode_step(q, k, v, g, beta, gate, state, *, scale=1.0, qk_l2norm=False, ou
                                 float(scale), _flags(qk_l2norm, beta_logits, gate_logits,
                                                      clamp_decay), _stream(stream))
     _check("kda_decode_step_ex", st)
+    return out
+
+
+def chunk_summary(k, v, g, beta, cu_seqlens, *, qk_l2norm=False, beta_logits=False,
+                  clamp_decay=False, cu_seqlens_host=None, workspace=None, stream=None):
+    """The affine map S -> M S + Z of every sequence's tokens.  k, g [T, H, dk];
+    v [T, H, dv]; beta [T, H].  Returns (M [N, H, dk, dk], Z [N, H, dk, dv]) fp32."""
+    lib = load()
+    _require_cuda(k, v, g, beta, cu_seqlens, workspace)
+    T, H, dk = k.shape
+    dv = v.shape[-1]
+    N = cu_seqlens.shape[0] - 1
+    code = _dtype_code(k)
+    M = torch.empty(N, H, dk, dk, dtype=torch.float32, device=k.device)
+    Z = torch.empty(N, H, dk, dv, dtype=torch.float32, device=k.device)
+    need = int(lib.kda_chunk_fwd_workspace_size(T, N, H, dk, dv, code))
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=k.device)
+    host = None
+    if cu_seqlens_host is not None:
+        host_arr = (ctypes.c_int32 * len(cu_seqlens_host))(*[int(x) for x in cu_seqlens_host])
+        host = ctypes.cast(host_arr, ctypes.c_void_p)
+    st = lib.kda_chunk_fwd_summary(_ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), host,
+                                   N, T, H, dk, dv, code,
+                                   _flags(qk_l2norm, beta_logits, False, clamp_decay),
+                                   _ptr(M), _ptr(Z), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("kda_chunk_fwd_summary", st)
+    return M, Z
+
+
+def state_compose(M, Z, state_in=None, *, out=None, stream=None):
+    """Apply the maps (M [R, N, H, dk, dk], Z [R, N, H, dk, dv]) in order to
+    state_in [N, H, dk, dv] (None = zeros).  Returns the state."""
+    lib = load()
+    _require_cuda(M, Z, state_in, out)
+    R, N, H, dk, _ = M.shape
+    dv = Z.shape[-1]
+    M, Z = M.contiguous(), Z.contiguous()
+    if out is None:
+        out = torch.empty(N, H, dk, dv, dtype=torch.float32, device=M.device)
+    st = lib.kda_state_compose(_ptr(M), _ptr(Z), R, _ptr(state_in), _ptr(out), N, H, dk, dv,
+                               _stream(stream))
+    _check("kda_state_compose", st)
     return out

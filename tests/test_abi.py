@@ -191,3 +191,22 @@ def test_decode_ex_validation(lib):
 def test_snapshot_offsets_host_helper():
     assert kda.snapshot_offsets([0, 5, 64, 300, 701], 64) == [0, 0, 0, 0, 4, 14]
     assert kda.snapshot_offsets([65, 128, 129], 64) == [0, 1, 2, 4]
+
+
+def test_summary_and_compose_validation(lib):
+    s = lib.kda_chunk_fwd_summary
+    base = [A, A, A, A, A, None, 1, 16, 1, 64, 64, BF16, 0, A, A, A, 1 << 40, None]
+    assert s(*base[:6], 0, 0, *base[8:]) == OK                   # no sequences
+    assert s(*base[:12], 16, *base[13:]) == INVALID               # unknown flag
+    assert s(*base[:13], None, *base[14:]) == INVALID             # no transition buffer
+    assert s(*base[:13], A + 4, *base[14:]) == ALIGN
+    assert s(*base[:15], None, *base[16:]) == WORKSPACE
+    assert s(*base[:9], 96, *base[10:]) == UNSUPPORTED
+    c = lib.kda_state_compose
+    assert c(A, A, 2, A, A, 0, 1, 64, 64, None) == OK               # no sequences
+    assert c(A, A, -1, A, A, 1, 1, 64, 64, None) == INVALID
+    assert c(A, A, 1, A, None, 1, 1, 64, 64, None) == INVALID       # no output
+    assert c(None, A, 1, A, A, 1, 1, 64, 64, None) == INVALID       # maps missing
+    assert c(A, A, 1, A, A + 8, 1, 1, 64, 64, None) == ALIGN
+    assert c(A, A, 1, A, A + 256, 1, 1, 64, 64, None) == INVALID    # partial overlap
+    assert c(A, A, 1, A, A, 1, 1, 32, 64, None) == UNSUPPORTED
