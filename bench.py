@@ -230,6 +230,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-kcp", action="store_true",
+                    help="skip the per-rank context-parallel measurement")
     ap.add_argument("--no-ex", action="store_true",
                     help="skip the extended-path measurement (flags + state snapshots)")
     ap.add_argument("--out-dir", default=os.path.join(ROOT, "gpurun_out"))
@@ -343,6 +345,51 @@ def main():
                "gpu_launches": plan["launches"] * args.steps}
         del snaps, offs_dev
 
+    # ------- context parallelism: what one rank of an 8-way split runs -------
+    # (measured on this GPU: the map of its segment, the fold of the 7 maps
+    # before it, the prefill of its segment; the all-gather is not timed here)
+    kcpm = None
+    if not args.no_kcp and N == 1:
+        R = 8
+        seg = T // R
+        sl = slice((R - 1) * seg, R * seg)  # the last rank folds the most maps
+        sk = {x: inp[x][sl].contiguous() for x in ("q", "k", "v", "g", "beta", "gate")}
+        scu = torch.tensor([0, seg], dtype=torch.int32, device=dev)
+        scu_h = [0, seg]
+        Mz = torch.zeros(R - 1, 1, w.H, w.dk, w.dk, device=dev)
+        Zz = torch.zeros(R - 1, 1, w.H, w.dk, w.dv, device=dev)
+        sout = torch.empty(seg, w.H, w.dv, dtype=w.torch_dtype, device=dev)
+        sfin = torch.empty(1, w.H, w.dk, w.dv, device=dev)
+
+        def t_ms(fn, reps):
+            for _ in range(2):
+                fn()
+            torch.cuda.synchronize()
+            c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            c0.record(stream)
+            for _ in range(reps):
+                fn()
+            c1.record(stream)
+            torch.cuda.synchronize()
+            return reduce_max(c0.elapsed_time(c1), ws) / reps
+
+        ms_sum = t_ms(lambda: kda.chunk_summary(sk["k"], sk["v"], sk["g"], sk["beta"], scu,
+                                                cu_seqlens_host=scu_h, workspace=wsp,
+                                                stream=stream), args.steps)
+        s_in = torch.zeros(1, w.H, w.dk, w.dv, device=dev)
+        ms_cmp = t_ms(lambda: kda.state_compose(Mz, Zz, s_in, stream=stream), args.steps)
+        ms_pre = t_ms(lambda: kda.chunk_fwd(sk["q"], sk["k"], sk["v"], sk["g"], sk["beta"],
+                                            sk["gate"], scu, initial_state=s_in, final_state=sfin,
+                                            out=sout, workspace=wsp, cu_seqlens_host=scu_h,
+                                            stream=stream), args.steps)
+        per_rank = ms_sum + ms_cmp + ms_pre
+        kcpm = {"ranks_emulated": R, "segment_tokens": seg, "summary_ms": ms_sum,
+                "fold_ms": ms_cmp, "segment_prefill_ms": ms_pre, "per_rank_ms": per_rank,
+                "per_rank_tokens_per_s": seg / (per_rank / 1e3),
+                "allgather_bytes_per_rank": w.H * w.dk * (w.dk + w.dv) * 4,
+                "note": "one rank's kernels timed on one GPU; the all-gather is not measured"}
+        del sk, Mz, Zz, sout
+
     # ---------------- decode ----------------
     dec = None
     if not args.no_decode:
@@ -442,7 +489,7 @@ def main():
                            "piece_len": plan["piece_len"]},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": plan["launches"] * args.steps, "clocks": clk, "decode": dec,
-                "extended": exm}
+                "extended": exm, "kcp": kcpm}
         print(json.dumps(line), flush=True)
     if ws > 1:
         import torch.distributed as dist
