@@ -76,19 +76,24 @@ using namespace sm100;
 
 constexpr int kStages = 3;     // prepared chunks in flight: chunk c -> stage c % 3
 constexpr int kRaw = 3;        // q, k, g tiles in flight: chunk c -> raw[c % 3]
-constexpr int kPair = 64;      // threads of the decay pair (warps 4-5) and of the matrix pair (6-7)
-constexpr int kThreads = 128 + 2 * kPair;
+// A CTA has NWG state warpgroups (1, or 2 in the paired summary kernel: the
+// zero-start state and the transition of one piece, sharing one preparation),
+// then the decay pair and the matrix pair.
+constexpr int kPair = 64;      // threads of the decay pair and of the matrix pair
+template <int NWG> constexpr int kThreadsOf = 128 * NWG + 2 * kPair;
+constexpr int kThreads = kThreadsOf<1>;
 constexpr int kBlocksPerSM = 2;
-constexpr int BAR_FULL = 1;    // ids 1..3: the matrix pair arrives, the state warpgroup waits
-constexpr int BAR_EMPTY = 4;   // ids 4..6: the state warpgroup arrives, the decay pair waits
-constexpr int BAR_WG = 7;      // state warpgroup only
+constexpr int BAR_FULL = 1;    // ids 1..3: the matrix pair arrives, the state warpgroups wait
+constexpr int BAR_EMPTY = 4;   // ids 4..6: the state warpgroups arrive, the decay pair waits
+constexpr int BAR_WG = 7;      // state warpgroup 0 only
 constexpr int BAR_DEC = 8;     // ids 8..10: the decay pair arrives, the matrix pair waits
 constexpr int BAR_DPAIR = 11;  // decay pair only
 constexpr int BAR_MPAIR = 12;  // matrix pair only
-constexpr int kBarCount = 128 + kPair;  // FULL and EMPTY: the state warpgroup and one pair
+constexpr int BAR_WG2 = 13;    // state warpgroup 1 only
+template <int NWG> constexpr int kBarCountOf = 128 * NWG + kPair;  // FULL and EMPTY
 constexpr int kDecCount = 2 * kPair;
 constexpr int NC = 128;        // state columns = TMEM lanes = MMA M
-constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kTmemColsPerWG = 256;
 
 // TMA descriptors of q, k and g as [T][H][128] bf16 (3-D: channel, head,
 // token); one box = 64 channels x 1 head x 16 tokens, 128-byte swizzle.
@@ -103,13 +108,14 @@ KDA_DEVICE uint32_t sw128(int r, int ch) {
     return (uint32_t)((ch >> 6) * 2048 + r * 128 + ((((ch & 63) >> 3) ^ (r & 7)) << 4) + ((ch & 7) << 1));
 }
 
-template <int DK>
+template <int DK, int NWG = 1>
 struct Layout {
-    // TMEM columns (per CTA: 256 of the SM's 512)
+    // TMEM columns of one state warpgroup (256 of the SM's 512; warpgroup i
+    // adds 256 i)
     static constexpr uint32_t COL_S = 0;          // S^T, fp32: DK columns (MMA 3 accumulator)
     static constexpr uint32_t COL_D1 = DK;        // 2 x [U^T | O^T]: 2 x 32 fp32 columns
     static constexpr uint32_t COL_AS = DK + 64;   // bf16 S^T (MMA A operand): DK/2 columns
-    static_assert(COL_AS + DK / 2 <= kTmemCols, "TMEM budget");
+    static_assert(COL_AS + DK / 2 <= kTmemColsPerWG, "TMEM budget");
     static_assert(DK == 128, "one tile row = two 64-channel TMA boxes");
     struct Raw {                                  // TMA targets (swizzled), overwritten in place:
         alignas(1024) unsigned char q[16 * DK * 2];  //   q -> Qd
@@ -134,9 +140,9 @@ struct Layout {
         Raw raw[kRaw];
         Stage st[kStages];
         Prep pr;
-        alignas(16) bf16 au[NC * 16];   // K-major [NC][16]: U^T as the A operand
+        alignas(16) bf16 au[NWG][NC * 16];  // K-major [NC][16]: U^T as the A operand
         alignas(16) bf16 io[2][16 * NC];  // gate tile in, y tile out (row-major [16][NC])
-        alignas(8) unsigned long long mbar[2];
+        alignas(8) unsigned long long mbar[2 * NWG];
         alignas(8) unsigned long long mbar_raw[kRaw];  // TMA completion of raw[i]
         uint32_t tmem_base;
     };
@@ -153,11 +159,19 @@ KDA_DEVICE T *at_bytes(T *base, uint32_t off) {
 // y.  USE_V: the write uses v (false: the transition part, U0 = 0).  The
 // state starts as the identity, a copy of s_init ([DK][NC] fp32) or zeros and
 // is written to s_out.  The fp32 state lives in tensor memory.
-template <int DK, bool OUT, bool USE_V, bool L2N>
+// NWG = 2 (summary only): warpgroup 0 runs the zero-start state (from s_init)
+// into s_out, warpgroup 1 the transition (identity start) into s_out2; a
+// warpgroup with active[i] false takes part in every hand-off but computes
+// nothing.
+template <int DK, bool OUT, bool USE_V, bool L2N, int NWG = 1>
 __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, int len, int h,
                           const float *s_init, bool identity, float *s_out, unsigned char *smem_raw,
-                          const Snap &snap = Snap()) {
-    using Lay = Layout<DK>;
+                          const Snap &snap = Snap(), float *s_out2 = nullptr, bool active0 = true,
+                          bool active1 = true) {
+    static_assert(NWG == 1 || (NWG == 2 && !OUT && USE_V), "paired warpgroups: summaries only");
+    using Lay = Layout<DK, NWG>;
+    constexpr int kBarCount = kBarCountOf<NWG>;
+    constexpr uint32_t kTmemCols = kTmemColsPerWG * NWG;
     typename Lay::All &sm = *reinterpret_cast<typename Lay::All *>(
         smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -173,8 +187,7 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     if (tid == 32) {
-        mbar_init(smem_u32(&sm.mbar[0]), 1);
-        mbar_init(smem_u32(&sm.mbar[1]), 1);
+        for (int i = 0; i < 2 * NWG; ++i) mbar_init(smem_u32(&sm.mbar[i]), 1);
         for (int i = 0; i < kRaw; ++i) mbar_init(smem_u32(&sm.mbar_raw[i]), 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -183,14 +196,26 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
     tc_fence_after();
     const uint32_t tbase = sm.tmem_base;
 
-    if (warp < 4) {
+    if (warp < 4 * NWG) {
         // ------------------------------------------------------ state warpgroup
-        const int j = tid;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-        const uint32_t t_s = tbase + lane_off + Lay::COL_S;
-        const uint32_t t_d1 = tbase + lane_off + Lay::COL_D1;
-        const uint32_t t_as = tbase + lane_off + Lay::COL_AS;
-        const uint32_t mb1 = smem_u32(&sm.mbar[0]), mb2 = smem_u32(&sm.mbar[1]);
+        const int wgi = warp >> 2;                // which state warpgroup
+        const int j = tid - 128 * wgi;            // state column = TMEM lane
+        const int wwarp = warp & 3;               // warp within the group = TMEM lane quarter
+        const bool use_v = USE_V && wgi == 0;     // the transition part has no v
+        if (NWG == 2 && wgi == 1) {               // the transition: identity start
+            identity = true;
+            s_init = nullptr;
+            s_out = s_out2;
+        }
+        const bool active = wgi == 0 ? active0 : active1;
+        const int bar_wg = wgi == 0 ? BAR_WG : BAR_WG2;
+        const uint32_t colb = kTmemColsPerWG * wgi;
+        const uint32_t lane_off = (uint32_t)(wwarp * 32) << 16;
+        const uint32_t t_s = tbase + colb + lane_off + Lay::COL_S;
+        const uint32_t t_d1 = tbase + colb + lane_off + Lay::COL_D1;
+        const uint32_t t_as = tbase + colb + lane_off + Lay::COL_AS;
+        const uint32_t mb1 = smem_u32(&sm.mbar[2 * wgi]), mb2 = smem_u32(&sm.mbar[2 * wgi + 1]);
+        bf16 *au = sm.au[wgi];
         constexpr int N1 = OUT ? 32 : 16;
         constexpr uint32_t ID_U0 = idesc_bf16(128, N1, 1, 0);
         constexpr uint32_t ID_WS = idesc_bf16(128, N1, 0, 0);
@@ -200,7 +225,7 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
         bf16 *out = (bf16 *)p.out;
         const bool gate_logits = gate && (p.flags & FLAG_GATE_LOGITS);
 
-        bool ok = true;
+        bool ok = active;
         // gate of this thread's column for the chunk whose output is pending;
         // loaded one chunk ahead so the loads are off the critical path
         // gate tile of chunk c -> io[c & 1] (two 16-byte pieces per thread)
@@ -209,7 +234,7 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
             bf16 *tile = sm.io[c & 1];
 #pragma unroll
             for (int x2 = 0; x2 < 2; ++x2) {
-                const int x = tid + 128 * x2;
+                const int x = j + 128 * x2;
                 const int r = x >> 4, cc = x & 15;
                 const bool okr = gate && r < rows;
                 const size_t off = ((size_t)(okr ? t0 + 16 * c + r : t0) * H + h) * NC + cc * 8;
@@ -242,7 +267,7 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
             const bf16 *tile = sm.io[c & 1];
 #pragma unroll
             for (int x2 = 0; x2 < 2; ++x2) {
-                const int x = tid + 128 * x2;
+                const int x = j + 128 * x2;
                 const int r = x >> 4, cc = x & 15;
                 if (r < rows)
                     *reinterpret_cast<uint4 *>(out + ((size_t)(t0 + 16 * c + r) * H + h) * NC + cc * 8) =
@@ -313,7 +338,7 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
             }
         } else {
             bar_sync(BAR_FULL + 0, kBarCount);  // stage of chunk 0: its exp(G_C)
-            state_pass(sm.st[0].gam, true, nullptr);
+            if (ok) state_pass(sm.st[0].gam, true, nullptr);
         }
         // MMA operand descriptors of stage 0; stages are contiguous, so stage s
         // adds s * sizeof(Stage) / 16 to the start-address field (all of shared
@@ -323,7 +348,7 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
         const uint64_t dsc_b10 = sdesc(smem_u32(sm.st[0].b1), 128, DK * 16);
         const uint64_t dsc_b20 = sdesc(smem_u32(sm.st[0].b2), 128, 256);
         const uint64_t dsc_b30 = sdesc(smem_u32(sm.st[0].b3), 128, 256);
-        const uint64_t dsc_au = sdesc(smem_u32(sm.au), 128, 256);
+        const uint64_t dsc_au = sdesc(smem_u32(au), 128, 256);
         constexpr uint64_t kStageStep = sizeof(typename Lay::Stage) / 16;
         static_assert(sizeof(typename Lay::Stage) % 16 == 0, "stage stride");
 
@@ -335,19 +360,19 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
             const uint32_t d1_col = Lay::COL_D1 + 32 * (c & 1);
             KDA_MARK(tid == 0 && c < 128, c * 16 + 0);
             if (OUT) cp_async_wait<0>();  // this thread's pieces of the gate tile of chunk c - 1
-            bar_sync(BAR_WG, 128);        // state-pass TMEM stores; gate tile; y(c - 2) stored
+            bar_sync(bar_wg, 128);        // state-pass TMEM stores; gate tile; y(c - 2) stored
             if (OUT) load_gate(c);
             KDA_MARK(tid == 0 && c < 128, c * 16 + 1);
-            if (warp == 0 && ok) {  // U0^T and [-W | Qd] S^T: needs only the bf16 copy
-                const uint32_t d1 = tbase + d1_col;
+            if (wwarp == 0 && ok) {  // U0^T and [-W | Qd] S^T: needs only the bf16 copy
+                const uint32_t d1 = tbase + colb + d1_col;
                 const uint64_t so = kStageStep * stg;
                 if (elect_one_sync()) {
                     tc_fence_after();
-                    if (USE_V) tc_mma_ss(d1, dsc_v0 + so, dsc_b00 + so, ID_U0, 0);
+                    if (use_v) tc_mma_ss(d1, dsc_v0 + so, dsc_b00 + so, ID_U0, 0);
 #pragma unroll
                     for (int kk = 0; kk < DK / 16; ++kk)  // +256 bytes of K = +16 in the start field
-                        tc_mma_ts(d1, tbase + Lay::COL_AS + 8 * kk, dsc_b10 + so + 16 * kk, ID_WS,
-                                  (USE_V || kk > 0) ? 1u : 0u);
+                        tc_mma_ts(d1, tbase + colb + Lay::COL_AS + 8 * kk, dsc_b10 + so + 16 * kk, ID_WS,
+                                  (use_v || kk > 0) ? 1u : 0u);
                     tc_commit(mb1);
                 }
                 __syncwarp();  // reconverge warp 0 before the aligned TMEM loads below
@@ -366,19 +391,19 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
 #pragma unroll
                 for (int e = 0; e < 8; ++e)
                     pk[e] = pack_bf16(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1]));
-                *reinterpret_cast<uint4 *>(at_bytes(sm.au, kmaj(j, 0, 16))) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                *reinterpret_cast<uint4 *>(at_bytes(sm.au, kmaj(j, 8, 16))) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                *reinterpret_cast<uint4 *>(at_bytes(au, kmaj(j, 0, 16))) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                *reinterpret_cast<uint4 *>(at_bytes(au, kmaj(j, 8, 16))) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
             }
             fence_async_smem();
             tc_fence_before();
             KDA_MARK(tid == 0 && c < 128, c * 16 + 7);
-            bar_sync(BAR_WG, 128);
-            if (warp == 0 && ok) {  // S^T += U^T Kb (into the state itself);  O^T += U^T P^T
+            bar_sync(bar_wg, 128);
+            if (wwarp == 0 && ok) {  // S^T += U^T Kb (into the state itself);  O^T += U^T P^T
                 const uint64_t so = kStageStep * stg;
                 if (elect_one_sync()) {
                     tc_fence_after();
-                    tc_mma_ss(tbase + Lay::COL_S, dsc_au, dsc_b20 + so, ID_UK, 1);
-                    if (OUT) tc_mma_ss(tbase + d1_col + 16, dsc_au, dsc_b30 + so, ID_UP, 1);
+                    tc_mma_ss(tbase + colb + Lay::COL_S, dsc_au, dsc_b20 + so, ID_UK, 1);
+                    if (OUT) tc_mma_ss(tbase + colb + d1_col + 16, dsc_au, dsc_b30 + so, ID_UP, 1);
                     tc_commit(mb2);
                 }
                 __syncwarp();  // reconverge warp 0 before the aligned barrier below
@@ -404,19 +429,19 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
         }
         if (nchunks > 0) {
             if (OUT) cp_async_wait<0>();
-            bar_sync(BAR_WG, 128);
+            bar_sync(bar_wg, 128);
             finish_chunk(nchunks - 1);
             if (OUT) {
-                bar_sync(BAR_WG, 128);
+                bar_sync(bar_wg, 128);
                 store_y(nchunks - 1);
             }
         }
-        if (!ok && lane == 0 && p.err) atomicOr(p.err, 1);
-    } else if (warp < 6) {
+        if (active && !ok && lane == 0 && p.err) atomicOr(p.err, 1);
+    } else if (warp < 4 * NWG + 2) {
         // ------------------------------------------------------------ decay pair
         // Warps 4-5: thread d owns the key-channel pair (ip, ip + 1) on all 16
         // rows of a chunk; it runs up to kRaw chunks ahead of the matrix pair.
-        const int d = tid - 128, dw = d >> 5, ip = 2 * d;
+        const int d = tid - 128 * NWG, dw = d >> 5, ip = 2 * d;
         const bf16 *v = (const bf16 *)p.v, *beta = (const bf16 *)p.beta;
         typename Lay::Prep &pr = sm.pr;
         // beta of chunks c and c + 1 (threads d < 16), kept as raw bf16 bits so
@@ -572,7 +597,7 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
         // ----------------------------------------------------------- matrix pair
         // Warps 6-7: the Gram matrices, the unit-lower solve, W, and the TMA
         // loads of q, k, g (thread 0).
-        const int m = tid - 192, mw = m >> 5;
+        const int m = tid - 128 * NWG - kPair, mw = m >> 5;
         typename Lay::Prep &pr = sm.pr;
         auto issue_raw = [&](int c) {
             typename Lay::Raw &R = sm.raw[c % kRaw];
@@ -720,8 +745,15 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
                      : "memory");
 }
 
+// The summary pass: one CTA per (piece, head), one SM each.  State warpgroup
+// 0 runs the piece from zero (or from the sequence's initial state for its
+// first piece) into S_zero, warpgroup 1 runs it from the identity without v
+// into the transition M; both share one preparation of every chunk.  A part
+// the scan does not need (S_zero of a sequence's last piece, M of its first)
+// is skipped unless every piece's map is asked for.
 template <int DK, bool L2N>
-__global__ void __launch_bounds__(kThreads, kBlocksPerSM) summary_kernel(PrefillParams p, const __grid_constant__ TmaMaps maps) {
+__global__ void __launch_bounds__(kThreadsOf<2>, 1)
+    summary_kernel(PrefillParams p, const __grid_constant__ TmaMaps maps) {
     extern __shared__ __align__(128) unsigned char smem[];
     // (piece, head) pairs with the head fastest: co-resident CTAs cover all
     // heads of a few pieces, spreading their rows over every memory channel
@@ -730,17 +762,16 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSM) summary_kernel(Prefill
     if (pc.x < 0) return;
     const int n = pc.x, j = pc.w;
     const int np = p.seq_first[n + 1] - p.seq_first[n];
-    if (!p.summarize_all && j >= np - 1) return;
+    const bool want_s = p.summarize_all || j < np - 1;
+    const bool want_m = p.summarize_all || j > 0;
+    if (!want_s && !want_m) return;
     const size_t ph = (size_t)pi * p.H + h;
-    if (blockIdx.y == 0) {
-        const float *init = (j == 0 && p.initial_state)
-                                ? p.initial_state + ((size_t)n * p.H + h) * DK * NC
-                                : nullptr;
-        run_piece<DK, false, true, L2N>(p, maps, pc.y, pc.z, h, init, false, p.Szero + ph * DK * NC, smem);
-    } else {
-        if (!p.summarize_all && j == 0) return;
-        run_piece<DK, false, false, L2N>(p, maps, pc.y, pc.z, h, nullptr, true, p.M + ph * DK * DK, smem);
-    }
+    const float *init = (j == 0 && p.initial_state)
+                            ? p.initial_state + ((size_t)n * p.H + h) * DK * NC
+                            : nullptr;
+    run_piece<DK, false, true, L2N, 2>(p, maps, pc.y, pc.z, h, init, false,
+                                       want_s ? p.Szero + ph * DK * NC : nullptr, smem, Snap(),
+                                       want_m ? p.M + ph * DK * DK : nullptr, want_s, want_m);
 }
 
 template <int DK, bool L2N>
@@ -796,6 +827,7 @@ bool encode_rows(CUtensorMap *m, const void *base, int T, int H) {
 template <bool L2N>
 cudaError_t launch_tc5(const PrefillParams &p, bool summaries, cudaStream_t st) {
     const size_t sm = tc5::Layout<128>::bytes;
+    const size_t sm2 = tc5::Layout<128, 2>::bytes;
     cudaError_t e;
     tc5::TmaMaps maps;
     memset(&maps, 0, sizeof(maps));
@@ -805,9 +837,10 @@ cudaError_t launch_tc5(const PrefillParams &p, bool summaries, cudaStream_t st) 
         return cudaErrorInvalidValue;
     if (summaries) {
         e = cudaFuncSetAttribute(tc5::summary_kernel<128, L2N>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
         if (e != cudaSuccess) return e;
-        tc5::summary_kernel<128, L2N><<<dim3((unsigned)(p.P_max * p.H), 2), tc5::kThreads, sm, st>>>(p, maps);
+        tc5::summary_kernel<128, L2N><<<dim3((unsigned)(p.P_max * p.H)), tc5::kThreadsOf<2>, sm2, st>>>(
+            p, maps);
         return cudaGetLastError();
     }
     e = cudaFuncSetAttribute(tc5::output_kernel<128, L2N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
