@@ -54,10 +54,16 @@
 // prep warps' chunk loops, read back through kda_tc5_trace_copy().
 #ifdef KDA_TC5_TRACE
 __device__ unsigned long long g_kda_tc5_trace[8192];
+// traced CTA: piece 0 of head 1 of the output pass, or, with
+// -DKDA_TRACE_SUMMARY, piece 1 of head 0 of the summary pass
+#ifdef KDA_TRACE_SUMMARY
+#define KDA_TRACE_HERE (!OUT && blockIdx.x == (unsigned)p.H)
+#else
+#define KDA_TRACE_HERE (OUT && blockIdx.x == 1)
+#endif
 #define KDA_MARK(cond, slot)                                                          \
     do {                                                                              \
-        if ((cond) && blockIdx.x == 1 && blockIdx.y == 0 &&        \
-            (slot) < 8192)                                                            \
+        if ((cond) && KDA_TRACE_HERE && (slot) < 8192)                                \
             g_kda_tc5_trace[(slot)] = clock64();                                      \
         __syncwarp();                                                                 \
     } while (0)
@@ -163,7 +169,9 @@ KDA_DEVICE T *at_bytes(T *base, uint32_t off) {
 // into s_out, warpgroup 1 the transition (identity start) into s_out2; a
 // warpgroup with active[i] false takes part in every hand-off but computes
 // nothing.
-template <int DK, bool OUT, bool USE_V, bool L2N, int NWG = 1>
+// EXT: the extended entry points' features (beta / gate logits, the decay
+// clamp, state snapshots) are compiled in; the plain calls run without them.
+template <int DK, bool OUT, bool USE_V, bool L2N, bool EXT, int NWG = 1>
 __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, int len, int h,
                           const float *s_init, bool identity, float *s_out, unsigned char *smem_raw,
                           const Snap &snap = Snap(), float *s_out2 = nullptr, bool active0 = true,
@@ -171,6 +179,7 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
     static_assert(NWG == 1 || (NWG == 2 && !OUT && USE_V), "paired warpgroups: summaries only");
     using Lay = Layout<DK, NWG>;
     constexpr int kBarCount = kBarCountOf<NWG>;
+    const int flags = EXT ? p.flags : 0;  // bits other than the norm switch
     constexpr uint32_t kTmemCols = kTmemColsPerWG * NWG;
     typename Lay::All &sm = *reinterpret_cast<typename Lay::All *>(
         smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
@@ -223,7 +232,7 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
         constexpr uint32_t ID_UP = idesc_bf16(128, 16, 0, 0);
         const bf16 *gate = (const bf16 *)p.gate;
         bf16 *out = (bf16 *)p.out;
-        const bool gate_logits = gate && (p.flags & FLAG_GATE_LOGITS);
+        const bool gate_logits = gate && (flags & FLAG_GATE_LOGITS);
 
         bool ok = active;
         // gate of this thread's column for the chunk whose output is pending;
@@ -421,7 +430,7 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
             KDA_MARK(tid == 0 && c < 128, c * 16 + 10);
             if (ok) {
                 state_pass(has_next ? sm.st[(c + 1) % kStages].gam : nullptr, false,
-                           snap.at(snap.pos0 + 16 * (c + 1)));
+                           EXT ? snap.at(snap.pos0 + 16 * (c + 1)) : nullptr);
             } else {
                 tc_fence_before();
             }
@@ -496,7 +505,7 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
                     }
                 }
             }
-            if (d < 16) pr.beta[stg][d] = beta_in(__bfloat162float(__ushort_as_bfloat16(bq0)), p.flags);
+            if (d < 16) pr.beta[stg][d] = beta_in(__bfloat162float(__ushort_as_bfloat16(bq0)), flags);
             __syncwarp();
             bar_sync(BAR_DPAIR, kPair);             // the tiles (with cleared rows) are visible
             KDA_MARK(d == 0 && c < 128, 2048 + c * 8 + 2);
@@ -536,7 +545,7 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
 #pragma unroll
             for (int r = 0; r < 16; ++r) {
                 const float2 gg = unpack_bf16(*reinterpret_cast<const uint32_t *>(Wk.g + sw128(r, ip)));
-                e[r] = make_float2(__expf(g_in(gg.x, p.flags)), __expf(g_in(gg.y, p.flags)));
+                e[r] = make_float2(__expf(g_in(gg.x, flags)), __expf(g_in(gg.y, flags)));
             }
             {
                 float2 acc = make_float2(1.f, 1.f);
@@ -751,7 +760,7 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
 // into the transition M; both share one preparation of every chunk.  A part
 // the scan does not need (S_zero of a sequence's last piece, M of its first)
 // is skipped unless every piece's map is asked for.
-template <int DK, bool L2N>
+template <int DK, bool L2N, bool EXT>
 __global__ void __launch_bounds__(kThreadsOf<2>, 1)
     summary_kernel(PrefillParams p, const __grid_constant__ TmaMaps maps) {
     extern __shared__ __align__(128) unsigned char smem[];
@@ -769,12 +778,12 @@ __global__ void __launch_bounds__(kThreadsOf<2>, 1)
     const float *init = (j == 0 && p.initial_state)
                             ? p.initial_state + ((size_t)n * p.H + h) * DK * NC
                             : nullptr;
-    run_piece<DK, false, true, L2N, 2>(p, maps, pc.y, pc.z, h, init, false,
+    run_piece<DK, false, true, L2N, EXT, 2>(p, maps, pc.y, pc.z, h, init, false,
                                        want_s ? p.Szero + ph * DK * NC : nullptr, smem, Snap(),
                                        want_m ? p.M + ph * DK * DK : nullptr, want_s, want_m);
 }
 
-template <int DK, bool L2N>
+template <int DK, bool L2N, bool EXT>
 __global__ void __launch_bounds__(kThreads, kBlocksPerSM) output_kernel(PrefillParams p, const __grid_constant__ TmaMaps maps) {
     extern __shared__ __align__(128) unsigned char smem[];
     // (piece, head) pairs with the head fastest: co-resident CTAs cover all
@@ -788,8 +797,8 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSM) output_kernel(PrefillP
     const float *init = (np == 1) ? (p.initial_state ? p.initial_state + nh * DK * NC : nullptr)
                                   : p.Sin + ((size_t)pi * p.H + h) * DK * NC;
     float *fin = (j == np - 1 && p.final_state) ? p.final_state + nh * DK * NC : nullptr;
-    run_piece<DK, true, true, L2N>(p, maps, pc.y, pc.z, h, init, false, fin, smem,
-                                   make_snap(p, n, h, pc.y, (size_t)DK * NC));
+    run_piece<DK, true, true, L2N, EXT>(p, maps, pc.y, pc.z, h, init, false, fin, smem,
+                                        EXT ? make_snap(p, n, h, pc.y, (size_t)DK * NC) : Snap());
 }
 
 }  // namespace tc5
@@ -824,7 +833,7 @@ bool encode_rows(CUtensorMap *m, const void *base, int T, int H) {
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool L2N>
+template <bool L2N, bool EXT>
 cudaError_t launch_tc5(const PrefillParams &p, bool summaries, cudaStream_t st) {
     const size_t sm = tc5::Layout<128>::bytes;
     const size_t sm2 = tc5::Layout<128, 2>::bytes;
@@ -836,23 +845,26 @@ cudaError_t launch_tc5(const PrefillParams &p, bool summaries, cudaStream_t st) 
          !encode_rows(&maps.g, p.g, p.total_tokens, p.H)))
         return cudaErrorInvalidValue;
     if (summaries) {
-        e = cudaFuncSetAttribute(tc5::summary_kernel<128, L2N>,
+        e = cudaFuncSetAttribute(tc5::summary_kernel<128, L2N, EXT>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
         if (e != cudaSuccess) return e;
-        tc5::summary_kernel<128, L2N><<<dim3((unsigned)(p.P_max * p.H)), tc5::kThreadsOf<2>, sm2, st>>>(
+        tc5::summary_kernel<128, L2N, EXT><<<dim3((unsigned)(p.P_max * p.H)), tc5::kThreadsOf<2>, sm2, st>>>(
             p, maps);
         return cudaGetLastError();
     }
-    e = cudaFuncSetAttribute(tc5::output_kernel<128, L2N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(tc5::output_kernel<128, L2N, EXT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)sm);
     if (e != cudaSuccess) return e;
-    tc5::output_kernel<128, L2N><<<dim3((unsigned)(p.P_max * p.H)), tc5::kThreads, sm, st>>>(p, maps);
+    tc5::output_kernel<128, L2N, EXT><<<dim3((unsigned)(p.P_max * p.H)), tc5::kThreads, sm, st>>>(p, maps);
     return cudaGetLastError();
 }
 }  // namespace
 
 cudaError_t launch_prefill_tc5(const PrefillParams &p, bool summaries, cudaStream_t st) {
-    return (p.flags & FLAG_L2NORM) ? launch_tc5<true>(p, summaries, st) : launch_tc5<false>(p, summaries, st);
+    const bool l2 = p.flags & FLAG_L2NORM;
+    const bool ext = (p.flags & ~FLAG_L2NORM) || p.snap_tokens > 0;
+    if (ext) return l2 ? launch_tc5<true, true>(p, summaries, st) : launch_tc5<false, true>(p, summaries, st);
+    return l2 ? launch_tc5<true, false>(p, summaries, st) : launch_tc5<false, false>(p, summaries, st);
 }
 
 }  // namespace kda
