@@ -46,6 +46,14 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum, summed over the four
+# launches) of one call, from one ncu capture of
+#   bench.py --steps 1 --warmup 1 --no-e2e --no-cpu --no-decode --no-ex --no-kcp
+# keyed by (workload, piece length).  Valid only for the kernels as captured:
+# a change to any kernel of the call makes the figure stale (report null then).
+NCU_CALL_TRAFFIC = {("long_bf16", 3552): 10.18e9}
+
+
 def prefill_bytes(w, T, N):
     """Algorithmic HBM bytes of one prefill call: read q, k, g, v, gate, beta,
     write y (dtype), read the initial and write the final state (fp32)."""
@@ -297,7 +305,8 @@ def main():
     hbm = pk["hbm_gbs"]
     achieved = pbytes / (ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                "frac": achieved / hbm, "traffic": None,
+                "frac": achieved / hbm,
+                "traffic": NCU_CALL_TRAFFIC.get((args.workload, plan["piece_len"])),
                 "kernel": "kda_chunk_fwd call (%d launches)" % plan["launches"],
                 "peak_source": f"{pk_kind} hbm_gbs",
                 "tensor_tflops": pflops / (ms / 1e3) / 1e12,

@@ -17,16 +17,19 @@
 // values in registers between the read and the write, so S crosses HBM
 // exactly once in each direction.  The reduction over the key channels is
 // per-thread partial sums followed by a shared-memory combine across warps.
+// EXT compiles in the preprocessing flags other than the q/k norm (beta and
+// gate as logits, the decay clamp); the plain call runs without them.
 #include "kda_common.cuh"
 
 namespace kda {
 
-template <int DK, int DV, typename T>
+template <int DK, int DV, typename T, bool EXT>
 __global__ void __launch_bounds__(256, 2)
     decode_step_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                        const T *__restrict__ g, const T *__restrict__ beta,
                        const T *__restrict__ gate, T *__restrict__ out, float *state, float scale,
-                       int flags) {
+                       int flags_in) {
+    const int flags = EXT ? flags_in : (flags_in & FLAG_L2NORM);
     constexpr int NT = 256;
     constexpr int COLG = DV / 4;       // float4 groups per state row
     constexpr int RPP = NT / COLG;     // rows covered by one pass of the CTA
@@ -127,9 +130,14 @@ template <int DK, int DV, typename T>
 static cudaError_t launch_decode_t(const void *q, const void *k, const void *v, const void *g,
                                    const void *beta, const void *gate, void *out, float *state,
                                    long nh, float scale, int flags, cudaStream_t st) {
-    decode_step_kernel<DK, DV, T><<<(unsigned)nh, 256, 0, st>>>(
-        (const T *)q, (const T *)k, (const T *)v, (const T *)g, (const T *)beta, (const T *)gate,
-        (T *)out, state, scale, flags);
+    if (flags & ~FLAG_L2NORM)
+        decode_step_kernel<DK, DV, T, true><<<(unsigned)nh, 256, 0, st>>>(
+            (const T *)q, (const T *)k, (const T *)v, (const T *)g, (const T *)beta,
+            (const T *)gate, (T *)out, state, scale, flags);
+    else
+        decode_step_kernel<DK, DV, T, false><<<(unsigned)nh, 256, 0, st>>>(
+            (const T *)q, (const T *)k, (const T *)v, (const T *)g, (const T *)beta,
+            (const T *)gate, (T *)out, state, scale, flags);
     return cudaGetLastError();
 }
 
