@@ -61,15 +61,17 @@ inline WorkspaceLayout workspace_layout(long P_max, int num_seqs, int H, int dk,
 
 // ---------------------------------------------------------------- the plan
 // Piece length (tokens, a multiple of 16).  Each (piece, head) is one CTA of
-// the chunk kernels, which run two CTAs per SM, so time is counted in whole
-// waves of `slots` = 2 x SMs CTAs.  A sequence of p > 1 pieces costs an output pass over
-// all p pieces plus a summary pass over 2p - 3 (piece, part) units (pieces
-// 0..p-2 summarise their zero-start state, pieces 1..p-2 their transition)
-// and p - 1 steps of the prefix scan.  With equal-length sequences (the
-// lengths are not known on the host in general) the model is
-//   cost(L) = waves(output) * chunks(L) + 0.8 * waves(summary) * chunks(L)
+// the output pass, which runs two CTAs per SM, so its time is counted in whole
+// waves of `slots` = 2 x SMs CTAs.  A sequence of p > 1 pieces costs an output
+// pass over all p pieces, a summary pass over pieces 0..p-2 (one CTA per
+// (piece, head) computes both the zero-start state and the transition, one CTA
+// per SM: waves of slots / 2) and p - 1 steps of the prefix scan.  With
+// equal-length sequences (the lengths are not known on the host in general)
+// the model is
+//   cost(L) = waves(output) * chunks(L) + 0.79 * waves(summary) * chunks(L)
 //             + 2 * (pieces - 1)
-// in units of one chunk step; the summary pass has no outputs, hence 0.8.
+// in units of one chunk step of the output pass; 0.79 is the measured ratio
+// of the two passes' per-chunk periods (about 3.0 K and 3.8 K SM cycles).
 // When the host copy of the offsets is given, the real lengths are used, and
 // only piece lengths at least as long as the length-blind choice are
 // considered, so that the workspace sized without the lengths still fits.
@@ -82,14 +84,15 @@ inline double plan_cost(long L, int num_seqs, int H, int slots, const int32_t *c
         const long pcs = len <= 0 ? 1 : (len + L - 1) / L;
         const long mult = cu_host ? 1 : num_seqs;
         out += mult * pcs;
-        if (pcs > 1) sum += mult * (2 * pcs - 3);
+        sum += mult * (pcs - 1);
         const long ch = (std::min(len, L) + 15) / 16;
         if (ch > max_chunks) max_chunks = ch;
         if (pcs > max_pieces) max_pieces = pcs;
     }
     const long w_out = (out * H + slots - 1) / slots;
-    const long w_sum = (sum * H + slots - 1) / slots;
-    return (double)w_out * max_chunks + 0.8 * (double)w_sum * max_chunks +
+    const long sum_slots = std::max(slots / 2, 1);
+    const long w_sum = (sum * H + sum_slots - 1) / sum_slots;
+    return (double)w_out * max_chunks + 0.79 * (double)w_sum * max_chunks +
            2.0 * (double)(max_pieces - 1);
 }
 
