@@ -242,6 +242,8 @@ def main():
                     help="skip the per-rank context-parallel measurement")
     ap.add_argument("--no-ex", action="store_true",
                     help="skip the extended-path measurement (flags + state snapshots)")
+    ap.add_argument("--no-bwd", action="store_true",
+                    help="skip the backward measurement")
     ap.add_argument("--out-dir", default=os.path.join(ROOT, "gpurun_out"))
     ap.add_argument("--ref-tokens", type=int, default=0,
                     help="reference arm: tokens per step sample (0 = scale with cores)")
@@ -399,6 +401,63 @@ def main():
                 "note": "one rank's kernels timed on one GPU; the all-gather is not measured"}
         del sk, Mz, Zz, sout
 
+    # ------- backward (kda_bwd) on prefill_bf16: 2 x 4096 tokens, H = 16 -------
+    bwdm = None
+    if not args.no_bwd:
+        wb = W.get("prefill_bf16")
+        bi = W.fast_prefill(wb, seed=wb.seed + 1000 * rank, device=dev)
+        Tb, Nb = wb.total_tokens, wb.num_seqs
+        gb = torch.Generator(device=dev).manual_seed(wb.seed + 7)
+        dyb = torch.randn(Tb, wb.H, wb.dv, generator=gb, device=dev).to(wb.torch_dtype)
+        dsfb = torch.randn(Nb, wb.H, wb.dk, wb.dv, generator=gb, device=dev)
+        f32b = dict(dtype=torch.float32, device=dev)
+        gq, gk, gg = (torch.empty(Tb, wb.H, wb.dk, **f32b) for _ in range(3))
+        gv, ggt = (torch.empty(Tb, wb.H, wb.dv, **f32b) for _ in range(2))
+        gbt = torch.empty(Tb, wb.H, **f32b)
+        gs0 = torch.empty(Nb, wb.H, wb.dk, wb.dv, **f32b)
+        wsb_bytes = kda.bwd_workspace_size(Tb, Nb, wb.H, wb.dk, wb.dv)
+        wsb = torch.empty(wsb_bytes, dtype=torch.uint8, device=dev)
+        cub = bi["cu_seqlens"].tolist()
+        cub_arr = (ctypes.c_int32 * len(cub))(*cub)
+        Pb = ctypes.c_void_p
+        pb = lambda t: Pb(t.data_ptr())
+        bargs = (pb(bi["q"]), pb(bi["k"]), pb(bi["v"]), pb(bi["g"]), pb(bi["beta"]),
+                 pb(bi["gate"]), pb(dyb), pb(bi["cu_seqlens"]), ctypes.cast(cub_arr, Pb), Nb, Tb,
+                 wb.H, wb.dk, wb.dv, kda._dtype_code(bi["q"]), 1.0, None, pb(dsfb), pb(gq),
+                 pb(gk), pb(gv), pb(gg), pb(gbt), pb(ggt), pb(gs0), pb(wsb), wsb_bytes,
+                 Pb(stream.cuda_stream))
+
+        def bwd_call():
+            rc = lib.kda_bwd(*bargs)
+            if rc != 0:
+                raise RuntimeError(kda.status_string(rc))
+
+        for _ in range(args.warmup):
+            bwd_call()
+        torch.cuda.synchronize()
+        barrier(ws)
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        b0.record(stream)
+        for _ in range(args.steps):
+            bwd_call()
+        b1.record(stream)
+        torch.cuda.synchronize()
+        barrier(ws)
+        bms = reduce_max(b0.elapsed_time(b1), ws) / args.steps
+        e = 2  # bf16 inputs
+        bbytes = (Tb * wb.H * ((3 * wb.dk + 3 * wb.dv + 1) * e + 4 * (3 * wb.dk + 2 * wb.dv + 1))
+                  + 2 * Nb * wb.H * wb.dk * wb.dv * 4)
+        bgbs = bbytes / (bms / 1e3) / 1e9
+        bwdm = {"value": ws * Tb / (bms / 1e3), "unit": "tokens/s", "ms_per_call": bms,
+                "workload": "prefill_bf16 backward: 2 x 4096 tokens, H=16, dk=dv=128, bf16 in, "
+                            "fp32 gradients, final-state gradient given",
+                "roofline": {"bound": "hbm", "achieved": bgbs, "peak": hbm, "unit": "GB/s",
+                             "frac": bgbs / hbm, "traffic": None,
+                             "kernel": "bwd_kernel<128,bf16> (checkpointed reverse recurrence)",
+                             "peak_source": f"{pk_kind} hbm_gbs"},
+                "gpu_launches": args.steps}
+        del bi, dyb, dsfb, gq, gk, gg, gv, ggt, gbt, gs0, wsb
+
     # ---------------- decode ----------------
     dec = None
     if not args.no_decode:
@@ -498,7 +557,7 @@ def main():
                            "piece_len": plan["piece_len"]},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": plan["launches"] * args.steps, "clocks": clk, "decode": dec,
-                "extended": exm, "kcp": kcpm}
+                "extended": exm, "kcp": kcpm, "backward": bwdm}
         print(json.dumps(line), flush=True)
     if ws > 1:
         import torch.distributed as dist

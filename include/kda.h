@@ -262,6 +262,51 @@ int kda_state_compose(const float *transitions, const float *zero_states, int32_
                       const float *state_in, float *state_out, int32_t num_seqs, int32_t H,
                       int32_t dk, int32_t dv, kda_stream_t stream);
 
+/* ------------------------------------------------------------------ backward
+ * Gradients of the plain forward (kda_chunk_fwd with qk_l2norm = 0: beta and
+ * gate as given, the delta-rule write) for the loss
+ *   L = sum dy (.) y + sum d_final_state (.) final_state.
+ * The pages state the forward only (Kimi K3 report explainer, affta.cn,
+ * section "第一关：KDA 解决算得动": forget, corrective write with an update
+ * strength, read, output gate); this is that recurrence differentiated by the
+ * chain rule, token by token in reverse, with the states recomputed from
+ * checkpoints every 64 tokens.  fp32 arithmetic; results are deterministic up
+ * to the order of fp32 atomic additions across 32-column slices of dv.
+ *
+ * kda_bwd_workspace_size: bytes of workspace kda_bwd needs (0 for
+ *   unsupported sizes): checkpoints ((total_tokens / 64 + num_seqs) * H * dk
+ *   * dv floats) plus per-(sequence, head, 32 columns) scratch of 64 states.
+ *
+ * kda_bwd:
+ *   q, k, g       device [total_tokens][H][dk], dtype; v, gate, dy device
+ *                 [total_tokens][H][dv], dtype (gate may be NULL: y = o);
+ *                 beta device [total_tokens][H], dtype.  Element-aligned.
+ *   cu_seqlens, cu_seqlens_host, num_seqs, total_tokens, H, dk, dv, dtype,
+ *                 scale: as kda_chunk_fwd (dk, dv in {64, 128}).  The device
+ *                 offsets are clamped into [0, total_tokens] in the kernel.
+ *   initial_state device fp32 [num_seqs][H][dk][dv] or NULL (zeros).
+ *   d_final_state device fp32 [num_seqs][H][dk][dv] or NULL (zeros).
+ *   dq, dk_out, dg  device fp32 [total_tokens][H][dk], written.
+ *   dv_out          device fp32 [total_tokens][H][dv], written.
+ *   dbeta           device fp32 [total_tokens][H], written.
+ *   dgate           device fp32 [total_tokens][H][dv] or NULL (must be NULL
+ *                   when gate is NULL -> KDA_ERR_INVALID_ARG).
+ *   d_initial_state device fp32 [num_seqs][H][dk][dv] or NULL.
+ *   workspace       >= kda_bwd_workspace_size(...) bytes, 256-byte aligned.
+ * Gradient outputs are 4-byte aligned; all device buffers stay owned by the
+ * caller.  Errors: as kda_chunk_fwd.
+ */
+size_t kda_bwd_workspace_size(int32_t total_tokens, int32_t num_seqs, int32_t H, int32_t dk,
+                              int32_t dv);
+
+int kda_bwd(const void *q, const void *k, const void *v, const void *g, const void *beta,
+            const void *gate, const void *dy, const int32_t *cu_seqlens,
+            const int32_t *cu_seqlens_host, int32_t num_seqs, int32_t total_tokens, int32_t H,
+            int32_t dk, int32_t dv, kda_dtype dtype, float scale, const float *initial_state,
+            const float *d_final_state, float *dq, float *dk_out, float *dv_out, float *dg,
+            float *dbeta, float *dgate, float *d_initial_state, void *workspace,
+            size_t workspace_bytes, kda_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -20,7 +20,7 @@ KDA_DTYPE_BF16 = 1
 
 EXPORTS = ("kda_status_string", "kda_chunk_fwd_workspace_size", "kda_chunk_fwd_plan",
            "kda_chunk_fwd", "kda_decode_step", "kda_chunk_fwd_ex", "kda_decode_step_ex",
-           "kda_chunk_fwd_summary", "kda_state_compose")
+           "kda_chunk_fwd_summary", "kda_state_compose", "kda_bwd_workspace_size", "kda_bwd")
 
 # flags of the extended entry points (include/kda.h)
 FLAG_QK_L2NORM, FLAG_BETA_LOGITS, FLAG_GATE_LOGITS, FLAG_CLAMP_DECAY = 1, 2, 4, 8
@@ -67,6 +67,11 @@ def load(path: str = LIB_PATH):
     lib.kda_chunk_fwd_summary.restype = ctypes.c_int
     lib.kda_state_compose.argtypes = [P, P, i32, P, P, i32, i32, i32, i32, P]
     lib.kda_state_compose.restype = ctypes.c_int
+    lib.kda_bwd_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+    lib.kda_bwd_workspace_size.restype = sz
+    lib.kda_bwd.argtypes = [P, P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, ctypes.c_int,
+                            f32, P, P, P, P, P, P, P, P, P, P, sz, P]
+    lib.kda_bwd.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -240,4 +245,45 @@ def state_compose(M, Z, state_in=None, *, out=None, stream=None):
     st = lib.kda_state_compose(_ptr(M), _ptr(Z), R, _ptr(state_in), _ptr(out), N, H, dk, dv,
                                _stream(stream))
     _check("kda_state_compose", st)
+    return out
+
+
+def bwd_workspace_size(total_tokens, num_seqs, H, dk, dv) -> int:
+    return int(load().kda_bwd_workspace_size(total_tokens, num_seqs, H, dk, dv))
+
+
+def bwd(q, k, v, g, beta, gate, dy, cu_seqlens, *, scale=1.0, initial_state=None,
+        d_final_state=None, cu_seqlens_host=None, workspace=None, stream=None):
+    """Gradients of the plain forward (kda_bwd): returns a dict of fp32
+    tensors dq, dk, dg [T, H, dk]; dv, dgate [T, H, dv] (dgate None without a
+    gate); dbeta [T, H]; ds0 [N, H, dk, dv]."""
+    lib = load()
+    _require_cuda(q, k, v, g, beta, gate, dy, cu_seqlens, initial_state, d_final_state)
+    q, k, v, g, beta, dy = (t.contiguous() for t in (q, k, v, g, beta, dy))
+    gate = None if gate is None else gate.contiguous()
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    N = cu_seqlens.numel() - 1
+    dev = q.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = {"dq": torch.empty(T, H, dk, **f32), "dk": torch.empty(T, H, dk, **f32),
+           "dg": torch.empty(T, H, dk, **f32), "dv": torch.empty(T, H, dv, **f32),
+           "dbeta": torch.empty(T, H, **f32),
+           "dgate": None if gate is None else torch.empty(T, H, dv, **f32),
+           "ds0": torch.empty(N, H, dk, dv, **f32)}
+    need = bwd_workspace_size(T, N, H, dk, dv)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    cu_arr = None
+    if cu_seqlens_host is not None:
+        cu_arr = (ctypes.c_int32 * len(cu_seqlens_host))(*cu_seqlens_host)
+    s0 = None if initial_state is None else initial_state.float().contiguous()
+    dsf = None if d_final_state is None else d_final_state.float().contiguous()
+    st = lib.kda_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(gate), _ptr(dy),
+                     _ptr(cu_seqlens), None if cu_arr is None else ctypes.cast(cu_arr, ctypes.c_void_p),
+                     N, T, H, dk, dv, _dtype_code(q), float(scale), _ptr(s0), _ptr(dsf),
+                     _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]),
+                     _ptr(out["dbeta"]), _ptr(out["dgate"]), _ptr(out["ds0"]), _ptr(workspace),
+                     workspace.numel(), _stream(stream))
+    _check("kda_bwd", st)
     return out

@@ -210,3 +210,27 @@ def test_summary_and_compose_validation(lib):
     assert c(A, A, 1, A, A + 8, 1, 1, 64, 64, None) == ALIGN
     assert c(A, A, 1, A, A + 256, 1, 1, 64, 64, None) == INVALID    # partial overlap
     assert c(A, A, 1, A, A, 1, 1, 32, 64, None) == UNSUPPORTED
+
+
+def test_bwd_validation(lib):
+    """kda_bwd rejects bad arguments before touching the device."""
+    f = lib.kda_bwd
+    ws = lib.kda_bwd_workspace_size(16, 1, 1, 64, 64)
+    assert ws > 0 and lib.kda_bwd_workspace_size(16, 1, 1, 96, 64) == 0
+    # q k v g beta gate dy cu cu_host N T H dk dv dtype scale s0 dsT
+    # dq dk dv dg dbeta dgate ds0 ws ws_bytes stream
+    base = [A, A, A, A, A, A, A, A, None, 1, 16, 1, 64, 64, BF16, 1.0, None, None,
+            A, A, A, A, A, A, A, A, ws, None]
+    assert f(*base[:9], 0, 0, *base[11:]) == OK                   # no sequences
+    assert f(*base[:12], 96, *base[13:]) == UNSUPPORTED             # dk
+    assert f(*base[:14], 7, *base[15:]) == UNSUPPORTED              # dtype
+    assert f(*base[:5], None, *base[6:]) == INVALID                 # dgate without gate
+    assert f(*base[:7], None, *base[8:]) == INVALID                 # no device offsets
+    assert f(*base[:18], None, *base[19:]) == INVALID               # no dq
+    assert f(*base[:4], A + 1, *base[5:]) == ALIGN                  # beta (bf16)
+    assert f(*base[:20], A + 2, *base[21:]) == ALIGN                # dv (fp32)
+    assert f(*base[:25], None, *base[26:]) == WORKSPACE
+    assert f(*base[:26], ws - 1, *base[27:]) == WORKSPACE
+    assert f(*base[:25], A + 16, *base[26:]) == ALIGN               # workspace alignment
+    bad = (ctypes.c_int32 * 2)(0, 15)                                # does not end at T
+    assert f(*base[:8], ctypes.cast(bad, ctypes.c_void_p), *base[9:]) == INVALID
