@@ -1,5 +1,5 @@
 /*
- * kda.h -- KDA (Kimi Delta Attention) forward on NVIDIA B200 (sm_100a).
+ * kda.h -- KDA (Kimi Delta Attention) forward, and its gradient, on NVIDIA B200 (sm_100a).
  *
  * A C-ABI library (libkda_b200.so).  Plain pointers and sizes only; every
  * pointer is a DEVICE pointer unless its name ends in _host.  The caller owns
@@ -271,11 +271,11 @@ int kda_state_compose(const float *transitions, const float *zero_states, int32_
  * strength, read, output gate); this is that recurrence differentiated by the
  * chain rule, token by token in reverse, with the states recomputed from
  * checkpoints every 64 tokens.  fp32 arithmetic; results are deterministic up
- * to the order of fp32 atomic additions across 32-column slices of dv.
+ * to the order of fp32 atomic additions across 16-column slices of dv.
  *
  * kda_bwd_workspace_size: bytes of workspace kda_bwd needs (0 for
  *   unsupported sizes): checkpoints ((total_tokens / 64 + num_seqs) * H * dk
- *   * dv floats) plus per-(sequence, head, 32 columns) scratch of 64 states.
+ *   * dv floats) plus per-(sequence, head, 16 columns) scratch of 64 states.
  *
  * kda_bwd:
  *   q, k, g       device [total_tokens][H][dk], dtype; v, gate, dy device

@@ -15,7 +15,7 @@
 //
 // Layout of the work: the columns of the state are independent in every step
 // except through the row sums (dq, dk, dg) and dbeta, so one CTA owns one
-// (sequence, head, 32-column slice of dv) and adds its share of those sums
+// (sequence, head, 16-column slice of dv) and adds its share of those sums
 // into fp32 outputs with atomics; dv, dgate and the initial-state gradient are
 // per column and stored directly.  Thread i (one per key channel) holds row i
 // of the state slice and of dS in registers; sums over the key channels (a, o,
@@ -33,7 +33,8 @@ namespace kda {
 namespace {
 
 constexpr int kBlk = 64;   // tokens between checkpoints
-constexpr int kCols = 32;  // state columns per CTA
+constexpr int kCols = 16;  // state columns per CTA (NC below)
+constexpr int NC = kCols;
 
 struct BwdParams {
     const void *q, *k, *v, *g, *beta, *gate, *dy;
@@ -45,12 +46,17 @@ struct BwdParams {
     float scale;
 };
 
-// x[c] summed over the 32 lanes of the warp, for every c; lane c returns
-// column c.  Recursive halving: at width s a lane keeps the half of its
-// columns selected by bit s of its lane id and adds the partner's copy.
-KDA_DEVICE float reduce_scatter32(float (&x)[32], int lane) {
+// x[c] (c < NC) summed over the 32 lanes of the warp; lane l returns column
+// l % NC.  With NC = 16 the two half-warps are added first.  Then recursive
+// halving: at width s a lane keeps the half of its columns selected by bit s
+// of its lane id and adds the partner's copy of that half.
+KDA_DEVICE float reduce_scatter(float (&x)[NC], int lane) {
+    if constexpr (NC == 16) {
 #pragma unroll
-    for (int s = 16; s >= 1; s >>= 1) {
+        for (int c = 0; c < 16; ++c) x[c] += __shfl_xor_sync(0xffffffffu, x[c], 16);
+    }
+#pragma unroll
+    for (int s = NC / 2; s >= 1; s >>= 1) {
         const bool up = lane & s;
 #pragma unroll
         for (int m = 0; m < s; ++m) {
@@ -65,26 +71,62 @@ KDA_DEVICE float reduce_scatter32(float (&x)[32], int lane) {
 // Column sums over all key channels of the CTA: out[c] = sum_i x_i[c].
 // Two barriers: the first also publishes the token's shared inputs.
 template <int NW>
-KDA_DEVICE void col_sum(float (&x)[32], float *red, float *out, int warp, int lane) {
-    red[warp * 32 + lane] = reduce_scatter32(x, lane);
+KDA_DEVICE void col_sum(float (&x)[NC], float *red, float *out, int warp, int lane) {
+    const float sx = reduce_scatter(x, lane);
+    if (lane < NC) red[warp * NC + lane] = sx;
     __syncthreads();
-    if (warp == 0) {
+    if (warp == 0 && lane < NC) {
         float t = 0.f;
 #pragma unroll
-        for (int w = 0; w < NW; ++w) t += red[w * 32 + lane];
+        for (int w = 0; w < NW; ++w) t += red[w * NC + lane];
         out[lane] = t;
     }
     __syncthreads();
 }
 
+// Three column sums and one scalar sum in one exchange: out[0, NC) = sum x,
+// out[NC, 2 NC) = sum y, out[2 NC, 3 NC) = sum z, out[3 NC] = sum w.
+constexpr int kRed3 = 3 * NC + 1;
+template <int NW>
+KDA_DEVICE void col_sum3(float (&x)[NC], float (&y)[NC], float (&z)[NC], float w, float *red,
+                         float *out, int warp, int lane) {
+    const float sx = reduce_scatter(x, lane);
+    const float sy = reduce_scatter(y, lane);
+    const float sz = reduce_scatter(z, lane);
+    const float sw = warp_sum(w);
+    float *r = red + warp * kRed3;
+    if (lane < NC) {
+        r[lane] = sx;
+        r[NC + lane] = sy;
+        r[2 * NC + lane] = sz;
+    }
+    if (lane == 0) r[3 * NC] = sw;
+    __syncthreads();
+    for (int e = threadIdx.x; e < kRed3; e += 32 * NW) {
+        float t = 0.f;
+#pragma unroll
+        for (int q = 0; q < NW; ++q) t += red[q * kRed3 + e];
+        out[e] = t;
+    }
+    __syncthreads();
+}
+
+struct FwdIn {  // one token's inputs to the forward step (v: column i, i < NC)
+    float k, g, beta, v;
+};
+struct RevIn {  // one token's inputs to the reverse step (v, gate, dy: column i, i < NC)
+    float k, q, g, beta, v, gate, dy;
+};
+
 template <int DK, typename T>
-__global__ void __launch_bounds__(DK) bwd_kernel(BwdParams p) {
+__global__ void __launch_bounds__(DK, 1) bwd_kernel(BwdParams p) {
     constexpr int NW = DK / 32;
-    // per-token column data, double-buffered by token parity so that a fast
-    // thread writing token t + 1 never overwrites what a slow one still reads
-    __shared__ float red[NW * 32];
-    __shared__ float cv[2][32], cgt[2][32], cdy[2][32];
-    __shared__ float ca[2][32], co[2][32], cdu[2][32];
+    // per-token shared data, double-buffered by token parity so that a fast
+    // thread writing the next token never overwrites what a slow one still
+    // reads (the barriers of one token separate uses two tokens apart)
+    __shared__ float red[NW * kRed3];
+    __shared__ float cv[2][NC], cgt[2][NC], cdy[2][NC];
+    __shared__ float ca[2][NC], cs[2][kRed3];
 
     const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
     const int nh = blockIdx.x, n = nh / p.H, h = nh % p.H;
@@ -101,123 +143,166 @@ __global__ void __launch_bounds__(DK) bwd_kernel(BwdParams p) {
     const float scale = p.scale;
     float *scr = p.scratch + ((size_t)(nh * gridDim.y + blockIdx.y) * kBlk * DK + i) * kCols;
     auto ck_row = [&](int b) { return p.ckpt + (((size_t)(ck0 + b) * H + h) * DK + i) * DV + j0; };
-    auto save = [](float *dst, const float (&x)[32]) {
+    auto save = [](float *dst, const float (&x)[NC]) {
 #pragma unroll
-        for (int c = 0; c < 32; c += 4)
+        for (int c = 0; c < NC; c += 4)
             *reinterpret_cast<float4 *>(dst + c) = make_float4(x[c], x[c + 1], x[c + 2], x[c + 3]);
     };
-    auto load = [](const float *src, float (&x)[32]) {
+    auto load = [](const float *src, float (&x)[NC]) {
 #pragma unroll
-        for (int c = 0; c < 32; c += 4) {
+        for (int c = 0; c < NC; c += 4) {
             const float4 f = *reinterpret_cast<const float4 *>(src + c);
             x[c] = f.x; x[c + 1] = f.y; x[c + 2] = f.z; x[c + 3] = f.w;
         }
     };
+    auto load_fwd = [&](int t) {
+        const size_t r = (size_t)t * H + h;
+        FwdIn x;
+        x.k = ld(k + r * DK + i);
+        x.g = ld(g + r * DK + i);
+        x.beta = ld(beta + r);
+        x.v = i < NC ? ld(v + r * DV + j0 + i) : 0.f;
+        return x;
+    };
+    auto load_rev = [&](int t) {
+        const size_t r = (size_t)t * H + h;
+        RevIn x;
+        x.k = ld(k + r * DK + i);
+        x.q = ld(q + r * DK + i);
+        x.g = ld(g + r * DK + i);
+        x.beta = ld(beta + r);
+        x.v = x.gate = x.dy = 0.f;
+        if (i < NC) {
+            const size_t rc = r * DV + j0 + i;
+            x.v = ld(v + rc);
+            x.gate = gate ? ld(gate + rc) : 1.f;
+            x.dy = ld(dy + rc);
+        }
+        return x;
+    };
 
     // S <- the state after token t (S holds the state before it)
-    auto forward_token = [&](int t, float (&S)[32]) {
+    auto fwd_step = [&](int t, const FwdIn &in, float (&S)[NC]) {
         const int par = t & 1;
-        const size_t r = (size_t)t * H + h;
-        const float ki = ld(k + r * DK + i);
-        const float al = __expf(ld(g + r * DK + i));
-        const float bt = ld(beta + r);
-        if (i < 32) cv[par][i] = ld(v + r * DV + j0 + i);
-        float x[32];
+        const float al = __expf(in.g);
+        if (i < NC) cv[par][i] = in.v;
+        float x[NC];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
+        for (int c = 0; c < NC; ++c) {
             S[c] *= al;
-            x[c] = S[c] * ki;
+            x[c] = S[c] * in.k;
         }
         col_sum<NW>(x, red, ca[par], warp, lane);
 #pragma unroll
-        for (int c = 0; c < 32; ++c) S[c] += ki * (bt * (cv[par][c] - ca[par][c]));
+        for (int c = 0; c < NC; ++c) S[c] += in.k * (in.beta * (cv[par][c] - ca[par][c]));
+    };
+    // forward over tokens [t0, t1) with the next token's inputs in flight
+    auto fwd_run = [&](int t0, int t1, float (&S)[NC], bool keep) {
+        if (t0 >= t1) return;
+        FwdIn cur = load_fwd(t0);
+        for (int t = t0; t < t1; ++t) {
+            if (keep) save(scr + (size_t)(t - t0) * DK * kCols, S);
+            else if ((t - bos) % kBlk == 0) save(ck_row((t - bos) / kBlk), S);
+            const FwdIn nxt = t + 1 < t1 ? load_fwd(t + 1) : cur;
+            fwd_step(t, cur, S);
+            cur = nxt;
+        }
     };
 
     // ---- forward sweep: a checkpoint at the start of every block
-    float S[32];
+    float S[NC];
 #pragma unroll
-    for (int c = 0; c < 32; ++c) S[c] = p.s0 ? p.s0[((size_t)nh * DK + i) * DV + j0 + c] : 0.f;
-    for (int b = 0; b < nb; ++b) {
-        save(ck_row(b), S);
-        if (b + 1 < nb)
-            for (int t = bos + b * kBlk; t < bos + (b + 1) * kBlk; ++t) forward_token(t, S);
+    for (int c = 0; c < NC; ++c) S[c] = p.s0 ? p.s0[((size_t)nh * DK + i) * DV + j0 + c] : 0.f;
+    if (nb > 0) {
+        fwd_run(bos, bos + (nb - 1) * kBlk, S, false);
+        save(ck_row(nb - 1), S);
     }
 
     // ---- reverse sweep
-    float dS[32];
+    float dS[NC];
 #pragma unroll
-    for (int c = 0; c < 32; ++c) dS[c] = p.dsT ? p.dsT[((size_t)nh * DK + i) * DV + j0 + c] : 0.f;
+    for (int c = 0; c < NC; ++c) dS[c] = p.dsT ? p.dsT[((size_t)nh * DK + i) * DV + j0 + c] : 0.f;
     for (int b = nb - 1; b >= 0; --b) {
         const int tb = bos + b * kBlk, te = min(eos, tb + kBlk);
         // the last token walked (tb + kBlk of the previous block, or the
         // forward sweep's) may share a buffer parity with the first one below
         __syncthreads();
         load(ck_row(b), S);
-        for (int t = tb; t < te; ++t) {  // the block's states S_{t-1}, forwards
-            save(scr + (size_t)(t - tb) * DK * kCols, S);
-            if (t + 1 < te) forward_token(t, S);
-        }
+        // the block's states S_{t-1} into scratch (the last one saved, not stepped)
+        fwd_run(tb, te - 1, S, true);
+        save(scr + (size_t)(te - 1 - tb) * DK * kCols, S);
+
+        RevIn cur = load_rev(te - 1);
+        float Sp[NC];
+        load(scr + (size_t)(te - 1 - tb) * DK * kCols, Sp);
         for (int t = te - 1; t >= tb; --t) {
             const int par = t & 1;
             const size_t r = (size_t)t * H + h;
-            const float ki = ld(k + r * DK + i), qi = ld(q + r * DK + i);
-            const float al = __expf(ld(g + r * DK + i));
-            const float bt = ld(beta + r);
-            if (i < 32) {
-                const size_t rc = r * DV + j0 + i;
-                cv[par][i] = ld(v + rc);
-                cgt[par][i] = gate ? ld(gate + rc) : 1.f;
-                cdy[par][i] = ld(dy + rc);
+            RevIn nxt = cur;
+            float Sn[NC];
+            if (t > tb) {
+                nxt = load_rev(t - 1);
+                load(scr + (size_t)(t - 1 - tb) * DK * kCols, Sn);
             }
-            float Sp[32], x[32];
-            load(scr + (size_t)(t - tb) * DK * kCols, Sp);
+            const float al = __expf(cur.g);
+            if (i < NC) {
+                cv[par][i] = cur.v;
+                cgt[par][i] = cur.gate;
+                cdy[par][i] = cur.dy;
+            }
+            // one exchange: a = S'^T k, b = S'^T q, c = dS^T k (dS = dL/dS_t
+            // without this token's read) and k.q
+            float x[NC], y[NC], z[NC];
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
+            for (int c = 0; c < NC; ++c) {
                 Sp[c] *= al;
-                x[c] = Sp[c] * ki;
+                x[c] = Sp[c] * cur.k;
+                y[c] = Sp[c] * cur.q;
+                z[c] = dS[c] * cur.k;
             }
-            col_sum<NW>(x, red, ca[par], warp, lane);  // a = S'^T k
-            // u_c = beta (v_c - a_c);  S_t = S' + k u^T;  o = S_t^T (scale q)
-#pragma unroll
-            for (int c = 0; c < 32; ++c)
-                x[c] = (Sp[c] + ki * (bt * (cv[par][c] - ca[par][c]))) * (scale * qi);
-            col_sum<NW>(x, red, co[par], warp, lane);
-            if (i < 32 && p.dgate) p.dgate[r * DV + j0 + i] = cdy[par][i] * co[par][i];
-            float dqi = 0.f;
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                const float doc = cgt[par][c] * cdy[par][c];
-                const float st = Sp[c] + ki * (bt * (cv[par][c] - ca[par][c]));
-                dqi += st * doc;
-                dS[c] += scale * qi * doc;
-                x[c] = dS[c] * ki;
+            col_sum3<NW>(x, y, z, cur.k * cur.q, red, cs[par], warp, lane);
+            const float *A = cs[par], *Bq = cs[par] + NC, *C = cs[par] + 2 * NC;
+            const float kq = cs[par][3 * NC], bt = cur.beta;
+            if (i < NC) {  // per column: u, o (= scale (b + (k.q) u)), du, dv, dgate
+                const float u = bt * (cur.v - A[i]);
+                const float o = scale * (Bq[i] + kq * u);
+                const float du = C[i] + scale * kq * (cur.gate * cur.dy);
+                p.dv[r * DV + j0 + i] = bt * du;
+                if (p.dgate) p.dgate[r * DV + j0 + i] = cur.dy * o;
             }
-            col_sum<NW>(x, red, cdu[par], warp, lane);  // du = dS^T k
-            if (i < 32) p.dv[r * DV + j0 + i] = bt * cdu[par][i];
             if (i == 0) {
                 float db = 0.f;
 #pragma unroll
-                for (int c = 0; c < 32; ++c) db += cdu[par][c] * (cv[par][c] - ca[par][c]);
+                for (int c = 0; c < NC; ++c) {
+                    const float du = C[c] + scale * kq * (cgt[par][c] * cdy[par][c]);
+                    db += du * (cv[par][c] - A[c]);
+                }
                 atomicAdd(p.dbeta + r, db);
             }
-            float dki = 0.f, dgi = 0.f;
+            float dqi = 0.f, dki = 0.f, dgi = 0.f;
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                const float uc = bt * (cv[par][c] - ca[par][c]);
-                const float da = -bt * cdu[par][c];
-                dki += dS[c] * uc + Sp[c] * da;
-                const float dsp = dS[c] + ki * da;
+            for (int c = 0; c < NC; ++c) {
+                const float doc = cgt[par][c] * cdy[par][c];
+                const float uc = bt * (cv[par][c] - A[c]);
+                dqi += (Sp[c] + cur.k * uc) * doc;              // S_t do
+                const float dsc = dS[c] + scale * cur.q * doc;  // dL/dS_t
+                const float da = -bt * (C[c] + scale * kq * doc);
+                dki += dsc * uc + Sp[c] * da;
+                const float dsp = dsc + cur.k * da;              // dL/dS'
                 dgi += dsp * Sp[c];
-                dS[c] = al * dsp;
+                dS[c] = al * dsp;                                // dL/dS_{t-1}
             }
             atomicAdd(p.dq + r * DK + i, scale * dqi);
             atomicAdd(p.dk + r * DK + i, dki);
             atomicAdd(p.dg + r * DK + i, dgi);
+            cur = nxt;
+#pragma unroll
+            for (int c = 0; c < NC; ++c) Sp[c] = Sn[c];
         }
     }
     if (p.ds0) {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) p.ds0[((size_t)nh * DK + i) * DV + j0 + c] = dS[c];
+        for (int c = 0; c < NC; ++c) p.ds0[((size_t)nh * DK + i) * DV + j0 + c] = dS[c];
     }
 }
 
