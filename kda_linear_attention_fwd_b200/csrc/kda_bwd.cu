@@ -33,6 +33,7 @@ namespace kda {
 namespace {
 
 constexpr int kBlk = 64;   // tokens between checkpoints
+constexpr int kAhead = 8;  // tokens ahead whose lines are prefetched into L2
 constexpr int kCols = 16;  // state columns per CTA (NC below)
 constexpr int NC = kCols;
 
@@ -111,6 +112,10 @@ KDA_DEVICE void col_sum3(float (&x)[NC], float (&y)[NC], float (&z)[NC], float w
     __syncthreads();
 }
 
+KDA_DEVICE void prefetch_l2(const void *ptr) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
+}
+
 struct FwdIn {  // one token's inputs to the forward step (v: column i, i < NC)
     float k, g, beta, v;
 };
@@ -181,6 +186,26 @@ __global__ void __launch_bounds__(DK, 1) bwd_kernel(BwdParams p) {
         return x;
     };
 
+    // L2 prefetch of token t's input lines (one thread per 128-byte line of a
+    // row; t must be a token of this sequence)
+    constexpr int kLine = 128 / (int)sizeof(T);
+    auto prefetch_in = [&](int t, bool rev) {
+        const size_t r = (size_t)t * H + h;
+        if (i % kLine == 0) {
+            prefetch_l2(k + r * DK + i);
+            prefetch_l2(g + r * DK + i);
+            if (rev) prefetch_l2(q + r * DK + i);
+        }
+        if (i == 0) {
+            prefetch_l2(beta + r);
+            prefetch_l2(v + r * DV + j0);
+            if (rev) {
+                prefetch_l2(dy + r * DV + j0);
+                if (gate) prefetch_l2(gate + r * DV + j0);
+            }
+        }
+    };
+
     // S <- the state after token t (S holds the state before it)
     auto fwd_step = [&](int t, const FwdIn &in, float (&S)[NC]) {
         const int par = t & 1;
@@ -200,7 +225,9 @@ __global__ void __launch_bounds__(DK, 1) bwd_kernel(BwdParams p) {
     auto fwd_run = [&](int t0, int t1, float (&S)[NC], bool keep) {
         if (t0 >= t1) return;
         FwdIn cur = load_fwd(t0);
+        for (int t = t0; t < t0 + kAhead && t < t1; ++t) prefetch_in(t, false);
         for (int t = t0; t < t1; ++t) {
+            if (t + kAhead < t1) prefetch_in(t + kAhead, false);
             if (keep) save(scr + (size_t)(t - t0) * DK * kCols, S);
             else if ((t - bos) % kBlk == 0) save(ck_row((t - bos) / kBlk), S);
             const FwdIn nxt = t + 1 < t1 ? load_fwd(t + 1) : cur;
@@ -235,9 +262,17 @@ __global__ void __launch_bounds__(DK, 1) bwd_kernel(BwdParams p) {
         RevIn cur = load_rev(te - 1);
         float Sp[NC];
         load(scr + (size_t)(te - 1 - tb) * DK * kCols, Sp);
+        for (int t = te - 1; t >= tb && t >= te - kAhead; --t) {
+            prefetch_in(t, true);
+            prefetch_l2(scr + (size_t)(t - tb) * DK * kCols);
+        }
         for (int t = te - 1; t >= tb; --t) {
             const int par = t & 1;
             const size_t r = (size_t)t * H + h;
+            if (t - kAhead >= tb) {
+                prefetch_in(t - kAhead, true);
+                prefetch_l2(scr + (size_t)(t - kAhead - tb) * DK * kCols);
+            }
             RevIn nxt = cur;
             float Sn[NC];
             if (t > tb) {
