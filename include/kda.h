@@ -270,12 +270,12 @@ int kda_state_compose(const float *transitions, const float *zero_states, int32_
  * section "第一关：KDA 解决算得动": forget, corrective write with an update
  * strength, read, output gate); this is that recurrence differentiated by the
  * chain rule, token by token in reverse, with the states recomputed from
- * checkpoints every 64 tokens.  fp32 arithmetic; results are deterministic up
+ * checkpoints every 16 tokens.  fp32 arithmetic; results are deterministic up
  * to the order of fp32 atomic additions across 16-column slices of dv.
  *
  * kda_bwd_workspace_size: bytes of workspace kda_bwd needs (0 for
- *   unsupported sizes): checkpoints ((total_tokens / 64 + num_seqs) * H * dk
- *   * dv floats) plus per-(sequence, head, 16 columns) scratch of 64 states.
+ *   unsupported sizes): checkpoints ((total_tokens / 16 + num_seqs) * H * dk
+ *   * dv floats) plus per-(sequence, head, 16 columns) scratch of 16 states.
  *
  * kda_bwd:
  *   q, k, g       device [total_tokens][H][dk], dtype; v, gate, dy device

@@ -32,7 +32,7 @@
 namespace kda {
 namespace {
 
-constexpr int kBlk = 64;   // tokens between checkpoints
+constexpr int kBlk = 16;   // tokens between checkpoints (a block's states stay L2-resident)
 constexpr int kAhead = 8;  // tokens ahead whose lines are prefetched into L2
 constexpr int kCols = 16;  // state columns per CTA (NC below)
 constexpr int NC = kCols;

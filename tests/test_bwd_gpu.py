@@ -54,7 +54,7 @@ def _oracle(inp, dy, dsf, scale, gate=True):
 @pytest.mark.parametrize("dtype,dk,dv", [("bf16", 128, 128), ("bf16", 64, 128),
                                           ("f32", 64, 64), ("f32", 128, 64)])
 def test_bwd_matches_oracle(cuda_lib, dtype, dk, dv):
-    """Varlen with an empty, a partial-block and multi-block sequences (64-token
+    """Varlen with an empty, a partial-block and multi-block sequences (16-token
     checkpoint blocks), initial state, final-state gradient and a gate."""
     w = W.custom(dtype=dtype, H=2, dk=dk, dv=dv, lengths=(0, 5, 64, 130, 300),
                  init_state=True, seed=91)
