@@ -196,6 +196,16 @@ def cpu_baseline(w, threads=None, tokens=None):
     return tokens / dt, used, f"{tokens} tokens x {w.H} heads of {w.name} (fp64, per token)"
 
 
+def workload_config(w, ws):
+    """The `config` keys both arms share (the workload, named by its sizes)."""
+    T, N = w.total_tokens, w.num_seqs
+    return {"workload": f"{w.name}: {N} sequence(s), {T} tokens, H={w.H}, "
+                        f"dk={w.dk}, dv={w.dv}, {w.dtype}, chunk=16",
+            "global_batch": ws * N, "seq_len": T,
+            "parallelism": f"replicas x{ws} (sequences/heads independent)",
+            "l2": "inputs larger than L2 (%.1f GB per step)" % (prefill_bytes(w, T, N) / 1e9)}
+
+
 def run_reference(args, ws, rank):
     """Reference arm: the fp64 CPU oracle, timed on the host cores, on a
     bounded sample of the same workload each step."""
@@ -215,8 +225,7 @@ def run_reference(args, ws, rank):
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "seq_len": w.lengths[0], "heads": w.H,
-                       "dk": w.dk, "dv": w.dv, "sample_tokens_per_step": tokens},
+            "config": dict(workload_config(w, ws), sample_tokens_per_step=tokens),
             "impl": "reference",
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": used, "kind": "oracle",
                              "sample": sample},
@@ -549,12 +558,7 @@ def main():
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": w.dtype, "data": "synthetic",
-                "config": {"workload": f"{w.name}: {N} sequence(s), {T} tokens, H={w.H}, "
-                                       f"dk={w.dk}, dv={w.dv}, {w.dtype}, chunk=16",
-                           "global_batch": ws * N, "seq_len": T,
-                           "parallelism": f"replicas x{ws} (sequences/heads independent)",
-                           "l2": "inputs larger than L2 (%.1f GB per step)" % (pbytes / 1e9),
-                           "piece_len": plan["piece_len"]},
+                "config": dict(workload_config(w, ws), piece_len=plan["piece_len"]),
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": plan["launches"] * args.steps, "clocks": clk, "decode": dec,
                 "extended": exm, "kcp": kcpm, "backward": bwdm}
