@@ -271,11 +271,11 @@ int kda_state_compose(const float *transitions, const float *zero_states, int32_
  * strength, read, output gate); this is that recurrence differentiated by the
  * chain rule, token by token in reverse, with the states recomputed from
  * checkpoints every 16 tokens.  fp32 arithmetic; results are deterministic up
- * to the order of fp32 atomic additions across 16-column slices of dv.
+ * to the order of fp32 atomic additions across 8-column slices of dv.
  *
  * kda_bwd_workspace_size: bytes of workspace kda_bwd needs (0 for
  *   unsupported sizes): checkpoints ((total_tokens / 16 + num_seqs) * H * dk
- *   * dv floats) plus per-(sequence, head, 16 columns) scratch of 16 states.
+ *   * dv floats) plus per-(sequence, head, 8 columns) scratch of 16 states.
  *
  * kda_bwd:
  *   q, k, g       device [total_tokens][H][dk], dtype; v, gate, dy device

@@ -15,7 +15,7 @@
 //
 // Layout of the work: the columns of the state are independent in every step
 // except through the row sums (dq, dk, dg) and dbeta, so one CTA owns one
-// (sequence, head, 16-column slice of dv) and adds its share of those sums
+// (sequence, head, 8-column slice of dv) and adds its share of those sums
 // into fp32 outputs with atomics; dv, dgate and the initial-state gradient are
 // per column and stored directly.  Thread i (one per key channel) holds row i
 // of the state slice and of dS in registers; sums over the key channels (a, o,
@@ -34,7 +34,7 @@ namespace {
 
 constexpr int kBlk = 16;   // tokens between checkpoints (a block's states stay L2-resident)
 constexpr int kAhead = 8;  // tokens ahead whose lines are prefetched into L2
-constexpr int kCols = 16;  // state columns per CTA (NC below)
+constexpr int kCols = 8;   // state columns per CTA (NC below)
 constexpr int NC = kCols;
 
 struct BwdParams {
@@ -48,13 +48,18 @@ struct BwdParams {
 };
 
 // x[c] (c < NC) summed over the 32 lanes of the warp; lane l returns column
-// l % NC.  With NC = 16 the two half-warps are added first.  Then recursive
-// halving: at width s a lane keeps the half of its columns selected by bit s
-// of its lane id and adds the partner's copy of that half.
+// l % NC.  With NC < 32 the lanes 16 (and 8) apart are added first.  Then
+// recursive halving: at width s a lane keeps the half of its columns selected
+// by bit s of its lane id and adds the partner's copy of that half.
 KDA_DEVICE float reduce_scatter(float (&x)[NC], int lane) {
-    if constexpr (NC == 16) {
+    static_assert(NC == 8 || NC == 16 || NC == 32, "slice width");
+    if constexpr (NC <= 16) {
 #pragma unroll
-        for (int c = 0; c < 16; ++c) x[c] += __shfl_xor_sync(0xffffffffu, x[c], 16);
+        for (int c = 0; c < NC; ++c) x[c] += __shfl_xor_sync(0xffffffffu, x[c], 16);
+    }
+    if constexpr (NC <= 8) {
+#pragma unroll
+        for (int c = 0; c < NC; ++c) x[c] += __shfl_xor_sync(0xffffffffu, x[c], 8);
     }
 #pragma unroll
     for (int s = NC / 2; s >= 1; s >>= 1) {
@@ -124,7 +129,8 @@ struct RevIn {  // one token's inputs to the reverse step (v, gate, dy: column i
 };
 
 template <int DK, typename T>
-__global__ void __launch_bounds__(DK, 1) bwd_kernel(BwdParams p) {
+// 512 threads per SM at least (four 128-thread CTAs): more chains share each SM
+__global__ void __launch_bounds__(DK, 512 / DK) bwd_kernel(BwdParams p) {
     constexpr int NW = DK / 32;
     // per-token shared data, double-buffered by token parity so that a fast
     // thread writing the next token never overwrites what a slow one still
