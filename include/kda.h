@@ -125,6 +125,26 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const void *g, co
                   void *workspace, size_t workspace_bytes, kda_stream_t stream);
 
 /*
+ * Errors found on the device by kda_chunk_fwd / kda_chunk_fwd_ex are kept in
+ * the first bytes of the workspace they ran with (cleared by each call):
+ * offsets that are not monotone or do not end at total_tokens; a bounded
+ * device wait that gave up; and, in the checked build of the library
+ * (libkda_b200_checked.so, compiled with -DKDA_CHECK_G), a log-decay value
+ * outside the precondition ln(0.0067) <= g <= 0 (with KDA_FLAG_CLAMP_DECAY
+ * only g <= 0 is required), or NaN.  The release build does not check g.
+ *
+ * kda_chunk_fwd_check: waits for `stream` (this call, unlike the others,
+ * synchronises), then reads those words.  Returns KDA_OK, KDA_ERR_INVALID_ARG
+ * (bad offsets, or g out of range in the checked build; also for a NULL or
+ * too-small workspace argument), KDA_ERR_TIMEOUT, or KDA_ERR_CUDA.  Call it
+ * after the prefill and before the workspace is reused.
+ *
+ * kda_build_checks_g: 1 in the checked build, 0 in the release build.
+ */
+int kda_chunk_fwd_check(const void *workspace, size_t workspace_bytes, kda_stream_t stream);
+int kda_build_checks_g(void);
+
+/*
  * kda_chunk_fwd without a workspace argument, for callers that cannot
  * allocate device memory when they run the layer (code running inside an
  * allocator or memory-pool callback, runtimes that hand out only fixed

@@ -1,10 +1,13 @@
 """Build libkda_b200.so (in-tree, sm_100a) with nvcc.
 
-    python -m kda_linear_attention_fwd_b200.build [--force] [--verbose]
+    python -m kda_linear_attention_fwd_b200.build [--force] [--verbose] [--checked]
 
 Each .cu under csrc/ is compiled in parallel to an object in _build/, then
 linked into kda_linear_attention_fwd_b200/libkda_b200.so.  Rebuilds only
-when a source or header is newer than the library.
+when a source or header is newer than the library.  --checked builds the
+checked variant instead (-DKDA_CHECK_G: the prefill verifies the log-decay
+precondition on the device) into libkda_b200_checked.so, objects in
+_build/checked/.
 """
 from __future__ import annotations
 
@@ -19,6 +22,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libkda_b200.so")
+LIB_CHECKED = os.path.join(HERE, "libkda_b200_checked.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -35,21 +39,26 @@ def _deps():
         os.path.join(ROOT, "include", "kda.h")]
 
 
-def stale() -> bool:
-    if not os.path.exists(LIB):
+def stale(checked: bool = False) -> bool:
+    lib = LIB_CHECKED if checked else LIB
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(p) > t for p in _deps())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not stale():
-        return LIB
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, checked: bool = False) -> str:
+    lib = LIB_CHECKED if checked else LIB
+    if not force and not stale(checked):
+        return lib
+    bdir = os.path.join(BUILD, "checked") if checked else BUILD
+    os.makedirs(bdir, exist_ok=True)
     extra = ["-Xptxas", "-v"] if verbose else []
+    if checked:
+        extra = extra + ["-DKDA_CHECK_G"]
 
     def compile_one(src):
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(bdir, os.path.basename(src)[:-3] + ".o")
         cmd = [NVCC] + FLAGS + extra + ["-c", src, "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
@@ -60,14 +69,15 @@ def build(force: bool = False, verbose: bool = False) -> str:
 
     with ThreadPoolExecutor(max(1, min(8, os.cpu_count() or 1))) as ex:
         objs = list(ex.map(compile_one, _sources()))
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = lib + f".tmp{os.getpid()}"
     cmd = [NVCC] + ARCH + ["-shared", "-o", tmp] + objs + ["-lcudart"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv,
+                checked="--checked" in sys.argv))

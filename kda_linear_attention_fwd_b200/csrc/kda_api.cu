@@ -1,6 +1,7 @@
 // C-ABI entry points of libkda_b200.so (declared in include/kda.h): argument
 // validation, the piece plan, and the launch sequence.  No allocation, no
 // host synchronisation, no exceptions across the boundary.
+#include <algorithm>
 #include <cstdlib>
 #include <cstring>
 
@@ -17,6 +18,32 @@ cudaError_t launch_plan(const int32_t *cu, int num_seqs, int total_tokens, int p
 cudaError_t launch_scan(const PrefillParams &p, int dk, int dv, cudaStream_t st);
 cudaError_t launch_prefill_chunks(const PrefillParams &p, bool bf16, int dk, int dv,
                                   bool summaries, cudaStream_t st);
+
+#ifdef KDA_CHECK_G
+// Checked builds: the log-decay precondition ln(0.0067) <= g <= 0 (with the
+// clamp flag only g <= 0, the kernels raise smaller values to the floor);
+// NaN fails either test.  A violation sets bit 4 of the workspace error word.
+template <typename T>
+__global__ void __launch_bounds__(256) check_g_kernel(const T *g, long n, int clamp, int32_t *err) {
+    bool bad = false;
+    for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) {
+        const float x = ld(g + i);
+        bad |= !(x <= 0.f && (clamp || x >= kLogDecayFloor));
+    }
+    if (__syncthreads_or(bad) && threadIdx.x == 0) atomicOr(err, 4);
+}
+
+cudaError_t launch_check_g(const void *g, bool bf16, long n, int clamp, int32_t *err,
+                           cudaStream_t st) {
+    if (n <= 0) return cudaSuccess;
+    const unsigned blocks = (unsigned)std::min<long>((n + 255) / 256, 1184);
+    if (bf16)
+        check_g_kernel<<<blocks, 256, 0, st>>>((const __nv_bfloat16 *)g, n, clamp, err);
+    else
+        check_g_kernel<<<blocks, 256, 0, st>>>((const float *)g, n, clamp, err);
+    return cudaGetLastError();
+}
+#endif
 }  // namespace kda
 
 namespace {
@@ -159,6 +186,12 @@ int kda_chunk_fwd_ex(const void *q, const void *k, const void *v, const void *g,
                                      (int32_t *)(ws + WL.off_seq_first),
                                      (int4 *)(ws + WL.off_pieces), stream);
     if (e != cudaSuccess) return KDA_ERR_CUDA;
+#ifdef KDA_CHECK_G
+    // after the plan kernel, which clears the error word
+    e = kda::launch_check_g(g, bf16, (long)total_tokens * H * dk, (flags & kda::FLAG_CLAMP_G) ? 1 : 0,
+                            p.err, stream);
+    if (e != cudaSuccess) return KDA_ERR_CUDA;
+#endif
     const bool multi = total_tokens > L;  // some sequence may have >1 piece
     if (multi) {
         e = kda::launch_prefill_chunks(p, bf16, dk, dv, true, stream);
@@ -181,6 +214,25 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const void *g, co
     return kda_chunk_fwd_ex(q, k, v, g, beta, gate, out, cu_seqlens, cu_seqlens_host, num_seqs,
                             total_tokens, H, dk, dv, dtype, scale, qk_l2norm, initial_state,
                             final_state, 0, nullptr, nullptr, workspace, workspace_bytes, stream);
+}
+
+int kda_chunk_fwd_check(const void *workspace, size_t workspace_bytes, kda_stream_t stream) {
+    if (!workspace || workspace_bytes < 3 * sizeof(int32_t)) return KDA_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return KDA_ERR_CUDA;
+    int32_t h[3];
+    if (cudaMemcpy(h, workspace, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    if (h[1] != 0 || (h[2] & 4)) return KDA_ERR_INVALID_ARG;  // offsets, or g out of range
+    if (h[2] & 3) return KDA_ERR_TIMEOUT;                       // a device wait gave up
+    return KDA_OK;
+}
+
+int kda_build_checks_g(void) {
+#ifdef KDA_CHECK_G
+    return 1;
+#else
+    return 0;
+#endif
 }
 
 int kda_decode_step_ex(const void *q, const void *k, const void *v, const void *g, const void *beta,

@@ -14,18 +14,22 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libkda_b200.so")
+# the checked build (-DKDA_CHECK_G): the prefill also verifies the log-decay range
+LIB_CHECKED_PATH = os.path.join(_HERE, "libkda_b200_checked.so")
 
 KDA_DTYPE_F32 = 0
 KDA_DTYPE_BF16 = 1
 
 EXPORTS = ("kda_status_string", "kda_chunk_fwd_workspace_size", "kda_chunk_fwd_plan",
            "kda_chunk_fwd", "kda_decode_step", "kda_chunk_fwd_ex", "kda_decode_step_ex",
-           "kda_chunk_fwd_summary", "kda_state_compose", "kda_bwd_workspace_size", "kda_bwd")
+           "kda_chunk_fwd_summary", "kda_state_compose", "kda_bwd_workspace_size", "kda_bwd",
+           "kda_chunk_fwd_check", "kda_build_checks_g")
 
 # flags of the extended entry points (include/kda.h)
 FLAG_QK_L2NORM, FLAG_BETA_LOGITS, FLAG_GATE_LOGITS, FLAG_CLAMP_DECAY = 1, 2, 4, 8
 
 _lib = None
+_lib_checked = None
 
 
 class KdaError(RuntimeError):
@@ -37,8 +41,23 @@ class KdaError(RuntimeError):
 def load(path: str = LIB_PATH):
     """Load the CUDA library (raises if it has not been built)."""
     global _lib
-    if _lib is not None:
+    if path == LIB_PATH and _lib is not None:
         return _lib
+    lib = _open(path)
+    if path == LIB_PATH:
+        _lib = lib
+    return lib
+
+
+def load_checked():
+    """The checked build of the library (a separate handle)."""
+    global _lib_checked
+    if _lib_checked is None:
+        _lib_checked = _open(LIB_CHECKED_PATH)
+    return _lib_checked
+
+
+def _open(path):
     if not os.path.exists(path):
         raise RuntimeError(
             f"{path} not found: build it first (python -m kda_linear_attention_fwd_b200.build)")
@@ -72,7 +91,10 @@ def load(path: str = LIB_PATH):
     lib.kda_bwd.argtypes = [P, P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, ctypes.c_int,
                             f32, P, P, P, P, P, P, P, P, P, P, sz, P]
     lib.kda_bwd.restype = ctypes.c_int
-    _lib = lib
+    lib.kda_chunk_fwd_check.argtypes = [P, sz, P]
+    lib.kda_chunk_fwd_check.restype = ctypes.c_int
+    lib.kda_build_checks_g.argtypes = []
+    lib.kda_build_checks_g.restype = ctypes.c_int
     return lib
 
 
@@ -287,3 +309,11 @@ def bwd(q, k, v, g, beta, gate, dy, cu_seqlens, *, scale=1.0, initial_state=None
                      workspace.numel(), _stream(stream))
     _check("kda_bwd", st)
     return out
+
+
+def chunk_fwd_check(workspace, stream=None, lib=None) -> int:
+    """Status of the last prefill that used `workspace` (waits for the
+    stream): 0 = KDA_OK, else a kda_status code (see include/kda.h)."""
+    lib = lib or load()
+    return int(lib.kda_chunk_fwd_check(_ptr(workspace), workspace.numel() * workspace.element_size(),
+                                       _stream(stream)))

@@ -234,3 +234,16 @@ def test_bwd_validation(lib):
     assert f(*base[:25], A + 16, *base[26:]) == ALIGN               # workspace alignment
     bad = (ctypes.c_int32 * 2)(0, 15)                                # does not end at T
     assert f(*base[:8], ctypes.cast(bad, ctypes.c_void_p), *base[9:]) == INVALID
+
+
+def test_checked_build_exports_the_same_symbols(lib):
+    build.build(checked=True)
+    chk = kda.load_checked()
+    for name in declared_functions():
+        assert hasattr(chk, name), name
+    assert lib.kda_build_checks_g() == 0 and chk.kda_build_checks_g() == 1
+
+
+def test_chunk_fwd_check_validation(lib):
+    assert lib.kda_chunk_fwd_check(None, 1 << 20, None) == INVALID
+    assert lib.kda_chunk_fwd_check(A, 8, None) == INVALID  # smaller than the error words
