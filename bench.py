@@ -23,6 +23,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import torch
@@ -253,7 +254,8 @@ def main():
                     help="skip the extended-path measurement (flags + state snapshots)")
     ap.add_argument("--no-bwd", action="store_true",
                     help="skip the backward measurement")
-    ap.add_argument("--out-dir", default=os.path.join(ROOT, "gpurun_out"))
+    ap.add_argument("--out-dir", default=os.path.join(tempfile.gettempdir(), "kda_bench"),
+                    help="where the nvidia-smi clock samples of the timed region are written")
     ap.add_argument("--ref-tokens", type=int, default=0,
                     help="reference arm: tokens per step sample (0 = scale with cores)")
     args = ap.parse_args()
