@@ -47,12 +47,35 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum, summed over the four
-# launches) of one call, from one ncu capture of
-#   bench.py --steps 1 --warmup 1 --no-e2e --no-cpu --no-decode --no-ex --no-kcp
-# keyed by (workload, piece length).  Valid only for the kernels as captured:
-# a change to any kernel of the call makes the figure stale (report null then).
-NCU_CALL_TRAFFIC = {("long_bf16", 3552): 10.18e9}
+# DRAM traffic of the dominant kernel, per launch: read from the committed
+# ncu summary profiles/traffic.json, which records the figure together with a
+# hash of the CUDA sources it was captured from.  When the sources differ
+# from that hash (a kernel changed since the capture) the figure is stale and
+# `traffic` is reported as null.
+def source_hash():
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "kda_linear_attention_fwd_b200", "csrc")
+    for path in sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh"))):
+        with open(path, "rb") as f:
+            h.update(os.path.basename(path).encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload):
+    """(bytes per launch of the dominant kernel, kernel name, source) or
+    (None, None, reason)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None, None, "no committed capture"
+    with open(path) as f:
+        d = json.load(f).get(workload)
+    if not d:
+        return None, None, "no capture for this workload"
+    if d.get("source_hash") != source_hash():
+        return None, d.get("kernel"), "stale: kernel sources changed since the capture"
+    return float(d["bytes_per_launch"]), d.get("kernel"), d.get("source", "profiles/traffic.json")
 
 
 def prefill_bytes(w, T, N):
@@ -317,9 +340,11 @@ def main():
     pflops = prefill_flops(w, T)
     hbm = pk["hbm_gbs"]
     achieved = pbytes / (ms / 1e3) / 1e9
+    traffic, _, traffic_src = measured_traffic(args.workload)
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                 "frac": achieved / hbm,
-                "traffic": NCU_CALL_TRAFFIC.get((args.workload, plan["piece_len"])),
+                "traffic": traffic,
+                "traffic_source": traffic_src,
                 "kernel": "kda_chunk_fwd call (%d launches)" % plan["launches"],
                 "peak_source": f"{pk_kind} hbm_gbs",
                 "tensor_tflops": pflops / (ms / 1e3) / 1e12,

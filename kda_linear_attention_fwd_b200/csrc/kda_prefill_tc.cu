@@ -49,32 +49,6 @@
 #include <cstring>
 #include <type_traits>
 
-// Optional timeline hooks for one CTA (piece 1, head 0), compiled only with
-// -DKDA_TC5_TRACE: SM clock at fixed points of the state warpgroup's and the
-// prep warps' chunk loops, read back through kda_tc5_trace_copy().
-#ifdef KDA_TC5_TRACE
-__device__ unsigned long long g_kda_tc5_trace[8192];
-// traced CTA: piece 0 of head 1 of the output pass, or, with
-// -DKDA_TRACE_SUMMARY, piece 1 of head 0 of the summary pass
-#ifdef KDA_TRACE_SUMMARY
-#define KDA_TRACE_HERE (!OUT && blockIdx.x == (unsigned)p.H)
-#else
-#define KDA_TRACE_HERE (OUT && blockIdx.x == 1)
-#endif
-#define KDA_MARK(cond, slot)                                                          \
-    do {                                                                              \
-        if ((cond) && KDA_TRACE_HERE && (slot) < 8192)                                \
-            g_kda_tc5_trace[(slot)] = clock64();                                      \
-        __syncwarp();                                                                 \
-    } while (0)
-extern "C" int kda_tc5_trace_copy(unsigned long long *host, int n) {
-    return cudaMemcpyFromSymbol(host, g_kda_tc5_trace, sizeof(unsigned long long) * n) ==
-                   cudaSuccess ? 0 : -1;
-}
-#else
-#define KDA_MARK(cond, slot) do { } while (0)
-#endif
-
 namespace kda {
 namespace tc5 {
 
@@ -367,11 +341,9 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
         for (int c = 0; c < nchunks; ++c) {
             const int stg = c % kStages;
             const uint32_t d1_col = Lay::COL_D1 + 32 * (c & 1);
-            KDA_MARK(tid == 0 && c < 128, c * 16 + 0);
             if (OUT) cp_async_wait<0>();  // this thread's pieces of the gate tile of chunk c - 1
             bar_sync(bar_wg, 128);        // state-pass TMEM stores; gate tile; y(c - 2) stored
             if (OUT) load_gate(c);
-            KDA_MARK(tid == 0 && c < 128, c * 16 + 1);
             if (wwarp == 0 && ok) {  // U0^T and [-W | Qd] S^T: needs only the bf16 copy
                 const uint32_t d1 = tbase + colb + d1_col;
                 const uint64_t so = kStageStep * stg;
@@ -386,13 +358,10 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
                 }
                 __syncwarp();  // reconverge warp 0 before the aligned TMEM loads below
             }
-            KDA_MARK(tid == 0 && c < 128, c * 16 + 2);
             if (c > 0) finish_chunk(c - 1);
-            KDA_MARK(tid == 0 && c < 128, c * 16 + 5);
             if (ok) ok = mbar_wait(mb1, c & 1);
             ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
-            KDA_MARK(tid == 0 && c < 128, c * 16 + 6);
             if (ok) {  // U^T row j -> bf16 A operand in shared memory
                 uint32_t u[16];
                 tmem_ld16_wait(t_d1 + 32 * (c & 1), u);
@@ -405,7 +374,6 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
             }
             fence_async_smem();
             tc_fence_before();
-            KDA_MARK(tid == 0 && c < 128, c * 16 + 7);
             bar_sync(bar_wg, 128);
             if (wwarp == 0 && ok) {  // S^T += U^T Kb (into the state itself);  O^T += U^T P^T
                 const uint64_t so = kStageStep * stg;
@@ -419,22 +387,18 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
             }
             const bool has_next = c + 1 < nchunks;
             if (OUT && c > 0) store_y(c - 1);
-            KDA_MARK(tid == 0 && c < 128, c * 16 + 8);
             if (has_next) bar_sync(BAR_FULL + (c + 1) % kStages, kBarCount);
-            KDA_MARK(tid == 0 && c < 128, c * 16 + 9);
             if (ok) ok = mbar_wait(mb2, c & 1);
             ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
             tc_fence_before();
             bar_arrive(BAR_EMPTY + stg, kBarCount);  // every reader of this stage is done
-            KDA_MARK(tid == 0 && c < 128, c * 16 + 10);
             if (ok) {
                 state_pass(has_next ? sm.st[(c + 1) % kStages].gam : nullptr, false,
                            EXT ? snap.at(snap.pos0 + 16 * (c + 1)) : nullptr);
             } else {
                 tc_fence_before();
             }
-            KDA_MARK(tid == 0 && c < 128, c * 16 + 11);
         }
         if (nchunks > 0) {
             if (OUT) cp_async_wait<0>();
@@ -486,9 +450,7 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
             const int stg = c % kStages;
             typename Lay::Raw &Wk = sm.raw[c % kRaw];
             typename Lay::Stage &St = sm.st[stg];
-            KDA_MARK(d == 0 && c < 128, 2048 + c * 8 + 0);
             if (c >= kStages) bar_sync(BAR_EMPTY + stg, kBarCount);  // the stage is free again
-            KDA_MARK(d == 0 && c < 128, 2048 + c * 8 + 1);
             issue_v(c);
             cp_async_commit();
             unsigned short bq2 = 0;
@@ -508,7 +470,6 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
             if (d < 16) pr.beta[stg][d] = beta_in(__bfloat162float(__ushort_as_bfloat16(bq0)), flags);
             __syncwarp();
             bar_sync(BAR_DPAIR, kPair);             // the tiles (with cleared rows) are visible
-            KDA_MARK(d == 0 && c < 128, 2048 + c * 8 + 2);
             if (L2N) {  // row norms of k and q: the two warps cover all channels
                 float sk[16], sq[16];
 #pragma unroll
@@ -590,7 +551,6 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
             *reinterpret_cast<uint4 *>(at_bytes(St.b2, kmaj(ip, 8, 16))) = make_uint4(kb0[4], kb0[5], kb0[6], kb0[7]);
             *reinterpret_cast<uint4 *>(at_bytes(St.b2, kmaj(ip + 1, 0, 16))) = make_uint4(kb1[0], kb1[1], kb1[2], kb1[3]);
             *reinterpret_cast<uint4 *>(at_bytes(St.b2, kmaj(ip + 1, 8, 16))) = make_uint4(kb1[4], kb1[5], kb1[6], kb1[7]);
-            KDA_MARK(d == 0 && c < 128, 2048 + c * 8 + 3);
             // v of chunk c has landed; the stage's and the tile's generic writes
             // become visible to the tensor core and ordered before a TMA refill
             cp_async_wait<0>();
@@ -632,9 +592,7 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
             typename Lay::Raw &Wk = sm.raw[c % kRaw];
             typename Lay::Stage &St = sm.st[stg];
             const float *bet = pr.beta[stg];
-            KDA_MARK(m == 0 && c < 128, 2048 + c * 8 + 4);
             bar_sync(BAR_DEC + c % kRaw, kDecCount);  // Kd, Ki, Qd, Kb^T, exp(G_C), v of chunk c
-            KDA_MARK(m == 0 && c < 128, 2048 + c * 8 + 5);
             const unsigned char *Kd = Wk.k, *Ki = Wk.g, *Qd = Wk.q;
 
             // A = Kd Ki^T (warp 6) and P = Qd Ki^T (warp 7) on warp-level MMA
@@ -674,7 +632,6 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
             }
             __syncwarp();
             bar_sync(BAR_MPAIR, kPair);             // AT and P are written
-            KDA_MARK(m == 0 && c < 128, 2048 + c * 8 + 6);
 
             // Tb = (I + Diag(beta) A)^-1 Diag(beta): lane j < 16 of warp 6 owns
             // column j, and after row r is final it is pushed into every later
@@ -713,7 +670,6 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
             }
             __syncwarp();
             bar_sync(BAR_MPAIR, kPair);             // Tb is written
-            KDA_MARK(m == 0 && c < 128, 2048 + c * 8 + 7);
 
             // W = Tb Kd -> rows 0-15 of the [-W | Qd] operand hold -W; warp mw
             // covers key channels [DK/2 mw, DK/2 (mw + 1))

@@ -128,7 +128,10 @@ def _round(x: torch.Tensor, dtype: str) -> torch.Tensor:
     return x.to(torch.bfloat16).to(torch.float32) if dtype == "bf16" else x
 
 
-def _draw(gen, L, dk, dv, g_mode, with_init, dtype, device="cpu"):
+def _draw(gen, L, dk, dv, g_mode, with_init, dtype, device="cpu", heads=1):
+    """Rows are [L // heads][heads] when heads > 1 (all heads of a packed
+    tensor at once); with g_mode "floor25" every head then gets its own fixed
+    subset of floor channels, as a per-head draw does."""
     def randn(*shape):
         return torch.randn(*shape, generator=gen, device=device, dtype=torch.float32)
 
@@ -144,8 +147,10 @@ def _draw(gen, L, dk, dv, g_mode, with_init, dtype, device="cpu"):
         g = torch.clamp_min(-torch.nn.functional.softplus(2.0 * randn(L, dk)), LN_FLOOR)
     gate = torch.sigmoid(randn(L, dv))
     if g_mode == "floor25":
-        perm = torch.randperm(dk, generator=gen, device=device)[: dk // 4]
-        g[:, perm] = LN_FLOOR
+        gh = g.view(L // heads, heads, dk)
+        for h in range(heads):
+            perm = torch.randperm(dk, generator=gen, device=device)[: dk // 4]
+            gh[:, h, perm] = LN_FLOOR
     s0 = 0.02 * randn(dk, dv) if with_init else None
     out = dict(q=_round(q, dtype), k=_round(k, dtype), v=_round(v, dtype),
                beta=_round(beta, dtype), g=_round(g, dtype), gate=_round(gate, dtype))
@@ -228,7 +233,7 @@ def fast_prefill(w: Workload, seed: int, device="cpu") -> dict:
     T, H, dk, dv, N = cu[-1], w.H, w.dk, w.dv, w.num_seqs
     gen = torch.Generator(device=device).manual_seed(seed)
     d = _draw(gen, T * H, dk, dv, "standard" if w.g_mode != "floor25" else "floor25",
-              False, w.dtype, device)
+              False, w.dtype, device, heads=H)
     dt = w.torch_dtype
     out = dict(q=d["q"].view(T, H, dk).to(dt), k=d["k"].view(T, H, dk).to(dt),
                v=d["v"].view(T, H, dv).to(dt), g=d["g"].view(T, H, dk).to(dt),
