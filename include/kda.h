@@ -151,21 +151,34 @@ int kda_build_checks_g(void);
  * buffers, hosts that forbid allocation after start-up).  The pages have no
  * counterpart to this; it is a deployment convenience.
  *
- * Same arguments, semantics and results as kda_chunk_fwd, minus workspace.
- * The scratch the prefill needs (piece plan, per-piece transitions and
- * states) lives in a fixed 32 MiB array of device memory owned by the
- * library: it exists on every GPU that loads this code and is held until the
- * process exits.  The piece length is the usual one, lengthened until the
- * scratch fits; sizes whose plan does not fit even with one piece per
- * sequence are rejected with KDA_ERR_WORKSPACE.  Allocates nothing (no
- * cudaMalloc/cudaFree, directly or through a library).
+ * Same arguments, semantics, argument checks and results as kda_chunk_fwd,
+ * minus workspace.  The scratch the prefill needs (piece plan, per-piece
+ * transitions and states) lives in a fixed 32 MiB array of device memory
+ * owned by the library: it exists on every GPU that loads this code and is
+ * held until the process exits.  The piece length is the usual one or, when
+ * that plan does not fit, the shortest one that does; sizes whose plan does
+ * not fit even with one piece per sequence are rejected with
+ * KDA_ERR_WORKSPACE.  A call allocates nothing (no cudaMalloc/cudaFree,
+ * directly or through a library).
  *
- * The first call on each device, made while that device is current, looks up
- * the array's device address (cudaGetSymbolAddress); make that first call
- * before any stream capture.  All calls on a device share the array and its
+ * The array is placed on a device when the library's device code is loaded
+ * there; under CUDA's lazy module loading (the default) that happens on the
+ * first call into the library on that device, and is the one device
+ * allocation this entry point implies.  Callers that may not allocate later
+ * make one call at start-up (kda_chunk_fwd_noalloc_check(NULL) is enough),
+ * and before any stream capture.  Each call looks the array's address up on
+ * the current device.  All calls on a device share the array and its
  * contents persist between calls: calls that overlap on the GPU (other
  * streams, other host threads) race on it and must be serialised by the
  * caller.  No entry needs to start at zero; each call writes what it reads.
+ *
+ * Device-side errors (inconsistent device offsets, a bounded wait that gave
+ * up, g out of range in the checked build) land in the array's first words,
+ * as in a kda_chunk_fwd workspace; kda_chunk_fwd_noalloc_check waits for
+ * `stream` and maps the words of the last call on the current device to a
+ * status exactly as kda_chunk_fwd_check does (KDA_OK, KDA_ERR_INVALID_ARG,
+ * KDA_ERR_TIMEOUT, or KDA_ERR_CUDA if the synchronisation or the 12-byte
+ * copy fails).  It allocates nothing.
  */
 int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const void *g,
                           const void *beta, const void *gate, void *out,
@@ -173,6 +186,7 @@ int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const voi
                           int32_t num_seqs, int32_t total_tokens, int32_t H, int32_t dk,
                           int32_t dv, kda_dtype dtype, float scale, int32_t qk_l2norm,
                           const float *initial_state, float *final_state, kda_stream_t stream);
+int kda_chunk_fwd_noalloc_check(kda_stream_t stream);
 
 /*
  * Decode: one token per sequence, the recurrence above applied once, state

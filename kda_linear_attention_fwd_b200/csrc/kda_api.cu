@@ -6,6 +6,7 @@
 #include <cstring>
 
 #include "../../include/kda.h"
+#include "kda_args.h"
 #include "kda_common.cuh"
 #include "kda_prefill.cuh"
 
@@ -67,8 +68,10 @@ int sm_count() {
     return cache[dev];
 }
 
-int choose_piece_len(long total_tokens, int num_seqs, int H, const int32_t *cu_host = nullptr) {
-    return kda::plan_piece_len(total_tokens, num_seqs, H, sm_count(), cu_host);
+int choose_piece_len(long total_tokens, int num_seqs, int H, bool c32,
+                     const int32_t *cu_host = nullptr) {
+    const kda::PlanModel pm = c32 ? kda::plan_model_chunk32(sm_count()) : kda::plan_model_chunk16(sm_count());
+    return kda::plan_piece_len(total_tokens, num_seqs, H, pm, cu_host);
 }
 
 long max_pieces(long total_tokens, int num_seqs, int piece_len) {
@@ -96,15 +99,17 @@ size_t kda_chunk_fwd_workspace_size(int32_t total_tokens, int32_t num_seqs, int3
                                     int32_t dv, kda_dtype dtype) {
     if (total_tokens < 0 || num_seqs < 0 || H < 1 || !dim_ok(dk) || !dim_ok(dv)) return 0;
     if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return 0;
-    const int L = choose_piece_len(total_tokens, num_seqs, H);
-    const long P = max_pieces(total_tokens, num_seqs, L);
+    // enough for either plan (the extended features run in 16-token chunks)
+    long P = max_pieces(total_tokens, num_seqs, choose_piece_len(total_tokens, num_seqs, H, false));
+    if (dtype == KDA_DTYPE_BF16 && dk == 128 && dv == 128)
+        P = std::max(P, max_pieces(total_tokens, num_seqs, choose_piece_len(total_tokens, num_seqs, H, true)));
     return kda::workspace_layout(P, num_seqs, H, dk, dv).total;
 }
 
 int kda_chunk_fwd_plan(int32_t total_tokens, int32_t num_seqs, int32_t H, int32_t *piece_len,
                        int32_t *max_pieces_out, int32_t *launches) {
     if (total_tokens < 0 || num_seqs < 0 || H < 1) return KDA_ERR_INVALID_ARG;
-    const int L = choose_piece_len(total_tokens, num_seqs, H);
+    const int L = choose_piece_len(total_tokens, num_seqs, H, true);
     const long P = max_pieces(total_tokens, num_seqs, L);
     if (piece_len) *piece_len = L;
     if (max_pieces_out) *max_pieces_out = (int32_t)(P > 0x7fffffffL ? 0x7fffffffL : P);
@@ -120,38 +125,23 @@ int kda_chunk_fwd_ex(const void *q, const void *k, const void *v, const void *g,
                      float *snapshots, const int32_t *snapshot_offsets, void *workspace,
                      size_t workspace_bytes, kda_stream_t stream_) {
     cudaStream_t stream = (cudaStream_t)stream_;
-    if (num_seqs < 0 || total_tokens < 0 || H < 1) return KDA_ERR_INVALID_ARG;
-    if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
-    if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_UNSUPPORTED;
+    int rc = kda::check_prefill_sizes(num_seqs, total_tokens, H, dk, dv, dtype);
+    if (rc != KDA_OK) return rc;
     if (flags & ~kda::FLAG_ALL) return KDA_ERR_INVALID_ARG;
     if (snapshot_tokens < 0 || snapshot_tokens % 16 != 0) return KDA_ERR_INVALID_ARG;
     if (snapshot_tokens > 0) {
         if (!snapshots || !snapshot_offsets) return KDA_ERR_INVALID_ARG;
         if (!aligned(snapshots, 16) || !aligned(snapshot_offsets, 4)) return KDA_ERR_ALIGNMENT;
     }
-    if (num_seqs == 0) return total_tokens == 0 ? KDA_OK : KDA_ERR_INVALID_ARG;
-    if (!cu_seqlens) return KDA_ERR_INVALID_ARG;
-    if (total_tokens > 0 && (!q || !k || !v || !g || !beta || !out)) return KDA_ERR_INVALID_ARG;
-    const size_t esz = dtype == KDA_DTYPE_BF16 ? 2 : 4;
-    const void *a16[] = {q, k, v, g, gate, out, initial_state, final_state, workspace};
-    for (const void *p : a16)
-        if (p && !aligned(p, 16)) return KDA_ERR_ALIGNMENT;
-    if (beta && !aligned(beta, esz)) return KDA_ERR_ALIGNMENT;
-    if (!aligned(cu_seqlens, 4)) return KDA_ERR_ALIGNMENT;
-    const size_t state_bytes = (size_t)num_seqs * H * dk * dv * sizeof(float);
-    if (initial_state && final_state && initial_state != final_state) {
-        const char *a = (const char *)initial_state, *b = (const char *)final_state;
-        if (a < b + state_bytes && b < a + state_bytes) return KDA_ERR_INVALID_ARG;
-    }
-    if (cu_seqlens_host) {
-        if (cu_seqlens_host[0] != 0 || cu_seqlens_host[num_seqs] != total_tokens)
-            return KDA_ERR_INVALID_ARG;
-        for (int n = 0; n < num_seqs; ++n)
-            if (cu_seqlens_host[n + 1] < cu_seqlens_host[n]) return KDA_ERR_INVALID_ARG;
-    }
+    bool empty = false;
+    rc = kda::check_prefill_buffers(q, k, v, g, beta, gate, out, cu_seqlens, cu_seqlens_host, num_seqs,
+                                    total_tokens, H, dk, dv, dtype, initial_state, final_state, workspace,
+                                    &empty);
+    if (rc != KDA_OK || empty) return rc;
     // the piece length with the real lengths, when known, is never shorter
     // than the length-blind one the workspace was sized for
-    const int L = choose_piece_len(total_tokens, num_seqs, H, cu_seqlens_host);
+    const bool c32 = kda::chunk32_eligible(dtype == KDA_DTYPE_BF16, dk, dv, flags, snapshot_tokens);
+    const int L = choose_piece_len(total_tokens, num_seqs, H, c32, cu_seqlens_host);
     const long P_max = max_pieces(total_tokens, num_seqs, L);
     if (P_max > (1L << 30) || (long)H * P_max > (1L << 31)) return KDA_ERR_UNSUPPORTED;
     const kda::WorkspaceLayout WL = kda::workspace_layout(P_max, num_seqs, H, dk, dv);
@@ -179,6 +169,7 @@ int kda_chunk_fwd_ex(const void *q, const void *k, const void *v, const void *g,
     p.snap_tokens = snapshot_tokens;
     p.snapshots = snapshot_tokens > 0 ? snapshots : nullptr;
     p.snap_offsets = snapshot_tokens > 0 ? snapshot_offsets : nullptr;
+    p.piece_len = L;
 
     const bool bf16 = dtype == KDA_DTYPE_BF16;
     cudaError_t e = kda::launch_plan(cu_seqlens, num_seqs, total_tokens, L, (int)P_max,
@@ -222,9 +213,7 @@ int kda_chunk_fwd_check(const void *workspace, size_t workspace_bytes, kda_strea
     int32_t h[3];
     if (cudaMemcpy(h, workspace, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess)
         return KDA_ERR_CUDA;
-    if (h[1] != 0 || (h[2] & 4)) return KDA_ERR_INVALID_ARG;  // offsets, or g out of range
-    if (h[2] & 3) return KDA_ERR_TIMEOUT;                       // a device wait gave up
-    return KDA_OK;
+    return kda::decode_plan_header(h);
 }
 
 int kda_build_checks_g(void) {

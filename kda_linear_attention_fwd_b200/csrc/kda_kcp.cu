@@ -162,7 +162,10 @@ int kda_chunk_fwd_summary(const void *k, const void *v, const void *g, const voi
         for (int n = 0; n < num_seqs; ++n)
             if (cu_seqlens_host[n + 1] < cu_seqlens_host[n]) return KDA_ERR_INVALID_ARG;
     }
-    const long L = plan_piece_len(total_tokens, num_seqs, H, sm_count(), cu_seqlens_host);
+    const PlanModel pm = chunk32_eligible(dtype == KDA_DTYPE_BF16, dk, dv, flags, 0)
+                             ? plan_model_chunk32(sm_count())
+                             : plan_model_chunk16(sm_count());
+    const long L = plan_piece_len(total_tokens, num_seqs, H, pm, cu_seqlens_host);
     const long P_max = (long)num_seqs + ((long)total_tokens + L - 1) / L;
     if (P_max > (1L << 30) || (long)H * P_max > (1L << 31)) return KDA_ERR_UNSUPPORTED;
     const WorkspaceLayout WL = workspace_layout(P_max, num_seqs, H, dk, dv);
@@ -187,6 +190,7 @@ int kda_chunk_fwd_summary(const void *k, const void *v, const void *g, const voi
     p.scale = 1.f;
     p.flags = flags;
     p.summarize_all = 1;
+    p.piece_len = (int)L;
 
     cudaError_t e = launch_plan(cu_seqlens, num_seqs, total_tokens, (int)L, (int)P_max,
                                 (int32_t *)(ws + WL.off_header), (int32_t *)(ws + WL.off_seq_first),

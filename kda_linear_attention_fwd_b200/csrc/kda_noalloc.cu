@@ -11,18 +11,23 @@
 // and outputs.
 //
 // The array (kScratchBytes) exists once per GPU that loads this code and is
-// held until the process exits.  Host code cannot use its name as a device
-// address, so the address is looked up with cudaGetSymbolAddress once per
-// device, on the first call made while that device is current; make that
-// first call before any stream capture.  Every call on a device uses the
-// same array: calls that overlap on the GPU (different streams, or another
-// host thread) race on it and must be serialised by the caller.  Nothing in
-// the array has to start at zero: each call writes every entry it later
-// reads.
+// held until the process exits.  It is placed when the library's device code
+// is loaded on a device; under CUDA's lazy module loading that is the first
+// call into this library there, so a caller that may not allocate later
+// makes one call (kda_chunk_fwd_noalloc_check is enough) at start-up, before
+// any stream capture.  Host code cannot use the array's name as a device
+// address: every call looks the address up with cudaGetSymbolAddress on the
+// current device (cheap once the code is loaded, and right again after the
+// context has been reset).  Every call on a device uses the same array: calls
+// that overlap on the GPU (different streams, or another host thread) race on
+// it and must be serialised by the caller.  Nothing in the array has to start
+// at zero: each call writes every entry it later reads.  The device-side
+// error words of the last call sit in the array's first bytes and are read
+// by kda_chunk_fwd_noalloc_check.
 #include <cstdlib>
-#include <mutex>
 
 #include "../../include/kda.h"
+#include "kda_args.h"
 #include "kda_common.cuh"
 #include "kda_prefill.cuh"
 
@@ -32,6 +37,10 @@ cudaError_t launch_plan(const int32_t *cu, int num_seqs, int total_tokens, int p
 cudaError_t launch_scan(const PrefillParams &p, int dk, int dv, cudaStream_t st);
 cudaError_t launch_prefill_chunks(const PrefillParams &p, bool bf16, int dk, int dv,
                                   bool summaries, cudaStream_t st);
+#ifdef KDA_CHECK_G
+cudaError_t launch_check_g(const void *g, bool bf16, long n, int clamp, int32_t *err,
+                           cudaStream_t st);
+#endif
 }  // namespace kda
 
 namespace {
@@ -40,33 +49,17 @@ constexpr size_t kScratchBytes = size_t(32) << 20;  // 32 MiB per device
 
 static __device__ __align__(256) unsigned char kda_noalloc_scratch[kScratchBytes];
 
-std::mutex g_mu;
-void *g_scratch_ptr[64] = {nullptr};
-
-// Device address of the scratch array on the current device (set-up on the
-// first call per device).
+// Device address of the scratch array on the current device.
 int scratch_address(void **out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, kda_noalloc_scratch);
+    if (e != cudaSuccess || !p) {
         cudaGetLastError();
         return KDA_ERR_CUDA;
     }
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_ptr[dev]) {
-        void *p = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&p, kda_noalloc_scratch);
-        if (e != cudaSuccess || !p) {
-            cudaGetLastError();
-            return KDA_ERR_CUDA;
-        }
-        g_scratch_ptr[dev] = p;
-    }
-    *out = g_scratch_ptr[dev];
+    *out = p;
     return KDA_OK;
 }
-
-bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
-bool dim_ok(int d) { return d == 64 || d == 128; }
 
 int sm_count() {
     int dev = 0, n = 0;
@@ -76,6 +69,14 @@ int sm_count() {
         n = 148;
     }
     return n;
+}
+
+// Scratch bytes the plan with piece length L needs: with a single piece per
+// sequence only the plan table is used.
+size_t scratch_need(long L, int num_seqs, int total_tokens, int H, int dk, int dv) {
+    const long P = (long)num_seqs + ((long)total_tokens + L - 1) / L;
+    const kda::WorkspaceLayout W = kda::workspace_layout(P, num_seqs, H, dk, dv);
+    return total_tokens > L ? W.total : W.off_M;
 }
 
 }  // namespace
@@ -88,45 +89,38 @@ extern "C" int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v
                                      int32_t qk_l2norm, const float *initial_state,
                                      float *final_state, kda_stream_t stream_) {
     cudaStream_t stream = (cudaStream_t)stream_;
-    if (num_seqs < 0 || total_tokens < 0 || H < 1) return KDA_ERR_INVALID_ARG;
-    if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
-    if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_UNSUPPORTED;
+    int rc = kda::check_prefill_sizes(num_seqs, total_tokens, H, dk, dv, dtype);
+    if (rc != KDA_OK) return rc;
     if (qk_l2norm != 0 && qk_l2norm != 1) return KDA_ERR_INVALID_ARG;
-    if (num_seqs == 0) return total_tokens == 0 ? KDA_OK : KDA_ERR_INVALID_ARG;
-    if (!cu_seqlens) return KDA_ERR_INVALID_ARG;
-    if (total_tokens > 0 && (!q || !k || !v || !g || !beta || !out)) return KDA_ERR_INVALID_ARG;
-    const size_t esz = dtype == KDA_DTYPE_BF16 ? 2 : 4;
-    const void *a16[] = {q, k, v, g, gate, out, initial_state, final_state};
-    for (const void *p : a16)
-        if (p && !aligned(p, 16)) return KDA_ERR_ALIGNMENT;
-    if (beta && !aligned(beta, esz)) return KDA_ERR_ALIGNMENT;
-    if (!aligned(cu_seqlens, 4)) return KDA_ERR_ALIGNMENT;
-    const size_t state_bytes = (size_t)num_seqs * H * dk * dv * sizeof(float);
-    if (initial_state && final_state && initial_state != final_state) {
-        const char *a = (const char *)initial_state, *b = (const char *)final_state;
-        if (a < b + state_bytes && b < a + state_bytes) return KDA_ERR_INVALID_ARG;
-    }
-    if (cu_seqlens_host) {
-        if (cu_seqlens_host[0] != 0 || cu_seqlens_host[num_seqs] != total_tokens)
-            return KDA_ERR_INVALID_ARG;
-        for (int n = 0; n < num_seqs; ++n)
-            if (cu_seqlens_host[n + 1] < cu_seqlens_host[n]) return KDA_ERR_INVALID_ARG;
-    }
+    bool empty = false;
+    rc = kda::check_prefill_buffers(q, k, v, g, beta, gate, out, cu_seqlens, cu_seqlens_host, num_seqs,
+                                    total_tokens, H, dk, dv, dtype, initial_state, final_state, nullptr,
+                                    &empty);
+    if (rc != KDA_OK || empty) return rc;
 
-    // Piece length: the usual plan, lengthened until the piece summaries fit in the
-    // fixed scratch array.  Once a piece spans the whole input no summaries
-    // are needed and only the plan table remains; if even that does not fit,
-    // the sizes are beyond what this entry point supports.
-    long L = kda::plan_piece_len(total_tokens, num_seqs, H, sm_count(), cu_seqlens_host);
-    const long L_all = ((long)total_tokens + 15) / 16 * 16 + 16;
-    for (;;) {
-        const long P = (long)num_seqs + ((long)total_tokens + L - 1) / L;
-        const kda::WorkspaceLayout W = kda::workspace_layout(P, num_seqs, H, dk, dv);
-        // with a single piece per sequence only the plan table is used
-        const size_t need = total_tokens > L ? W.total : W.off_M;
-        if (need <= kScratchBytes) break;
-        if (L >= L_all) return KDA_ERR_WORKSPACE;  // sizes beyond the fixed scratch
-        L = L * 2 < L_all ? L * 2 : L_all;
+    // Piece length: the usual plan or, when its piece summaries do not fit in
+    // the fixed scratch, the shortest multiple of the chunk length that fits
+    // (the need only falls as pieces get longer).  Once a piece spans the
+    // whole input no summaries are needed and only the plan table remains; if
+    // even that does not fit, the sizes are beyond what this entry point
+    // supports.
+    const bool bf16 = dtype == KDA_DTYPE_BF16;
+    const bool c32 = kda::chunk32_eligible(bf16, dk, dv, qk_l2norm, 0);
+    const kda::PlanModel pm = c32 ? kda::plan_model_chunk32(sm_count()) : kda::plan_model_chunk16(sm_count());
+    const long C = pm.chunk;
+    long L = kda::plan_piece_len(total_tokens, num_seqs, H, pm, cu_seqlens_host);
+    if (scratch_need(L, num_seqs, total_tokens, H, dk, dv) > kScratchBytes) {
+        long hi = ((long)total_tokens + C - 1) / C * C + C;  // one piece per sequence
+        if (scratch_need(hi, num_seqs, total_tokens, H, dk, dv) > kScratchBytes)
+            return KDA_ERR_WORKSPACE;  // sizes beyond the fixed scratch
+        long lo = L;                   // does not fit
+        while (hi - lo > C) {
+            long mid = (lo + hi) / 2 / C * C;
+            if (mid <= lo) mid = lo + C;
+            if (scratch_need(mid, num_seqs, total_tokens, H, dk, dv) <= kScratchBytes) hi = mid;
+            else lo = mid;
+        }
+        L = hi;
     }
     if (L > (1L << 30)) return KDA_ERR_UNSUPPORTED;
     const long P_max = (long)num_seqs + ((long)total_tokens + L - 1) / L;
@@ -135,7 +129,7 @@ extern "C" int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v
     const bool summaries = total_tokens > L;
 
     void *scratch = nullptr;
-    const int rc = scratch_address(&scratch);
+    rc = scratch_address(&scratch);
     if (rc != KDA_OK) return rc;
     char *ws = (char *)scratch;
 
@@ -160,13 +154,18 @@ extern "C" int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v
     p.snapshots = nullptr;
     p.snap_offsets = nullptr;
     p.total_tokens = total_tokens;
+    p.piece_len = (int)L;
 
-    const bool bf16 = dtype == KDA_DTYPE_BF16;
     cudaError_t e = kda::launch_plan(cu_seqlens, num_seqs, total_tokens, (int)L, (int)P_max,
                                      (int32_t *)(ws + WL.off_header),
                                      (int32_t *)(ws + WL.off_seq_first),
                                      (int4 *)(ws + WL.off_pieces), stream);
     if (e != cudaSuccess) return KDA_ERR_CUDA;
+#ifdef KDA_CHECK_G
+    // after the plan kernel, which clears the error word
+    e = kda::launch_check_g(g, bf16, (long)total_tokens * H * dk, 0, p.err, stream);
+    if (e != cudaSuccess) return KDA_ERR_CUDA;
+#endif
     if (summaries) {
         e = kda::launch_prefill_chunks(p, bf16, dk, dv, true, stream);
         if (e != cudaSuccess) return KDA_ERR_CUDA;
@@ -175,4 +174,18 @@ extern "C" int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v
     }
     e = kda::launch_prefill_chunks(p, bf16, dk, dv, false, stream);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+// Waits for `stream` and maps the error words of the last
+// kda_chunk_fwd_noalloc call on the current device to a status (the same
+// decoding as kda_chunk_fwd_check).  Copies 12 bytes from the scratch array to
+// the host; allocates nothing.
+extern "C" int kda_chunk_fwd_noalloc_check(kda_stream_t stream) {
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return KDA_ERR_CUDA;
+    int32_t h[3];
+    if (cudaMemcpyFromSymbol(h, kda_noalloc_scratch, sizeof(h), 0, cudaMemcpyDeviceToHost) != cudaSuccess) {
+        cudaGetLastError();
+        return KDA_ERR_CUDA;
+    }
+    return kda::decode_plan_header(h);
 }

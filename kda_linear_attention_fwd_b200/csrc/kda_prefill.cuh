@@ -60,22 +60,34 @@ inline WorkspaceLayout workspace_layout(long P_max, int num_seqs, int H, int dk,
 }
 
 // ---------------------------------------------------------------- the plan
-// Piece length (tokens, a multiple of 16).  Each (piece, head) is one CTA of
-// the output pass, which runs two CTAs per SM, so its time is counted in whole
-// waves of `slots` = 2 x SMs CTAs.  A sequence of p > 1 pieces costs an output
-// pass over all p pieces, a summary pass over pieces 0..p-2 (one CTA per
-// (piece, head) computes both the zero-start state and the transition, one CTA
-// per SM: waves of slots / 2) and p - 1 steps of the prefix scan.  With
-// equal-length sequences (the lengths are not known on the host in general)
-// the model is
-//   cost(L) = waves(output) * chunks(L) + 0.79 * waves(summary) * chunks(L)
-//             + 2 * (pieces - 1)
-// in units of one chunk step of the output pass; 0.79 is the measured ratio
-// of the two passes' per-chunk periods (about 3.0 K and 3.8 K SM cycles).
-// When the host copy of the offsets is given, the real lengths are used, and
-// only piece lengths at least as long as the length-blind choice are
-// considered, so that the workspace sized without the lengths still fits.
-inline double plan_cost(long L, int num_seqs, int H, int slots, const int32_t *cu_host,
+// Piece length (tokens, a multiple of the kernels' chunk).  Each (piece, head)
+// is one CTA of the output pass, so its time is counted in whole waves of
+// `slots_out` CTAs.  A sequence of p > 1 pieces costs an output pass over all
+// p pieces, a summary pass over pieces 0..p-2 (one CTA per (piece, head)
+// computes both the zero-start state and the transition; waves of
+// `slots_sum`) and p - 1 steps of the prefix scan.  With equal-length
+// sequences (the lengths are not known on the host in general) the model is
+//   cost(L) = waves(output) * chunks(L) + sum_ratio * waves(summary) * chunks(L)
+//             + scan_cost * (pieces - 1)
+// in units of one chunk step of the output pass.  When the host copy of the
+// offsets is given, the real lengths are used, and only piece lengths at
+// least as long as the length-blind choice are considered, so that the
+// workspace sized without the lengths still fits.
+struct PlanModel {
+    int chunk;          // tokens per chunk step (16 or 32); pieces are multiples of it
+    long slots_out;     // output-pass CTAs resident at once
+    long slots_sum;     // summary-pass CTAs resident at once
+    double sum_ratio;   // summary chunk step / output chunk step
+    double scan_cost;   // one scan step, in output chunk steps
+};
+// The 16-token kernels: output pass two CTAs per SM, the paired summary one;
+// 0.79 is the measured ratio of their per-chunk periods (about 3.0 K and
+// 3.8 K SM cycles), a scan step about two output chunk steps.
+inline PlanModel plan_model_chunk16(int sms) { return PlanModel{16, 2L * sms, (long)sms, 0.79, 2.0}; }
+// The 32-token kernels (bf16, dk = dv = 128): both passes one CTA per SM.
+inline PlanModel plan_model_chunk32(int sms) { return PlanModel{32, (long)sms, (long)sms, 1.0, 6.0}; }
+
+inline double plan_cost(long L, int num_seqs, int H, const PlanModel &pm, const int32_t *cu_host,
                         long total_tokens) {
     long out = 0, sum = 0, max_chunks = 0, max_pieces = 1;
     for (int n = 0; n < (cu_host ? num_seqs : 1); ++n) {
@@ -85,15 +97,15 @@ inline double plan_cost(long L, int num_seqs, int H, int slots, const int32_t *c
         const long mult = cu_host ? 1 : num_seqs;
         out += mult * pcs;
         sum += mult * (pcs - 1);
-        const long ch = (std::min(len, L) + 15) / 16;
+        const long ch = (std::min(len, L) + pm.chunk - 1) / pm.chunk;
         if (ch > max_chunks) max_chunks = ch;
         if (pcs > max_pieces) max_pieces = pcs;
     }
-    const long w_out = (out * H + slots - 1) / slots;
-    const long sum_slots = std::max(slots / 2, 1);
+    const long w_out = (out * H + pm.slots_out - 1) / pm.slots_out;
+    const long sum_slots = std::max(pm.slots_sum, 1L);
     const long w_sum = (sum * H + sum_slots - 1) / sum_slots;
-    return (double)w_out * max_chunks + 0.79 * (double)w_sum * max_chunks +
-           2.0 * (double)(max_pieces - 1);
+    return (double)w_out * max_chunks + pm.sum_ratio * (double)w_sum * max_chunks +
+           pm.scan_cost * (double)(max_pieces - 1);
 }
 
 inline long env_positive(const char *name) {
@@ -104,21 +116,22 @@ inline long env_positive(const char *name) {
     return (end && *end == 0 && v > 0) ? v : 0;
 }
 
-inline int plan_piece_len(long total_tokens, int num_seqs, int H, int sms,
+inline int plan_piece_len(long total_tokens, int num_seqs, int H, const PlanModel &pm_in,
                           const int32_t *cu_host) {
+    const long C = pm_in.chunk;
     const long forced = env_positive("KDA_PIECE_LEN");
-    if (forced > 0) return (int)(((forced + 15) / 16) * 16);
-    // the bf16 dk = dv = 128 chunk kernels run two CTAs per SM
-    const long slots = env_positive("KDA_SLOTS") ? env_positive("KDA_SLOTS") : 2L * sms;
+    if (forced > 0) return (int)(((forced + C - 1) / C) * C);
+    PlanModel pm = pm_in;
+    if (env_positive("KDA_SLOTS")) pm.slots_out = env_positive("KDA_SLOTS");
     if (num_seqs <= 0 || total_tokens <= 0) return 256;
     auto search = [&](const int32_t *cu, long Lref, long L_floor) {
-        long best_L = std::max<long>(((Lref + 15) / 16) * 16, 256);
+        long best_L = std::max<long>(((Lref + C - 1) / C) * C, 256);
         best_L = std::max(best_L, L_floor);
-        double best = plan_cost(best_L, num_seqs, H, (int)slots, cu, total_tokens);
+        double best = plan_cost(best_L, num_seqs, H, pm, cu, total_tokens);
         for (int pcs = 2; pcs <= 128; ++pcs) {
-            long L = ((Lref + pcs - 1) / pcs + 15) / 16 * 16;
+            long L = ((Lref + pcs - 1) / pcs + C - 1) / C * C;
             if (L < 256 || L < L_floor) break;
-            const double c = plan_cost(L, num_seqs, H, (int)slots, cu, total_tokens);
+            const double c = plan_cost(L, num_seqs, H, pm, cu, total_tokens);
             if (c < best) { best = c; best_L = L; }
         }
         return best_L;
@@ -156,7 +169,26 @@ struct PrefillParams {
     // summary pass over every piece (both parts), for the per-sequence affine
     // map of kda_chunk_fwd_summary; 0 = the prefill's own summary pass
     int summarize_all;
+    // piece length of the plan (tokens): the 32-token kernels need a multiple of 32
+    int piece_len;
 };
+
+// The 32-token kernels serve bf16 inputs with dk = dv = 128 and none of the
+// extended features (flags, snapshots); everything else runs in 16-token
+// chunks.  KDA_PREFILL_IMPL (c32 | tc5 | mma | simt) forces a path where it applies.
+inline int prefill_impl_forced() {
+    const char *e = getenv("KDA_PREFILL_IMPL");
+    if (!e || !*e) return 0;
+    if (e[0] == 'c') return 1;
+    if (e[0] == 't') return 2;
+    if (e[0] == 'm') return 3;
+    if (e[0] == 's') return 4;
+    return 0;
+}
+inline bool chunk32_eligible(bool bf16, int dk, int dv, int flags, int snap_tokens) {
+    const int f = prefill_impl_forced();
+    return bf16 && dk == 128 && dv == 128 && flags == 0 && snap_tokens == 0 && (f == 0 || f == 1);
+}
 
 // Where the output pass of one (piece, head) writes state snapshots.
 struct Snap {

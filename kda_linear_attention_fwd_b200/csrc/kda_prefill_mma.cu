@@ -586,22 +586,21 @@ cudaError_t launch_prefill_tc(const PrefillParams &p, int dk, int dv, bool summa
 }
 
 cudaError_t launch_prefill_tc5(const PrefillParams &p, bool summaries, cudaStream_t st);
+cudaError_t launch_prefill_c32(const PrefillParams &p, bool summaries, cudaStream_t st);
 
-// The chunk pass for one call.  bf16 inputs run on the tensor cores: the
-// tcgen05 kernel for dk = dv = 128, the warp-level MMA kernel for the other
+// The chunk pass for one call.  bf16 inputs run on the tensor cores: for
+// dk = dv = 128 the 32-token tcgen05 kernels (plain calls) or the 16-token
+// tcgen05 kernels (extended features), the warp-level MMA kernel for the other
 // head sizes.  fp32 inputs run the fp32 CUDA-core kernel (bf16 operands would
-// not reach fp32 accuracy).  KDA_PREFILL_IMPL=mma|simt forces a kernel.
+// not reach fp32 accuracy).  KDA_PREFILL_IMPL=c32|tc5|mma|simt forces a kernel
+// where it applies.
 cudaError_t launch_prefill_chunks(const PrefillParams &p, bool bf16, int dk, int dv,
                                   bool summaries, cudaStream_t st) {
-    static const int forced = [] {
-        const char *e = std::getenv("KDA_PREFILL_IMPL");
-        if (!e) return 0;
-        if (e[0] == 'm') return 1;
-        if (e[0] == 's') return 2;
-        return 0;
-    }();
-    if (!bf16 || forced == 2) return launch_prefill_simt(p, bf16, dk, dv, summaries, st);
-    if (forced == 0 && dk == 128 && dv == 128) return launch_prefill_tc5(p, summaries, st);
+    const int forced = prefill_impl_forced();
+    if (!bf16 || forced == 4) return launch_prefill_simt(p, bf16, dk, dv, summaries, st);
+    if (chunk32_eligible(bf16, dk, dv, p.flags, p.snap_tokens) && p.piece_len % 32 == 0)
+        return launch_prefill_c32(p, summaries, st);
+    if (forced != 3 && dk == 128 && dv == 128) return launch_prefill_tc5(p, summaries, st);
     return launch_prefill_tc(p, dk, dv, summaries, st);
 }
 

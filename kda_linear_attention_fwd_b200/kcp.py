@@ -61,9 +61,14 @@ def kcp_chunk_fwd(q, k, v, g, beta, gate, cu_seqlens, *, cu_seqlens_host=None,
     M, Z = backend.summary(k, v, g, beta, cu_seqlens, cu_seqlens_host, **flags)
     dk = M.shape[-1]
     packed = torch.cat([M, Z], dim=-1).contiguous()  # [N, H, dk, dk + dv]
-    gathered = [torch.empty_like(packed) for _ in range(world)]
-    dist.all_gather(gathered, packed, group=group)
+    # NCCL gathers the device tensors directly; a gloo group moves host copies
+    via_host = packed.is_cuda and dist.get_backend(group) == "gloo"
+    send = packed.cpu() if via_host else packed
+    gathered = [torch.empty_like(send) for _ in range(world)]
+    dist.all_gather(gathered, send, group=group)
     allp = torch.stack(gathered)                     # [R, N, H, dk, dk + dv]
+    if via_host:
+        allp = allp.to(packed.device)
     M_all, Z_all = allp[..., :dk].contiguous(), allp[..., dk:].contiguous()
     s_in = incoming_state(M_all, Z_all, rank, initial_state, backend)
     return backend.prefill(q, k, v, g, beta, gate, cu_seqlens, cu_seqlens_host, s_in, scale=scale,

@@ -23,7 +23,8 @@ KDA_DTYPE_BF16 = 1
 EXPORTS = ("kda_status_string", "kda_chunk_fwd_workspace_size", "kda_chunk_fwd_plan",
            "kda_chunk_fwd", "kda_decode_step", "kda_chunk_fwd_ex", "kda_decode_step_ex",
            "kda_chunk_fwd_summary", "kda_state_compose", "kda_bwd_workspace_size", "kda_bwd",
-           "kda_chunk_fwd_check", "kda_build_checks_g")
+           "kda_chunk_fwd_check", "kda_build_checks_g", "kda_chunk_fwd_noalloc",
+           "kda_chunk_fwd_noalloc_check")
 
 # flags of the extended entry points (include/kda.h)
 FLAG_QK_L2NORM, FLAG_BETA_LOGITS, FLAG_GATE_LOGITS, FLAG_CLAMP_DECAY = 1, 2, 4, 8
@@ -95,6 +96,11 @@ def _open(path):
     lib.kda_chunk_fwd_check.restype = ctypes.c_int
     lib.kda_build_checks_g.argtypes = []
     lib.kda_build_checks_g.restype = ctypes.c_int
+    lib.kda_chunk_fwd_noalloc.argtypes = [P, P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32,
+                                          ctypes.c_int, f32, i32, P, P, P]
+    lib.kda_chunk_fwd_noalloc.restype = ctypes.c_int
+    lib.kda_chunk_fwd_noalloc_check.argtypes = [P]
+    lib.kda_chunk_fwd_noalloc_check.restype = ctypes.c_int
     return lib
 
 

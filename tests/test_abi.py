@@ -250,12 +250,14 @@ def test_chunk_fwd_check_validation(lib):
 
 
 def test_plan_choices_on_148_sms(lib):
-    """The piece plan's cost model (waves of the output pass at two CTAs per SM,
-    of the paired summary pass at one, plus scan steps) on a 148-SM device;
-    without a device the library assumes 148 SMs."""
+    """The piece plan's cost model for the bf16 dk = dv = 128 plain call (the
+    32-token kernels: both passes one CTA per SM; waves of each pass plus scan
+    steps) on a 148-SM device; without a device the library assumes 148 SMs."""
     import torch
     if torch.cuda.is_available() and torch.cuda.get_device_properties(0).multi_processor_count != 148:
         pytest.skip("plan depends on the SM count")
-    assert kda.plan(131072, 1, 32)["piece_len"] == 3552   # 37 pieces per head
-    assert kda.plan(8192, 2, 16)["piece_len"] == 464      # 9 pieces per sequence
+    p = kda.plan(131072, 1, 32)
+    assert p["piece_len"] % 32 == 0
+    assert p["piece_len"] == 14592                        # 9 pieces per head: 288 CTAs, 2 waves
+    assert kda.plan(8192, 2, 16)["piece_len"] == 1024     # 4 pieces per sequence
     assert kda.plan(256, 1, 2) == {"piece_len": 256, "max_pieces": 2, "launches": 2}  # one piece

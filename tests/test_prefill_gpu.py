@@ -123,12 +123,31 @@ def test_final_state_may_alias_initial_state(cuda_lib, monkeypatch, piece):
 
 
 def test_without_host_offsets(cuda_lib, monkeypatch):
+    """The same forced plan with and without the host copy of the offsets:
+    identical results, both matching the oracle."""
     monkeypatch.setenv("KDA_PIECE_LEN", "256")
     w = W.custom(dtype="bf16", H=2, dk=64, dv=64, lengths=(600, 17), init_state=True, seed=11)
     inp = W.pack_prefill(w, device="cuda")
     y1, S1 = run(inp, host_cu=True)
     y2, S2 = run(inp, host_cu=False)
     assert np.array_equal(y1, y2) and np.array_equal(S1, S2)
+    yr, Sr = oracle_prefill(inp)
+    compare(inp, y2, S2, yr, Sr, "bf16", what="no host offsets")
+
+
+def test_length_blind_plan_bf16_128_matches_oracle(cuda_lib):
+    """bf16 dk = dv = 128 without the host copy of the offsets: the plan only
+    knows the average length, so the longer sequences of the varlen workload
+    are split into two pieces (summary, scan, output); one sampled head of
+    every sequence against the oracle."""
+    w = W.get("varlen_bf16")
+    plan = kda.plan(w.total_tokens, w.num_seqs, w.H)
+    assert max(w.lengths) > plan["piece_len"], plan  # some sequence has several pieces
+    heads = [(n, 3 + 4 * n) for n in range(w.num_seqs)]
+    inp = W.pack_prefill(w, heads=heads, device="cuda")
+    y, S = run(inp, host_cu=False)
+    yr, Sr = oracle_prefill(inp, heads=heads)
+    compare(inp, y, S, yr, Sr, "bf16", heads=heads, what="length-blind plan")
 
 
 def test_beta_zero_closed_form(cuda_lib):
