@@ -109,7 +109,7 @@ size_t kda_chunk_fwd_workspace_size(int32_t total_tokens, int32_t num_seqs, int3
 int kda_chunk_fwd_plan(int32_t total_tokens, int32_t num_seqs, int32_t H, int32_t *piece_len,
                        int32_t *max_pieces_out, int32_t *launches) {
     if (total_tokens < 0 || num_seqs < 0 || H < 1) return KDA_ERR_INVALID_ARG;
-    const int L = choose_piece_len(total_tokens, num_seqs, H, true);
+    const int L = choose_piece_len(total_tokens, num_seqs, H, kda::prefill_impl_forced() == 1);
     const long P = max_pieces(total_tokens, num_seqs, L);
     if (piece_len) *piece_len = L;
     if (max_pieces_out) *max_pieces_out = (int32_t)(P > 0x7fffffffL ? 0x7fffffffL : P);

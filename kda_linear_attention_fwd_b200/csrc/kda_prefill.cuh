@@ -173,9 +173,11 @@ struct PrefillParams {
     int piece_len;
 };
 
-// The 32-token kernels serve bf16 inputs with dk = dv = 128 and none of the
-// extended features (flags, snapshots); everything else runs in 16-token
-// chunks.  KDA_PREFILL_IMPL (c32 | tc5 | mma | simt) forces a path where it applies.
+// The 32-token kernels (bf16, dk = dv = 128, none of the extended features)
+// run when KDA_PREFILL_IMPL=c32 asks for them; by default every call runs in
+// 16-token chunks, which measured faster on B200 (two CTAs per SM against
+// one).  KDA_PREFILL_IMPL (c32 | tc5 | mma | simt) forces a path where it
+// applies.
 inline int prefill_impl_forced() {
     const char *e = getenv("KDA_PREFILL_IMPL");
     if (!e || !*e) return 0;
@@ -187,7 +189,7 @@ inline int prefill_impl_forced() {
 }
 inline bool chunk32_eligible(bool bf16, int dk, int dv, int flags, int snap_tokens) {
     const int f = prefill_impl_forced();
-    return bf16 && dk == 128 && dv == 128 && flags == 0 && snap_tokens == 0 && (f == 0 || f == 1);
+    return bf16 && dk == 128 && dv == 128 && flags == 0 && snap_tokens == 0 && f == 1;
 }
 
 // Where the output pass of one (piece, head) writes state snapshots.

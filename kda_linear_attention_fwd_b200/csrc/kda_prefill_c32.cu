@@ -51,7 +51,10 @@
 //              beta A for the solve), the 32 x 32 unit-lower solve (one warp,
 //              one column per lane, fp32), MMA W and its read-out (-W into
 //              its operand), TMA refills of q, k, g
-// Stages: two prepared chunks in flight; the q, k, g tiles of two chunks.
+// Hand-offs: decay -> matrix (named barrier DEC, per tile buffer), decay ->
+// state (mbarrier mb_gam: the chunk's gamma, all the next state pass needs),
+// matrix -> state (FULL: every operand of the chunk), state -> decay (EMPTY:
+// the update MMAs that read a stage have completed, so it may be refilled).
 // Every wait on an mbarrier is bounded (2 s); a wait that gives up sets an
 // error bit in the workspace header and the CTA drains through its barriers
 // without further tensor work.
@@ -78,13 +81,25 @@ constexpr int kHalf = 14336;
 constexpr int OFF_Q = 0, OFF_K = 4096, OFF_G = 8192, OFF_KB = 12288;
 constexpr int kRawBytes = 2 * kHalf;
 
-// named barriers (0 is __syncthreads)
-constexpr int BAR_FULL = 1;    // 1, 2: matrix team arrives (128), state team waits (256)
-constexpr int BAR_EMPTY = 3;   // 3, 4: state team arrives (256), decay team waits (128)
-constexpr int BAR_DEC = 5;     // 5, 6: decay team arrives (128), matrix team waits (128)
-constexpr int BAR_STATE = 7;   // state team (output pass: 256); summary: 7 and 8 per chain
-constexpr int BAR_DECAY = 9;   // decay team only
-constexpr int BAR_MAT = 10;    // matrix team only
+// Pipeline depths: NS prepared stages (chunk c -> stage c % NS) and NR chunks
+// of q, k, g tiles (chunk c -> raw[c % NR]).  The output pass keeps three
+// stages so that the preparation runs further ahead of the state chain; the
+// summary pass, whose stage data is smaller but which keeps a second state
+// copy in shared memory, keeps two stages and three tile buffers.
+template <bool OUT> struct Pipe {
+    static constexpr int NS = OUT ? 3 : 2;
+    static constexpr int NR = OUT ? 2 : 3;
+    // named barriers (0 is __syncthreads)
+    static constexpr int FULL = 1;             // NS: matrix team arrives (128), state team waits (256)
+    static constexpr int EMPTY = FULL + NS;    // NS: state team arrives (256), decay team waits (128)
+    static constexpr int DEC = EMPTY + NS;     // NR: decay team arrives (128), matrix team waits (128)
+    static constexpr int STATE = DEC + NR;     // 3: output pass: the state team (256), its U half
+                                               //    (warps 0-3) and its O half (warps 4-7); summary:
+                                               //    one per chain (128)
+    static constexpr int DECAY = STATE + 3;    // decay team only
+    static constexpr int MAT = DECAY + 1;      // matrix team only
+    static_assert(MAT <= 15, "named barrier ids");
+};
 constexpr int kFullCount = 384, kEmptyCount = 384, kDecCount = 256;
 
 // Byte offset of element (row r, channel ch) in a chunk of raw tiles, tile at
@@ -105,36 +120,48 @@ struct alignas(1024) Stage {
 
 template <bool OUT>
 struct Smem {
-    alignas(1024) unsigned char raw[2][kRawBytes];
-    Stage st[2];
+    alignas(1024) unsigned char raw[Pipe<OUT>::NR][kRawBytes];
+    Stage st[Pipe<OUT>::NS];
     alignas(16) unsigned char au[OUT ? 1 : 2][8192];         // U^T as A of MMA 3/4: K-major [128][32]
     alignas(16) unsigned char mbf[OUT ? 16 : 32768];         // summary: bf16 transition, K-major [128][128]
     alignas(128) unsigned char io[OUT ? 2 : 1][OUT ? 8192 : 16];  // gate tile in, y tile out ([32][128] bf16)
     alignas(16) float AT[kC * kC];                           // AT[s][r] = beta_r A[r][s]
+    alignas(16) float Td[2][16 * 16];                        // fp32 diagonal blocks of T
+    alignas(16) float Zx[16 * 16];                           // N10 T00
     alignas(16) float gexch[2][kD];                          // gamma of each tile (decay team)
-    alignas(16) float gam0[2][kD];                           // gamma_0 per chunk (W read-out)
-    alignas(8) unsigned long long mb_raw[2], mb_v[2], mb_io[2], mb_ap, mb_w, mb1[2], mb2[2];
+    alignas(16) float gam0[Pipe<OUT>::NS][kD];               // gamma_0 per chunk (W read-out)
+    // mb_gam[s]: the 128 decay threads arrive once gamma of the stage's chunk is
+    // written (all the state pass needs); the state team waits on it
+    alignas(8) unsigned long long mb_raw[Pipe<OUT>::NR], mb_ap[Pipe<OUT>::NS], mb_gam[Pipe<OUT>::NS], mb_w,
+        mb1[2], mb2[2];
     uint32_t tmem_base;
 };
 template <bool OUT> constexpr size_t kSmemBytes = sizeof(Smem<OUT>) + 1024;
+static_assert(kSmemBytes<true> <= 232448 && kSmemBytes<false> <= 232448, "shared memory per CTA");
+constexpr int kPrefetch = 6;   // chunks ahead whose tiles are pulled into L2
 
 // TMEM columns (512 allocated)
 template <bool OUT> struct Cols;
+// AP: one 64-column buffer per stage (chunk c -> c % NS); the W product of
+// a chunk reuses its AP buffer once the Gram blocks have been read out.
 template <> struct Cols<true> {
-    static constexpr uint32_t S = 0, BF = 128, D1 = 192, AP = 320, W = 384;  // D1: 2 x 64
+    static constexpr uint32_t S = 0, BF = 128, D1 = 192, AP = 320;  // D1: 2 x 64, AP: 3 x 64
 };
 template <> struct Cols<false> {
     // chain 0 (zero start): S, its bf16 copy, D1; chain 1 (transition): S2, D1b
     // (its bf16 copy lives in shared memory)
-    static constexpr uint32_t S = 0, BF = 128, D1 = 192, D1b = 224, S2 = 256, AP = 384, W = 448;
+    static constexpr uint32_t S = 0, BF = 128, D1 = 192, D1b = 224, S2 = 256, AP = 384;
 };
 
-// TMA descriptors: q, k, g, v as [T][H][128] bf16 (3-D: channel, head,
-// token), box 64 x 1 x 32 with the 128-byte swizzle; gate and out, box
-// 128 x 1 x 32 without swizzle.
+// TMA descriptors of q, k, g as [T][H][128] bf16 (3-D: channel, head,
+// token), box 64 x 1 x 32 with the 128-byte swizzle.  v and the gate arrive
+// by cp.async and y leaves by plain stores: the SM's TMA unit serves the
+// three tiles of every chunk and their L2 prefetches only.
 struct Maps {
-    CUtensorMap q, k, g, v, gate, out;
+    CUtensorMap q, k, g;
 };
+
+KDA_DEVICE void prefetch_l2(const void *p) { asm volatile("prefetch.L2 [%0];" ::"l"(p)); }
 
 KDA_DEVICE bool all_ok(bool ok) { return __all_sync(0xffffffffu, ok); }
 
@@ -147,6 +174,7 @@ template <bool OUT>
 __device__ void run_piece(const PrefillParams &p, const Maps &maps, int t0, int len, int h,
                           const float *s_init, float *s_out, float *m_out, unsigned char *smem_raw) {
     using L = Cols<OUT>;
+    using PP = Pipe<OUT>;
     Smem<OUT> &sm = *reinterpret_cast<Smem<OUT> *>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int H = p.H;
@@ -160,14 +188,15 @@ __device__ void run_piece(const PrefillParams &p, const Maps &maps, int t0, int 
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     if (tid == 32) {
+        for (int i = 0; i < Pipe<OUT>::NR; ++i) mbar_init(smem_u32(&sm.mb_raw[i]), 1);
+        for (int i = 0; i < Pipe<OUT>::NS; ++i) {
+            mbar_init(smem_u32(&sm.mb_ap[i]), 1);
+            mbar_init(smem_u32(&sm.mb_gam[i]), 128);
+        }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(smem_u32(&sm.mb_raw[i]), 1);
-            mbar_init(smem_u32(&sm.mb_v[i]), 1);
-            mbar_init(smem_u32(&sm.mb_io[i]), 1);
             mbar_init(smem_u32(&sm.mb1[i]), 1);
             mbar_init(smem_u32(&sm.mb2[i]), 1);
         }
-        mbar_init(smem_u32(&sm.mb_ap), 1);
         mbar_init(smem_u32(&sm.mb_w), 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -185,7 +214,7 @@ __device__ void run_piece(const PrefillParams &p, const Maps &maps, int t0, int 
         const int chain = OUT ? 0 : hf;
         const bool use_v = chain == 0;
         const bool active = OUT ? true : (chain == 0 ? s_out != nullptr : m_out != nullptr);
-        const int bar_team = OUT ? BAR_STATE : BAR_STATE + chain;
+        const int bar_team = OUT ? PP::STATE : PP::STATE + chain;
         const int team_n = OUT ? 256 : 128;
         // columns of S^T this thread keeps: output 64 (one half), summary all 128
         constexpr int NCOL = OUT ? 64 : 128;
@@ -279,113 +308,82 @@ __device__ void run_piece(const PrefillParams &p, const Maps &maps, int t0, int 
             tc_fence_before();
         };
 
-        // y = gate (.) O of chunk c: this thread's column j, rows 16 hf ..
-        // 16 hf + 15, in place in the gate tile; then the tile to global
+        // Output pass: warps 4-7 (the O half) produce y of the previous chunk
+        // while warps 0-3 (the U half) turn this chunk's U into the operand of
+        // MMA 3/4, so the epilogue stays off the state chain.
+        // Gate tile of chunk c -> io[c & 1] by cp.async: O-half thread j moves
+        // the 16-byte pieces j + 128 i (row x / 16, piece x % 16), the same
+        // pieces it stores as y, so a buffer is refilled right after its y left
+        // without a barrier.  One commit group per chunk (empty when there is
+        // nothing to load), so that wait_group 1 leaves exactly the newest one
+        // in flight.
+        auto issue_gate = [&](int c) {
+            if (gate && c < nchunks) {
+                const int rows = min(kC, len - kC * c);
+                unsigned char *tile = sm.io[c & 1];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int x = j + 128 * i, r = x >> 4, cc = x & 15;
+                    const bool okr = r < rows;
+                    cp_async16(tile + r * 256 + cc * 16,
+                               gate + ((size_t)(t0 + kC * c + (okr ? r : 0)) * H + h) * kD + cc * 8, okr);
+                }
+            }
+            cp_async_commit();
+        };
+        // L2 prefetch of the gate rows of chunk c (one 128-byte line per thread)
+        auto prefetch_gate = [&](int c) {
+            if (gate && c < nchunks && j < 64) {
+                const int r = j >> 1;
+                if (kC * c + r < len) prefetch_l2(gate + ((size_t)(t0 + kC * c + r) * H + h) * kD + (j & 1) * 64);
+            }
+        };
+        // y = gate (.) O of chunk c (O half): column j, all 32 rows, in place in
+        // the gate tile; then the tile's rows to global and the buffer refilled
+        // with the gate of chunk c + 2
         auto epilogue = [&](int c) {
-            if (!OUT) return;
             const int rows = min(kC, len - kC * c);
             unsigned char *tile = sm.io[c & 1];
-            bool iok = true;
-            if (gate) iok = mbar_wait(smem_u32(&sm.mb_io[c & 1]), (c >> 1) & 1);
-            ok = all_ok(ok && iok);
+            cp_async_wait<1>();  // the gate of chunk c (chunk c + 1's may still be in flight)
+            bar_sync(PP::STATE + 2, 128);
             if (ok) {
-                uint32_t o[16];
-                tmem_ld16(tbase + lane_off + d1_addr(c) + 32 + 16 * hf, o);
+                uint32_t o[32];
+                tmem_ld32(tbase + lane_off + d1_addr(c) + 32, o);
                 tc_wait_ld();
                 bf16 *tl = reinterpret_cast<bf16 *>(tile);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int t = 16 * hf + e;
+                for (int t = 0; t < kC; ++t) {
                     const float gv = gate ? __bfloat162float(tl[t * kD + j]) : 1.f;
-                    tl[t * kD + j] = __float2bfloat16_rn(gv * __uint_as_float(o[e]));
+                    tl[t * kD + j] = __float2bfloat16_rn(gv * __uint_as_float(o[t]));
                 }
             }
-            fence_async_smem();
             tc_fence_before();
-            bar_sync(bar_team, team_n);
-            if (!ok) return;
-            if (rows == kC) {
-                if (tid == 0) {
-                    tma_store_3d(&maps.out, smem_u32(tile), 0, h, t0 + kC * c);
-                    bulk_commit();
-                }
-            } else {
-                for (int x = tid; x < rows * 16; x += 256) {
-                    const int r = x >> 4, cc = x & 15;
-                    *reinterpret_cast<uint4 *>(out + ((size_t)(t0 + kC * c + r) * H + h) * kD + cc * 8) =
-                        *reinterpret_cast<const uint4 *>(tile + r * 256 + cc * 16);
-                }
-            }
-        };
-        auto issue_gate = [&](int c) {  // gate tile of chunk c -> io[c & 1] (thread 0)
-            if (OUT && gate && c < nchunks) {
-                const uint32_t mb = smem_u32(&sm.mb_io[c & 1]);
-                mbar_arrive_expect_tx(mb, 8192);
-                tma_load_3d(smem_u32(sm.io[c & 1]), &maps.gate, 0, h, t0 + kC * c, mb);
-            }
-        };
-
-        if (OUT && tid == 0) issue_gate(0);
-        if (nchunks == 0) {
-            if (fin) {
-                for (int i = c0; i < c0 + NCOL; ++i)
-                    fin[(size_t)i * kD + j] = chain == 1 ? (i == j ? 1.f : 0.f) : (init ? init[(size_t)i * kD + j] : 0.f);
-            }
-        } else {
-            bar_sync(BAR_FULL + 0, kFullCount);
-            if (active) state_pass(true, sm.st[0].gam);
-            tc_fence_before();
-            bar_sync(bar_team, team_n);
-        }
-
-        for (int c = 0; c < nchunks; ++c) {
-            const int stg = c & 1;
-            const uint64_t so = (uint64_t)kStageStep * stg;
-            const uint32_t d1 = tbase + d1_addr(c);
-            // ---- MMA 1 and 2: U^T and (Q~ S)^T, from the bf16 copy of S^T
-            if (issue_team && ok) {
-                if (elect_one_sync()) {
-                    bool vok = true;
-                    if (use_v) vok = mbar_wait(smem_u32(&sm.mb_v[stg]), (c >> 1) & 1);
-                    tc_fence_after();
-                    if (vok) {
-                        if (use_v) {
+            bar_sync(PP::STATE + 2, 128);
+            if (ok) {
 #pragma unroll
-                            for (int kk = 0; kk < 2; ++kk)  // 16 tokens = 2048 bytes of the V tile
-                                tc_mma_ss(d1, dsc_v + so + 128 * kk, dsc_b0 + so + 16 * kk, ID_1, kk > 0 ? 1u : 0u);
-                        }
-#pragma unroll
-                        for (int kk = 0; kk < 8; ++kk) {  // 16 channels = 256 bytes of [-W | Q~]
-                            if (chain == 0)
-                                tc_mma_ts(d1, tbase + L::BF + 8 * kk, dsc_b1 + so + 16 * kk, ID_2,
-                                          (use_v || kk > 0) ? 1u : 0u);
-                            else
-                                tc_mma_ss(d1, dsc_mbf + 16 * kk, dsc_b1 + so + 16 * kk, ID_2, kk > 0 ? 1u : 0u);
-                        }
-                        tc_commit(mb1);
-                    }
+                for (int i = 0; i < 4; ++i) {
+                    const int x = j + 128 * i, r = x >> 4, cc = x & 15;
+                    if (r < rows)
+                        *reinterpret_cast<uint4 *>(out + ((size_t)(t0 + kC * c + r) * H + h) * kD + cc * 8) =
+                            *reinterpret_cast<const uint4 *>(tile + r * 256 + cc * 16);
                 }
-                __syncwarp();
             }
-            // ---- the previous chunk's output, while MMA 1/2 run
-            if (c > 0) epilogue(c - 1);
-            // ---- U^T -> bf16 A operand of MMA 3/4
+            issue_gate(c + 2);
+            prefetch_gate(c + 6);
+        };
+        // U^T of chunk c (tokens u0 .. u0 + 31 of this thread's column) -> bf16
+        // A operand of MMA 3/4
+        auto u_readout = [&](int c) {
             if (ok) ok = mbar_wait(mb1, c & 1);
             ok = all_ok(ok);
             tc_fence_after();
             if (ok) {
-                constexpr int NU = OUT ? 16 : 32;        // tokens of U this thread converts
-                const int u0 = OUT ? 16 * hf : 0;
                 uint32_t u[32];
-                if (NU == 16) {
-                    tmem_ld16(tbase + lane_off + d1_addr(c) + u0, *reinterpret_cast<uint32_t(*)[16]>(&u[0]));
-                } else {
-                    tmem_ld32(tbase + lane_off + d1_addr(c), u);
-                }
+                tmem_ld32(tbase + lane_off + d1_addr(c), u);
                 tc_wait_ld();
 #pragma unroll
-                for (int q8 = 0; q8 < NU / 8; ++q8)
-                    *reinterpret_cast<uint4 *>(au + kmaj(j, u0 + 8 * q8, kC)) =
+                for (int q8 = 0; q8 < 4; ++q8)
+                    *reinterpret_cast<uint4 *>(au + kmaj(j, 8 * q8, kC)) =
                         make_uint4(pack_bf16(__uint_as_float(u[8 * q8 + 0]), __uint_as_float(u[8 * q8 + 1])),
                                    pack_bf16(__uint_as_float(u[8 * q8 + 2]), __uint_as_float(u[8 * q8 + 3])),
                                    pack_bf16(__uint_as_float(u[8 * q8 + 4]), __uint_as_float(u[8 * q8 + 5])),
@@ -393,9 +391,64 @@ __device__ void run_piece(const PrefillParams &p, const Maps &maps, int t0, int 
             }
             fence_async_smem();
             tc_fence_before();
+        };
+        auto wait_gamma = [&](int c) {  // gamma of chunk c is in its stage
+            if (ok) ok = mbar_wait(smem_u32(&sm.mb_gam[c % PP::NS]), (c / PP::NS) & 1);
+            ok = all_ok(ok);
+        };
+
+        if (OUT && hf == 1) {
+            issue_gate(0);
+            issue_gate(1);
+            for (int c = 0; c < 6; ++c) prefetch_gate(c);
+        }
+        if (nchunks == 0) {
+            if (fin) {
+                for (int i = c0; i < c0 + NCOL; ++i)
+                    fin[(size_t)i * kD + j] = chain == 1 ? (i == j ? 1.f : 0.f) : (init ? init[(size_t)i * kD + j] : 0.f);
+            }
+        } else {
+            wait_gamma(0);
+            if (active && ok) state_pass(true, sm.st[0].gam);
+            tc_fence_before();
             bar_sync(bar_team, team_n);
-            // ---- MMA 3 (state update) and 4 (P U into O)
+        }
+
+        for (int c = 0; c < nchunks; ++c) {
+            const int stg = c % PP::NS;
+            const uint64_t so = (uint64_t)kStageStep * stg;
+            const uint32_t d1 = tbase + d1_addr(c);
+            bar_sync(PP::FULL + stg, kFullCount);  // every operand of chunk c is in its stage
+            // ---- MMA 1 and 2: U^T and (Q~ S)^T, from the bf16 copy of S^T
             if (issue_team && ok) {
+                if (elect_one_sync()) {
+                    tc_fence_after();
+                    if (use_v) {
+#pragma unroll
+                        for (int kk = 0; kk < 2; ++kk)  // 16 tokens = 2048 bytes of the V tile
+                            tc_mma_ss(d1, dsc_v + so + 128 * kk, dsc_b0 + so + 16 * kk, ID_1, kk > 0 ? 1u : 0u);
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {  // 16 channels = 256 bytes of [-W | Q~]
+                        if (chain == 0)
+                            tc_mma_ts(d1, tbase + L::BF + 8 * kk, dsc_b1 + so + 16 * kk, ID_2,
+                                      (use_v || kk > 0) ? 1u : 0u);
+                        else
+                            tc_mma_ss(d1, dsc_mbf + 16 * kk, dsc_b1 + so + 16 * kk, ID_2, kk > 0 ? 1u : 0u);
+                    }
+                    tc_commit(mb1);
+                }
+                __syncwarp();
+            }
+            const bool issue34 = OUT ? (hf == 0) : true;  // threads that feed MMA 3/4
+            if (OUT && hf == 1) {
+                if (c > 0) epilogue(c - 1);  // the previous chunk's output, while MMA 1/2 run
+            } else {
+                u_readout(c);
+                bar_sync(OUT ? PP::STATE + 1 : bar_team, 128);  // the U half (output) or the chain
+            }
+            // ---- MMA 3 (state update) and 4 (P U into O)
+            if (issue34 && issue_team && ok) {
                 if (elect_one_sync()) {
                     tc_fence_after();
 #pragma unroll
@@ -411,29 +464,27 @@ __device__ void run_piece(const PrefillParams &p, const Maps &maps, int t0, int 
                 __syncwarp();
             }
             const bool has_next = c + 1 < nchunks;
-            // ---- the gate tile of the next chunk, once the y store of this
-            // buffer has been read out
-            if (OUT && tid == 0 && has_next) {
-                bulk_wait_read0();
-                issue_gate(c + 1);
-            }
-            if (has_next) bar_sync(BAR_FULL + ((c + 1) & 1), kFullCount);
             if (ok) ok = mbar_wait(mb2, c & 1);
             ok = all_ok(ok);
             tc_fence_after();
             tc_fence_before();
-            bar_arrive(BAR_EMPTY + stg, kEmptyCount);  // the stage's readers are done
-            if (ok) state_pass(false, has_next ? sm.st[(c + 1) & 1].gam : nullptr);
+            bar_arrive(PP::EMPTY + stg, kEmptyCount);  // the stage's readers are done
+            if (has_next) wait_gamma(c + 1);
+            if (ok) state_pass(false, has_next ? sm.st[(c + 1) % PP::NS].gam : nullptr);
             tc_fence_before();
             bar_sync(bar_team, team_n);
         }
-        if (OUT && nchunks > 0) epilogue(nchunks - 1);
-        if (OUT && tid == 0) bulk_wait0();
+        if (OUT && hf == 1 && nchunks > 0) epilogue(nchunks - 1);
+        cp_async_wait<0>();
         if (active && !ok && lane == 0 && p.err) atomicOr(p.err, 1);
     } else if (warp < 12) {
         // =========================================================== decay team
         const int d = tid - 256, sc = d >> 6, ip = 2 * (d & 63);
         const bf16 *beta = (const bf16 *)p.beta;
+        const bf16 *vv = (const bf16 *)p.v;
+        for (int cp = 0; cp < 6 && cp < nchunks; ++cp)  // the first chunks' v rows into L2
+            if (d < 64 && kC * cp + (d >> 1) < len)
+                prefetch_l2(vv + ((size_t)(t0 + kC * cp + (d >> 1)) * H + h) * kD + (d & 1) * 64);
         bool tok = true;
         auto load_beta = [&](int c) -> unsigned short {
             const int rows = min(kC, len - kC * c);
@@ -443,21 +494,30 @@ __device__ void run_piece(const PrefillParams &p, const Maps &maps, int t0, int 
         };
         unsigned short bq = d < kC ? load_beta(0) : (unsigned short)0;
         for (int c = 0; c < nchunks; ++c) {
-            const int stg = c & 1;
-            unsigned char *R = sm.raw[c & 1];
+            const int stg = c % PP::NS;
+            unsigned char *R = sm.raw[c % PP::NR];
             Stage &St = sm.st[stg];
             const int rows = min(kC, len - kC * c);
-            if (c >= 2) bar_sync(BAR_EMPTY + stg, kEmptyCount);  // the stage is free again
-            if (d == 0) {  // V tile of this chunk into the stage
-                const uint32_t mb = smem_u32(&sm.mb_v[stg]);
-                mbar_arrive_expect_tx(mb, 8192);
+            if (c >= PP::NS) bar_sync(PP::EMPTY + stg, kEmptyCount);  // the stage is free again
+            {   // V tile of this chunk into the stage by cp.async, in the layout a
+                // 128-byte-swizzled TMA box would have (MN-major A of MMA 1):
+                // piece (row r, half hh, 16-byte chunk q) at hh*4096 + r*128 + (q ^ (r & 7))*16
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh)
-                    tma_load_3d(smem_u32(St.v) + 4096 * hh, &maps.v, 64 * hh, h, t0 + kC * c, mb);
+                for (int i = 0; i < 4; ++i) {
+                    const int x = d + 128 * i, r = x >> 4, hh = (x >> 3) & 1, q = x & 7;
+                    const bool okr = r < rows;
+                    cp_async16(St.v + hh * 4096 + r * 128 + ((q ^ (r & 7)) << 4),
+                               vv + ((size_t)(t0 + kC * c + (okr ? r : 0)) * H + h) * kD + hh * 64 + q * 8, okr);
+                }
+                cp_async_commit();
+                // the v rows of a later chunk into L2 (one 128-byte line per thread)
+                const int cp = c + 6;
+                if (d < 64 && cp < nchunks && kC * cp + (d >> 1) < len)
+                    prefetch_l2(vv + ((size_t)(t0 + kC * cp + (d >> 1)) * H + h) * kD + (d & 1) * 64);
             }
             const unsigned short bq_next = d < kC ? load_beta(c + 1) : (unsigned short)0;
             if (d < kC) St.beta[d] = __bfloat162float(__ushort_as_bfloat16(bq));
-            if (tok) tok = mbar_wait(smem_u32(&sm.mb_raw[c & 1]), (c >> 1) & 1);
+            if (tok) tok = mbar_wait(smem_u32(&sm.mb_raw[c % PP::NR]), (c / PP::NR) & 1);
             if (rows < kC) {  // rows past the piece read as zero: decay 1, no write, no read
                 const int n = (kC - rows) * 8;  // 16-byte pieces per tile half
                 for (int x = d; x < 6 * n; x += 128) {
@@ -470,7 +530,7 @@ __device__ void run_piece(const PrefillParams &p, const Maps &maps, int t0, int 
                 }
             }
             __syncwarp();
-            bar_sync(BAR_DECAY, 128);
+            bar_sync(PP::DECAY, 128);
             // exp(g) and the inclusive prefix products over this tile's rows
             float2 e[16], E[16];
 #pragma unroll
@@ -488,45 +548,57 @@ __device__ void run_piece(const PrefillParams &p, const Maps &maps, int t0, int 
             }
             const float2 gc = E[15];
             *reinterpret_cast<float2 *>(&sm.gexch[sc][ip]) = gc;
-            bar_sync(BAR_DECAY, 128);
+            bar_sync(PP::DECAY, 128);
             const float2 go = *reinterpret_cast<const float2 *>(&sm.gexch[sc ^ 1][ip]);
             const float2 g0 = sc ? go : gc, g1 = sc ? gc : go;
             if (sc == 0) {
                 *reinterpret_cast<float2 *>(&St.gam[ip]) = f2mul(g0, g1);
-                *reinterpret_cast<float2 *>(&sm.gam0[c & 1][ip]) = g0;
+                *reinterpret_cast<float2 *>(&sm.gam0[stg][ip]) = g0;
             }
+            mbar_arrive(smem_u32(&sm.mb_gam[stg]));  // the state team may pre-scale with gamma
             const float2 inv = make_float2(__frcp_rn(gc.x), __frcp_rn(gc.y));
             const float2 kbs = sc ? make_float2(1.f, 1.f) : g1;  // Kbar scale of this tile
             const float2 qts = sc ? g0 : make_float2(1.f, 1.f);  // Q~ scale of this tile
-            float2 F = make_float2(1.f, 1.f);
             uint32_t kb0[8], kb1[8], qt0[8], qt1[8];  // Kbar / Q~ of channels ip, ip+1 (row pairs)
-            float2 kb_hi = make_float2(0.f, 0.f), qt_hi = make_float2(0.f, 0.f);
+            {   // k: the tile column first (the in-place stores below would otherwise
+                // keep every load behind the previous row's store), then suffix products
+                uint32_t kr[16];
 #pragma unroll
-            for (int r = 15; r >= 0; --r) {
-                const int row = 16 * sc + r;
-                const float2 kv = unpack_bf16(*reinterpret_cast<const uint32_t *>(R + rsw(OFF_K, row, ip)));
-                *reinterpret_cast<uint32_t *>(R + rsw(OFF_K, row, ip)) = pack_bf16(f2mul(kv, E[r]));
-                const float2 kF = f2mul(kv, F);
-                *reinterpret_cast<uint32_t *>(R + rsw(OFF_G, row, ip)) = pack_bf16(f2mul(kF, inv));
-                if (sc == 0) *reinterpret_cast<uint32_t *>(R + rsw(OFF_KB, r, ip)) = pack_bf16(kF);
-                const float2 kbv = f2mul(kF, kbs);
-                float2 qtv = make_float2(0.f, 0.f);
-                if (OUT) {
-                    const float2 qv = unpack_bf16(*reinterpret_cast<const uint32_t *>(R + rsw(OFF_Q, row, ip)));
-                    const float2 qd = f2mul(f2mul(qv, make_float2(p.scale, p.scale)), E[r]);
-                    *reinterpret_cast<uint32_t *>(R + rsw(OFF_Q, row, ip)) = pack_bf16(qd);
-                    qtv = f2mul(qd, qts);
+                for (int r = 0; r < 16; ++r) kr[r] = *reinterpret_cast<const uint32_t *>(R + rsw(OFF_K, 16 * sc + r, ip));
+                float2 F = make_float2(1.f, 1.f), kb_hi = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int r = 15; r >= 0; --r) {
+                    const int row = 16 * sc + r;
+                    const float2 kv = unpack_bf16(kr[r]);
+                    *reinterpret_cast<uint32_t *>(R + rsw(OFF_K, row, ip)) = pack_bf16(f2mul(kv, E[r]));
+                    const float2 kF = f2mul(kv, F);
+                    *reinterpret_cast<uint32_t *>(R + rsw(OFF_G, row, ip)) = pack_bf16(f2mul(kF, inv));
+                    if (sc == 0) *reinterpret_cast<uint32_t *>(R + rsw(OFF_KB, r, ip)) = pack_bf16(kF);
+                    const float2 kbv = f2mul(kF, kbs);
+                    if (r & 1) {
+                        kb_hi = kbv;
+                    } else {
+                        kb0[r >> 1] = pack_bf16(kbv.x, kb_hi.x);
+                        kb1[r >> 1] = pack_bf16(kbv.y, kb_hi.y);
+                    }
+                    F = f2mul(F, e[r]);
                 }
-                if (r & 1) {
-                    kb_hi = kbv;
-                    qt_hi = qtv;
-                } else {
-                    kb0[r >> 1] = pack_bf16(kbv.x, kb_hi.x);
-                    kb1[r >> 1] = pack_bf16(kbv.y, kb_hi.y);
-                    qt0[r >> 1] = pack_bf16(qtv.x, qt_hi.x);
-                    qt1[r >> 1] = pack_bf16(qtv.y, qt_hi.y);
+            }
+            if (OUT) {  // q: needs only the prefix products
+                uint32_t qr[16];
+#pragma unroll
+                for (int r = 0; r < 16; ++r) qr[r] = *reinterpret_cast<const uint32_t *>(R + rsw(OFF_Q, 16 * sc + r, ip));
+                const float2 sc2 = make_float2(p.scale, p.scale);
+#pragma unroll
+                for (int r = 0; r < 16; r += 2) {
+                    const float2 qd0 = f2mul(f2mul(unpack_bf16(qr[r]), sc2), E[r]);
+                    const float2 qd1 = f2mul(f2mul(unpack_bf16(qr[r + 1]), sc2), E[r + 1]);
+                    *reinterpret_cast<uint32_t *>(R + rsw(OFF_Q, 16 * sc + r, ip)) = pack_bf16(qd0);
+                    *reinterpret_cast<uint32_t *>(R + rsw(OFF_Q, 16 * sc + r + 1, ip)) = pack_bf16(qd1);
+                    const float2 t0 = f2mul(qd0, qts), t1 = f2mul(qd1, qts);
+                    qt0[r >> 1] = pack_bf16(t0.x, t1.x);
+                    qt1[r >> 1] = pack_bf16(t0.y, t1.y);
                 }
-                F = f2mul(F, e[r]);
             }
             // Kbar^T rows ip, ip + 1 (K-major [128][32]): tokens 16 sc .. 16 sc + 15
 #pragma unroll
@@ -546,20 +618,40 @@ __device__ void run_piece(const PrefillParams &p, const Maps &maps, int t0, int 
                         make_uint4(qt1[4 * hh], qt1[4 * hh + 1], qt1[4 * hh + 2], qt1[4 * hh + 3]);
                 }
             }
+            cp_async_wait<0>();  // this thread's part of the V tile has landed
             fence_async_smem();  // tiles and stage are read by the tensor core next
-            bar_arrive(BAR_DEC + (c & 1), kDecCount);
+            bar_sync(PP::DECAY, 128);
+            // ---- AP: [Qd_0; Qd_1; Kd_0; Kd_1] x [Ki_0; Ki_1; Kb_0]^T (summary: [Kd_0; Kd_1; ...])
+            // into AP buffer c % NS, issued as soon as the tiles are ready
+            if (d < 32) {
+                if (elect_one_sync()) {
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(R) + (OUT ? OFF_Q : OFF_K);
+                    const uint32_t b0 = smem_u32(R) + OFF_G;
+                    constexpr uint32_t ID_AP = idesc_bf16(64, 48, 0, 0);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+                        tc_mma_ss(tbase + Cols<OUT>::AP + 64 * stg, sdesc_sw128(a0 + off, 16, 1024),
+                                  sdesc_sw128(b0 + off, 16, 1024), ID_AP, kk > 0 ? 1u : 0u);
+                    }
+                    tc_commit(smem_u32(&sm.mb_ap[stg]));
+                }
+                __syncwarp();
+            }
+            bar_arrive(PP::DEC + c % PP::NR, kDecCount);
             bq = bq_next;
         }
         if (!tok && p.err) atomicOr(p.err, 2);
         // the stages of the last chunks come back before the CTA tears down
-        for (int c = max(nchunks - 2, 0); c < nchunks; ++c) bar_sync(BAR_EMPTY + (c & 1), kEmptyCount);
+        for (int c = max(nchunks - PP::NS, 0); c < nchunks; ++c) bar_sync(PP::EMPTY + c % PP::NS, kEmptyCount);
     } else {
         // =========================================================== matrix team
         const int m = tid - 384, mw = m >> 5;
         const uint32_t lane_off = (uint32_t)(mw * 32) << 16;
         auto issue_raw = [&](int c) {
-            unsigned char *R = sm.raw[c & 1];
-            const uint32_t mb = smem_u32(&sm.mb_raw[c & 1]);
+            unsigned char *R = sm.raw[c % PP::NR];
+            const uint32_t mb = smem_u32(&sm.mb_raw[c % PP::NR]);
             const int tc = t0 + kC * c;
             mbar_arrive_expect_tx(mb, (OUT ? 3u : 2u) * 2u * 4096u);
 #pragma unroll
@@ -571,44 +663,46 @@ __device__ void run_piece(const PrefillParams &p, const Maps &maps, int t0, int 
             }
         };
         if (m == 0)
-            for (int c = 0; c < min(nchunks, 2); ++c) issue_raw(c);
-        // rows 32-63 of [T~ ; 0] stay zero (the O columns of MMA 1)
-        for (int x = m; x < 2 * 128; x += 128)
+            for (int c = 0; c < min(nchunks, PP::NR); ++c) issue_raw(c);
+        // rows 32-63 of [T~ ; 0] (the O columns of MMA 1) and the block above
+        // the diagonal of T~ (rows 0-15, columns 16-31) stay zero
+        for (int x = m; x < PP::NS * 128; x += 128)
             reinterpret_cast<uint4 *>(sm.st[x >> 7].b0 + 2048)[x & 127] = make_uint4(0, 0, 0, 0);
+        for (int x = m; x < PP::NS * 32; x += 128) {
+            const int st = x >> 5, r = (x >> 1) & 15, hh = x & 1;
+            *reinterpret_cast<uint4 *>(sm.st[st].b0 + kmaj(r, 16 + 8 * hh, kC)) = make_uint4(0, 0, 0, 0);
+        }
+        // the first chunks' tiles into L2
+        auto prefetch = [&](int c) {
+            if (c >= nchunks) return;
+            const int tc = t0 + kC * c;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                tma_prefetch_3d(&maps.k, 64 * hh, h, tc);
+                tma_prefetch_3d(&maps.g, 64 * hh, h, tc);
+                if (OUT) tma_prefetch_3d(&maps.q, 64 * hh, h, tc);
+            }
+        };
+        if (m == 0)
+            for (int c = PP::NR; c < PP::NR + kPrefetch; ++c) prefetch(c);
         // A rows of the AP product: rows 32-63 in the output pass (after
         // Qd_0, Qd_1), rows 0-31 in the summary pass (no q)
         constexpr int kArow = OUT ? 2 : 0;
-        constexpr uint32_t ID_AP = idesc_bf16(64, 48, 0, 0);
         constexpr uint32_t ID_W = idesc_bf16(128, 32, 1, 0);
         bool ok = true;
 
         for (int c = 0; c < nchunks; ++c) {
-            const int stg = c & 1;
-            unsigned char *R = sm.raw[c & 1];
+            const int stg = c % PP::NS;
+            unsigned char *R = sm.raw[c % PP::NR];
             Stage &St = sm.st[stg];
-            bar_sync(BAR_DEC + (c & 1), kDecCount);  // Kd, Ki, Qd, Kb_0, beta, gamma of chunk c
-            // ---- AP: [Qd_0; Qd_1; Kd_0; Kd_1] x [Ki_0; Ki_1; Kb_0]^T
-            if (mw == 0 && ok) {
-                if (elect_one_sync()) {
-                    tc_fence_after();
-                    const uint32_t a0 = smem_u32(R) + (OUT ? OFF_Q : OFF_K);
-                    const uint32_t b0 = smem_u32(R) + OFF_G;
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-                        tc_mma_ss(tbase + Cols<OUT>::AP, sdesc_sw128(a0 + off, 16, 1024),
-                                  sdesc_sw128(b0 + off, 16, 1024), ID_AP, kk > 0 ? 1u : 0u);
-                    }
-                    tc_commit(smem_u32(&sm.mb_ap));
-                }
-                __syncwarp();
-            }
-            if (ok) ok = mbar_wait(smem_u32(&sm.mb_ap), c & 1);
+            bar_sync(PP::DEC + c % PP::NR, kDecCount);  // Kd, Ki, Qd, Kb_0, beta, gamma of chunk c
+            if (ok) ok = mbar_wait(smem_u32(&sm.mb_ap[stg]), (c / PP::NS) & 1);
             ok = all_ok(ok);
             tc_fence_after();
+            const uint32_t col_ap = Cols<OUT>::AP + 64 * stg;
             if (ok) {
                 // lanes 0-15 of quarter mw hold rows 16 mw .. 16 mw + 15 of D
-                const uint32_t ta = tbase + lane_off + Cols<OUT>::AP;
+                const uint32_t ta = tbase + lane_off + col_ap;
                 const int rr = lane;  // row within the 16-row block (lanes >= 16 idle)
                 if (mw == kArow) {  // rows of Kd_0: A00 (strictly lower)
                     uint32_t a[16];
@@ -676,34 +770,67 @@ __device__ void run_piece(const PrefillParams &p, const Maps &maps, int t0, int 
             }
             fence_async_smem();
             tc_fence_before();
-            bar_sync(BAR_MAT, 128);
-            // ---- T~ = (I + Diag(beta) A)^-1 Diag(beta): lane j of warp 12 owns
-            // column j; once row r is final it is pushed into every later row
+            bar_sync(PP::MAT, 128);
+            // ---- T = (I + N)^-1, N = Diag(beta) A, by blocks: the two 16 x 16
+            // diagonal blocks by forward substitution on one warp (lane l:
+            // block l / 16, column l % 16; once row r is final it is pushed into
+            // every later row), then T10 = -T11 (N10 T00) by all 128 threads,
+            // fp32 throughout.  T~ = T Diag(beta) into [T~ ; 0] as bf16.
             if (mw == 0 && ok) {
-                float x[kC];
+                const int blk = lane >> 4, jj = lane & 15, o = 16 * blk;
+                float x[16];
 #pragma unroll
-                for (int r = 0; r < kC; ++r) x[r] = (r == lane) ? 1.f : 0.f;
+                for (int r = 0; r < 16; ++r) x[r] = (r == jj) ? 1.f : 0.f;
 #pragma unroll
-                for (int r = 0; r < kC - 1; ++r) {
-                    float at[kC];
+                for (int r = 0; r < 15; ++r) {
+                    float at[16];
 #pragma unroll
-                    for (int q4 = 0; q4 < kC / 4; ++q4) {
-                        const float4 a4 = *reinterpret_cast<const float4 *>(&sm.AT[r * kC + 4 * q4]);
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const float4 a4 = *reinterpret_cast<const float4 *>(&sm.AT[(o + r) * kC + o + 4 * q4]);
                         at[4 * q4 + 0] = a4.x; at[4 * q4 + 1] = a4.y;
                         at[4 * q4 + 2] = a4.z; at[4 * q4 + 3] = a4.w;
                     }
 #pragma unroll
-                    for (int r2 = r + 1; r2 < kC; ++r2) x[r2] = fmaf(-at[r2], x[r], x[r2]);
+                    for (int r2 = r + 1; r2 < 16; ++r2) x[r2] = fmaf(-at[r2], x[r], x[r2]);
                 }
-                const float bj = St.beta[lane];
+                const float bj = St.beta[o + jj];
 #pragma unroll
-                for (int r = 0; r < kC; ++r)
-                    *reinterpret_cast<bf16 *>(St.b0 + kmaj(r, lane, kC)) = __float2bfloat16_rn(x[r] * bj);
-                fence_async_smem();
+                for (int r = 0; r < 16; ++r) {
+                    sm.Td[blk][r * 16 + jj] = x[r];
+                    *reinterpret_cast<bf16 *>(St.b0 + kmaj(o + r, o + jj, kC)) = __float2bfloat16_rn(x[r] * bj);
+                }
             }
+            bar_sync(PP::MAT, 128);
+            const int zi = m >> 3, zj = 2 * (m & 7);  // this thread's two entries of the 16 x 16 products
+            if (ok) {  // Z = N10 T00, N10[i][s] = AT[s][16 + i]
+                float2 z = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int s2 = 0; s2 < 16; ++s2) {
+                    const float n = sm.AT[s2 * kC + 16 + zi];
+                    const float2 t = *reinterpret_cast<const float2 *>(&sm.Td[0][s2 * 16 + zj]);
+                    z.x = fmaf(n, t.x, z.x);
+                    z.y = fmaf(n, t.y, z.y);
+                }
+                *reinterpret_cast<float2 *>(&sm.Zx[zi * 16 + zj]) = z;
+            }
+            bar_sync(PP::MAT, 128);
+            if (ok) {  // T10 = -T11 Z;  T~10 = T10 Diag(beta_0)
+                float2 t10 = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int k2 = 0; k2 < 16; ++k2) {
+                    const float t11 = sm.Td[1][zi * 16 + k2];
+                    const float2 z = *reinterpret_cast<const float2 *>(&sm.Zx[k2 * 16 + zj]);
+                    t10.x = fmaf(t11, z.x, t10.x);
+                    t10.y = fmaf(t11, z.y, t10.y);
+                }
+                *reinterpret_cast<uint32_t *>(St.b0 + kmaj(16 + zi, zj, kC)) =
+                    pack_bf16(-t10.x * St.beta[zj], -t10.y * St.beta[zj + 1]);
+            }
+            fence_async_smem();
             tc_fence_before();
-            bar_sync(BAR_MAT, 128);
-            // ---- W^T = Kd_0^T T~[:, 0:16]^T + Diag(gamma_0) Kd_1^T T~[:, 16:32]^T
+            bar_sync(PP::MAT, 128);
+            // ---- W^T = Kd_0^T T~[:, 0:16]^T + Diag(gamma_0) Kd_1^T T~[:, 16:32]^T,
+            // into this chunk's AP buffer (its Gram blocks have been read out)
             if (mw == 0 && ok) {
                 if (elect_one_sync()) {
                     tc_fence_after();
@@ -711,7 +838,7 @@ __device__ void run_piece(const PrefillParams &p, const Maps &maps, int t0, int 
                     const uint32_t bt = smem_u32(St.b0);
 #pragma unroll
                     for (int tt = 0; tt < 2; ++tt)  // tile tt: rows 16 tt .. of the k tile, columns 16 tt .. of T~
-                        tc_mma_ss(tbase + Cols<OUT>::W + 32 * tt, sdesc_sw128(kt + 2048 * tt, kHalf, 1024),
+                        tc_mma_ss(tbase + col_ap + 32 * tt, sdesc_sw128(kt + 2048 * tt, kHalf, 1024),
                                   sdesc(bt + 256 * tt, 128, 512), ID_W, 0u);
                     tc_commit(smem_u32(&sm.mb_w));
                 }
@@ -722,11 +849,11 @@ __device__ void run_piece(const PrefillParams &p, const Maps &maps, int t0, int 
             tc_fence_after();
             if (ok) {  // thread m = key channel i: -W[t][i] into row i of [-W | Q~]
                 uint32_t xa[32], ya[32];
-                const uint32_t tw = tbase + lane_off + Cols<OUT>::W;
+                const uint32_t tw = tbase + lane_off + col_ap;
                 tmem_ld32(tw, xa);
                 tmem_ld32(tw + 32, ya);
                 tc_wait_ld();
-                const float g0 = sm.gam0[c & 1][m];
+                const float g0 = sm.gam0[stg][m];
 #pragma unroll
                 for (int q8 = 0; q8 < 4; ++q8) {
                     uint32_t w4[4];
@@ -741,9 +868,12 @@ __device__ void run_piece(const PrefillParams &p, const Maps &maps, int t0, int 
             }
             fence_async_smem();
             tc_fence_before();
-            bar_sync(BAR_MAT, 128);  // every read of the raw tiles and of gam0 is done
-            if (m == 0 && c + 2 < nchunks) issue_raw(c + 2);
-            bar_arrive(BAR_FULL + stg, kFullCount);
+            bar_sync(PP::MAT, 128);  // every read of the raw tiles and of gam0 is done
+            if (m == 0) {
+                if (c + PP::NR < nchunks) issue_raw(c + PP::NR);
+                prefetch(c + PP::NR + kPrefetch);
+            }
+            bar_arrive(PP::FULL + stg, kFullCount);
         }
         if (!ok && m == 0 && p.err) atomicOr(p.err, 2);
     }
@@ -824,12 +954,8 @@ cudaError_t launch_prefill_c32(const PrefillParams &p, bool summaries, cudaStrea
     memset(&maps, 0, sizeof(maps));
     const int T = p.total_tokens, H = p.H;
     if (T > 0) {
-        bool ok = encode(&maps.k, p.k, T, H, true) && encode(&maps.g, p.g, T, H, true) &&
-                  encode(&maps.v, p.v, T, H, true);
-        if (!summaries) {
-            ok = ok && encode(&maps.q, p.q, T, H, true) && encode(&maps.out, p.out, T, H, false);
-            if (p.gate) ok = ok && encode(&maps.gate, p.gate, T, H, false);
-        }
+        bool ok = encode(&maps.k, p.k, T, H, true) && encode(&maps.g, p.g, T, H, true);
+        if (!summaries) ok = ok && encode(&maps.q, p.q, T, H, true);
         if (!ok) return cudaErrorInvalidValue;
     }
     const dim3 grid((unsigned)(p.P_max * p.H));

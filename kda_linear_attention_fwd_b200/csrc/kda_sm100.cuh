@@ -267,6 +267,11 @@ KDA_DEVICE bool mbar_try_wait(uint32_t mbar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// Plain arrive on an mbarrier (release: this thread's earlier writes are
+// visible to a thread whose wait observes the phase).
+KDA_DEVICE void mbar_arrive(uint32_t mbar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(mbar) : "memory");
+}
 // Arrive on the mbarrier and add `bytes` to the transaction count its current
 // phase waits for (the issuing thread of a TMA load).
 KDA_DEVICE void mbar_arrive_expect_tx(uint32_t mbar, uint32_t bytes) {
@@ -281,6 +286,12 @@ KDA_DEVICE void tma_load_3d(uint32_t dst, const void *tmap, int c0, int c1, int 
         "l"(tmap), "r"(mbar), "r"(c0), "r"(c1), "r"(c2)
         : "memory");
 }
+// Prefetch of one box of a 3-D tensor into L2 (no shared memory, no completion).
+KDA_DEVICE void tma_prefetch_3d(const void *tmap, int c0, int c1, int c2) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(tmap), "r"(c0),
+                 "r"(c1), "r"(c2)
+                 : "memory");
+}
 // Tiled TMA store of one box from this CTA's shared memory into a 3-D tensor
 // (bulk-group completion: commit, then wait on the group).
 KDA_DEVICE void tma_store_3d(const void *tmap, uint32_t src, int c0, int c1, int c2) {
@@ -293,12 +304,14 @@ KDA_DEVICE void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "
 KDA_DEVICE void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // This thread's committed bulk stores are complete.
 KDA_DEVICE void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-// Bounded wait on an mbarrier phase: gives up after ~2 s of wall time.
+// Bounded wait on an mbarrier phase: gives up after ~2 s of wall time.  Each
+// try may suspend the thread until the phase completes (or 10 us pass), so
+// waiting warps are parked instead of spinning through issue slots.
 KDA_DEVICE bool mbar_wait(uint32_t mbar, uint32_t parity) {
     if (mbar_try_wait(mbar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (;;) {
-        if (mbar_try_wait(mbar, parity)) return true;
+        if (mbar_try_wait_hint(mbar, parity, 10000u)) return true;
         if (global_timer_ns() - t0 > 2000000000ull) return false;
     }
 }

@@ -249,15 +249,25 @@ def test_chunk_fwd_check_validation(lib):
     assert lib.kda_chunk_fwd_check(A, 8, None) == INVALID  # smaller than the error words
 
 
-def test_plan_choices_on_148_sms(lib):
-    """The piece plan's cost model for the bf16 dk = dv = 128 plain call (the
-    32-token kernels: both passes one CTA per SM; waves of each pass plus scan
-    steps) on a 148-SM device; without a device the library assumes 148 SMs."""
+def test_plan_choices_on_148_sms(lib, monkeypatch):
+    """The piece plan's cost model on a 148-SM device (without a device the
+    library assumes 148 SMs).  Default (16-token kernels): waves of the output
+    pass at two CTAs per SM and of the paired summary pass at one, plus scan
+    steps.  With the 32-token kernels (KDA_PREFILL_IMPL=c32): both passes one
+    CTA per SM, pieces a multiple of 32 tokens."""
     import torch
     if torch.cuda.is_available() and torch.cuda.get_device_properties(0).multi_processor_count != 148:
         pytest.skip("plan depends on the SM count")
-    p = kda.plan(131072, 1, 32)
-    assert p["piece_len"] % 32 == 0
-    assert p["piece_len"] == 14592                        # 9 pieces per head: 288 CTAs, 2 waves
-    assert kda.plan(8192, 2, 16)["piece_len"] == 1024     # 4 pieces per sequence
+    assert kda.plan(131072, 1, 32)["piece_len"] == 3552   # 37 pieces per head
+    assert kda.plan(8192, 2, 16)["piece_len"] == 464      # 9 pieces per sequence
     assert kda.plan(256, 1, 2) == {"piece_len": 256, "max_pieces": 2, "launches": 2}  # one piece
+    monkeypatch.setenv("KDA_PREFILL_IMPL", "c32")
+    assert kda.plan(131072, 1, 32)["piece_len"] == 14592  # 9 pieces per head: 288 CTAs, 2 waves
+    assert kda.plan(8192, 2, 16)["piece_len"] == 1024     # 4 pieces per sequence
+    # the workspace covers either plan
+    f = lib.kda_chunk_fwd_workspace_size
+    for T, N, H in [(131072, 1, 32), (8192, 2, 16), (48317, 8, 32)]:
+        for impl in ("c32", "tc5"):
+            monkeypatch.setenv("KDA_PREFILL_IMPL", impl)
+            p = kda.plan(T, N, H)
+            assert f(T, N, H, 128, 128, BF16) >= p["max_pieces"] * H * 3 * 128 * 128 * 4
