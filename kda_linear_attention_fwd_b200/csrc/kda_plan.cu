@@ -132,6 +132,13 @@ __global__ void __launch_bounds__(256) scan_kernel(PrefillParams p) {
         p.Sin[((size_t)(f + 1) * H + h) * SS + (size_t)i * DV + c] = z;
         sm.Sp[i][col] = z;
     }
+    // S_zero of the piece the next step adds, loaded one step ahead so that
+    // its global-memory latency overlaps the current product
+    float zn[RW];
+    if (np > 2) {
+#pragma unroll
+        for (int r = 0; r < RW; ++r) zn[r] = p.Szero[((size_t)(f + 1) * H + h) * SS + (size_t)(rg * RW + r) * DV + c];
+    }
     for (int j = 2; j < np; ++j) {
         const int buf = j & 1;
         if (j + 1 < np) {
@@ -141,16 +148,27 @@ __global__ void __launch_bounds__(256) scan_kernel(PrefillParams p) {
             asm volatile("cp.async.wait_group 0;\n" ::: "memory");
         }
         __syncthreads();
-        const size_t pp = (size_t)(f + j - 1) * H + h;
         const float *Ms = sm.M[buf];
         float acc[RW];
 #pragma unroll
-        for (int r = 0; r < RW; ++r) acc[r] = p.Szero[pp * SS + (size_t)(rg * RW + r) * DV + c];
-#pragma unroll 4
-        for (int kk = 0; kk < DK; ++kk) {
-            const float sv = sm.Sp[kk][col];
+        for (int r = 0; r < RW; ++r) acc[r] = zn[r];
+        if (j + 1 < np) {
 #pragma unroll
-            for (int r = 0; r < RW; ++r) acc[r] += Ms[(rg * RW + r) * DK + kk] * sv;
+            for (int r = 0; r < RW; ++r)
+                zn[r] = p.Szero[((size_t)(f + j) * H + h) * SS + (size_t)(rg * RW + r) * DV + c];
+        }
+#pragma unroll 2
+        for (int kk = 0; kk < DK; kk += 4) {  // four k at a time: float4 reads of the M rows
+            const float s0 = sm.Sp[kk][col], s1 = sm.Sp[kk + 1][col];
+            const float s2 = sm.Sp[kk + 2][col], s3 = sm.Sp[kk + 3][col];
+#pragma unroll
+            for (int r = 0; r < RW; ++r) {
+                const float4 m4 = *reinterpret_cast<const float4 *>(&Ms[(rg * RW + r) * DK + kk]);
+                acc[r] = fmaf(m4.x, s0, acc[r]);
+                acc[r] = fmaf(m4.y, s1, acc[r]);
+                acc[r] = fmaf(m4.z, s2, acc[r]);
+                acc[r] = fmaf(m4.w, s3, acc[r]);
+            }
         }
         __syncthreads();
 #pragma unroll

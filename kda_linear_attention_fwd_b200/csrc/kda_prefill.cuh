@@ -81,9 +81,10 @@ struct PlanModel {
     double scan_cost;   // one scan step, in output chunk steps
 };
 // The 16-token kernels: output pass two CTAs per SM, the paired summary one;
-// 0.79 is the measured ratio of their per-chunk periods (about 3.0 K and
-// 3.8 K SM cycles), a scan step about two output chunk steps.
-inline PlanModel plan_model_chunk16(int sms) { return PlanModel{16, 2L * sms, (long)sms, 0.79, 2.0}; }
+// 0.67 is the measured ratio of their per-chunk periods at full occupancy
+// (about 2.96 K and 4.44 K SM cycles), a scan step about two output chunk
+// steps.
+inline PlanModel plan_model_chunk16(int sms) { return PlanModel{16, 2L * sms, (long)sms, 0.67, 2.0}; }
 // The 32-token kernels (bf16, dk = dv = 128): both passes one CTA per SM.
 inline PlanModel plan_model_chunk32(int sms) { return PlanModel{32, (long)sms, (long)sms, 1.0, 6.0}; }
 

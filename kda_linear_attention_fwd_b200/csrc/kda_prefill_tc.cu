@@ -263,49 +263,51 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
         // exp(G_C) so that its MMA 3 can accumulate U^T Kb straight into it.
         // src: nullptr = read the state from TMEM; else an initial state.
         auto state_pass = [&](const float *gam_next, bool from_init, float *snap_out) {
+            // 64 columns per round: both TMEM loads in flight before one wait
 #pragma unroll 1
-            for (int cb = 0; cb < DK / 32; ++cb) {
-                uint32_t d[32];
+            for (int cb = 0; cb < DK / 64; ++cb) {
+                uint32_t d[64];
                 if (from_init) {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int i = 32 * cb + e;
+                    for (int e = 0; e < 64; ++e) {
+                        const int i = 64 * cb + e;
                         d[e] = __float_as_uint(identity ? (i == j ? 1.f : 0.f)
                                                         : (s_init ? s_init[(size_t)i * NC + j] : 0.f));
                     }
                 } else {
-                    tmem_ld32_wait(t_s + 32 * cb, d);
+                    tmem_ld32(t_s + 64 * cb, *reinterpret_cast<uint32_t(*)[32]>(&d[0]));
+                    tmem_ld32(t_s + 64 * cb + 32, *reinterpret_cast<uint32_t(*)[32]>(&d[32]));
+                    tc_wait_ld();
                     if (snap_out) {  // a state snapshot after this chunk
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) snap_out[(size_t)(32 * cb + e) * NC + j] = __uint_as_float(d[e]);
+                        for (int e = 0; e < 64; ++e) snap_out[(size_t)(64 * cb + e) * NC + j] = __uint_as_float(d[e]);
                     }
                 }
-                uint32_t pk[16];
+                {
+                    uint32_t pk[32];
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    pk[e] = pack_bf16(__uint_as_float(d[2 * e]), __uint_as_float(d[2 * e + 1]));
-                tmem_st16(t_as + 16 * cb, pk);
+                    for (int e = 0; e < 32; ++e)
+                        pk[e] = pack_bf16(__uint_as_float(d[2 * e]), __uint_as_float(d[2 * e + 1]));
+                    tmem_st32(t_as + 32 * cb, pk);
+                }
                 if (gam_next) {
-                    uint32_t lo[16], hi[16];
 #pragma unroll
-                    for (int e4 = 0; e4 < 8; ++e4) {
-                        const float4 gm = *reinterpret_cast<const float4 *>(&gam_next[32 * cb + 4 * e4]);
+                    for (int e4 = 0; e4 < 16; ++e4) {
+                        const float4 gm = *reinterpret_cast<const float4 *>(&gam_next[64 * cb + 4 * e4]);
                         const float2 a = f2mul(make_float2(__uint_as_float(d[4 * e4]), __uint_as_float(d[4 * e4 + 1])),
                                                make_float2(gm.x, gm.y));
                         const float2 b = f2mul(make_float2(__uint_as_float(d[4 * e4 + 2]), __uint_as_float(d[4 * e4 + 3])),
                                                make_float2(gm.z, gm.w));
-                        uint32_t *dst = e4 < 4 ? lo : hi;
-                        const int o = (e4 & 3) * 4;
-                        dst[o + 0] = __float_as_uint(a.x);
-                        dst[o + 1] = __float_as_uint(a.y);
-                        dst[o + 2] = __float_as_uint(b.x);
-                        dst[o + 3] = __float_as_uint(b.y);
+                        d[4 * e4] = __float_as_uint(a.x);
+                        d[4 * e4 + 1] = __float_as_uint(a.y);
+                        d[4 * e4 + 2] = __float_as_uint(b.x);
+                        d[4 * e4 + 3] = __float_as_uint(b.y);
                     }
-                    tmem_st16(t_s + 32 * cb, lo);
-                    tmem_st16(t_s + 32 * cb + 16, hi);
+                    tmem_st32(t_s + 64 * cb, *reinterpret_cast<uint32_t(*)[32]>(&d[0]));
+                    tmem_st32(t_s + 64 * cb + 32, *reinterpret_cast<uint32_t(*)[32]>(&d[32]));
                 } else if (s_out) {  // after the last chunk: the final state
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) s_out[(size_t)(32 * cb + e) * NC + j] = __uint_as_float(d[e]);
+                    for (int e = 0; e < 64; ++e) s_out[(size_t)(64 * cb + e) * NC + j] = __uint_as_float(d[e]);
                 }
             }
             tc_wait_st();
@@ -519,33 +521,42 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
             const float2 El = E[15];
             const float2 invEl = make_float2(__frcp_rn(El.x), __frcp_rn(El.y));
             *reinterpret_cast<float2 *>(&St.gam[ip]) = El;
-            float2 F = make_float2(1.f, 1.f);
             uint32_t kb0[8], kb1[8];  // Kb^T rows ip, ip + 1 (token pairs)
-            float2 kb_hi = make_float2(0.f, 0.f);
+            {   // k: the tile column first (the in-place stores below would otherwise
+                // keep every load behind the previous row's store)
+                uint32_t kr[16];
 #pragma unroll
-            for (int r = 15; r >= 0; --r) {
-                float2 kv = unpack_bf16(*reinterpret_cast<const uint32_t *>(Wk.k + sw128(r, ip)));
-                float sc = p.scale;
-                if (L2N) {
-                    const float rk = pr.rk[r];
-                    kv = f2mul(kv, make_float2(rk, rk));
-                    sc = pr.rq[r];
+                for (int r = 0; r < 16; ++r) kr[r] = *reinterpret_cast<const uint32_t *>(Wk.k + sw128(r, ip));
+                float2 F = make_float2(1.f, 1.f), kb_hi = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int r = 15; r >= 0; --r) {
+                    float2 kv = unpack_bf16(kr[r]);
+                    if (L2N) {
+                        const float rk = pr.rk[r];
+                        kv = f2mul(kv, make_float2(rk, rk));
+                    }
+                    *reinterpret_cast<uint32_t *>(Wk.k + sw128(r, ip)) = pack_bf16(f2mul(kv, E[r]));
+                    *reinterpret_cast<uint32_t *>(Wk.g + sw128(r, ip)) = pack_bf16(f2mul(kv, f2mul(F, invEl)));
+                    const float2 kbv = f2mul(kv, F);
+                    if (r & 1) {
+                        kb_hi = kbv;
+                    } else {
+                        kb0[r >> 1] = pack_bf16(kbv.x, kb_hi.x);
+                        kb1[r >> 1] = pack_bf16(kbv.y, kb_hi.y);
+                    }
+                    F = f2mul(F, e[r]);
                 }
-                *reinterpret_cast<uint32_t *>(Wk.k + sw128(r, ip)) = pack_bf16(f2mul(kv, E[r]));
-                *reinterpret_cast<uint32_t *>(Wk.g + sw128(r, ip)) = pack_bf16(f2mul(kv, f2mul(F, invEl)));
-                const float2 kbv = f2mul(kv, F);
-                if (r & 1) {
-                    kb_hi = kbv;
-                } else {
-                    kb0[r >> 1] = pack_bf16(kbv.x, kb_hi.x);
-                    kb1[r >> 1] = pack_bf16(kbv.y, kb_hi.y);
-                }
-                if (OUT) {
-                    const float2 qv = unpack_bf16(*reinterpret_cast<const uint32_t *>(Wk.q + sw128(r, ip)));
+            }
+            if (OUT) {  // q: needs only the prefix products (and the row norms)
+                uint32_t qr[16];
+#pragma unroll
+                for (int r = 0; r < 16; ++r) qr[r] = *reinterpret_cast<const uint32_t *>(Wk.q + sw128(r, ip));
+#pragma unroll
+                for (int r = 0; r < 16; ++r) {
+                    const float sc = L2N ? pr.rq[r] : p.scale;
                     *reinterpret_cast<uint32_t *>(Wk.q + sw128(r, ip)) =
-                        pack_bf16(f2mul(f2mul(qv, make_float2(sc, sc)), E[r]));
+                        pack_bf16(f2mul(f2mul(unpack_bf16(qr[r]), make_float2(sc, sc)), E[r]));
                 }
-                F = f2mul(F, e[r]);
             }
             *reinterpret_cast<uint4 *>(at_bytes(St.b2, kmaj(ip, 0, 16))) = make_uint4(kb0[0], kb0[1], kb0[2], kb0[3]);
             *reinterpret_cast<uint4 *>(at_bytes(St.b2, kmaj(ip, 8, 16))) = make_uint4(kb0[4], kb0[5], kb0[6], kb0[7]);

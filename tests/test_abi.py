@@ -258,7 +258,7 @@ def test_plan_choices_on_148_sms(lib, monkeypatch):
     import torch
     if torch.cuda.is_available() and torch.cuda.get_device_properties(0).multi_processor_count != 148:
         pytest.skip("plan depends on the SM count")
-    assert kda.plan(131072, 1, 32)["piece_len"] == 3552   # 37 pieces per head
+    assert kda.plan(131072, 1, 32)["piece_len"] == 14576  # 9 pieces per head: 288 CTAs, one wave
     assert kda.plan(8192, 2, 16)["piece_len"] == 464      # 9 pieces per sequence
     assert kda.plan(256, 1, 2) == {"piece_len": 256, "max_pieces": 2, "launches": 2}  # one piece
     monkeypatch.setenv("KDA_PREFILL_IMPL", "c32")
