@@ -80,102 +80,139 @@ __global__ void __launch_bounds__(1024)
 }
 
 // Prefix scan over the pieces of one sequence, for one head and one block of
-// 16 state columns:
+// 32 state columns:
 //   Sin[first]     = initial state (or zeros)
 //   Sin[first + 1] = Szero[first]       (piece 0 is summarised from the
 //                                         initial state itself, no M needed)
 //   Sin[first + j] = M[first + j - 1] Sin[first + j - 1] + Szero[first + j - 1]
-// fp32 throughout.  Each M (dk x dk) is staged in shared memory with cp.async,
-// the next one loading while the current product runs.  Thread t: column
-// t % 16, rows (t / 16) * DK/16 ... + DK/16 - 1.
-constexpr int kScanCols = 16;
+// fp32 throughout.  Each M (dk x dk) is staged in shared memory in two halves
+// of dk/2 key channels by cp.async; while one half is in use the next one is
+// in flight, so a step never waits for a whole matrix.  Thread t owns the
+// four columns 4 (t % 8) .. + 3 of rows t / 8 + 32 r and updates them with
+// packed fp32 pair FMAs.  84 KB of shared memory (dk = 128): two CTAs per SM.
+constexpr int kScanCols = 32;
+constexpr int kScanThreads = 256;
 
-template <int DK, int DV>
+template <int DK>
 struct ScanSmem {
-    float M[2][DK * DK];
-    float Sp[DK][kScanCols + 1];
-    static constexpr size_t bytes() { return sizeof(float) * (2 * DK * DK + DK * (kScanCols + 1)); }
+    static constexpr int KH = DK / 2;  // key channels in one half of M
+    static constexpr int LD = KH + 4;  // padded row: rows one apart fall in different banks
+    float M[2][DK * LD];               // M[:, 0:KH] and M[:, KH:DK]
+    float4 Sp[DK][kScanCols / 4];      // the running state, this CTA's columns
+    static constexpr size_t bytes() {
+        return sizeof(float) * 2 * DK * LD + sizeof(float4) * DK * (kScanCols / 4);
+    }
 };
 
+KDA_DEVICE float2 fma2(float a, float2 b, float2 c) {
+    uint64_t d;
+    const float2 aa = make_float2(a, a);
+    asm("fma.rn.f32x2 %0, %1, %2, %3;"
+        : "=l"(d)
+        : "l"(*reinterpret_cast<const uint64_t *>(&aa)), "l"(*reinterpret_cast<const uint64_t *>(&b)),
+          "l"(*reinterpret_cast<const uint64_t *>(&c)));
+    return *reinterpret_cast<float2 *>(&d);
+}
+
 template <int DK, int DV>
-__global__ void __launch_bounds__(256) scan_kernel(PrefillParams p) {
-    constexpr int RW = DK / 16;  // rows per thread
+__global__ void __launch_bounds__(kScanThreads) scan_kernel(PrefillParams p) {
+    constexpr int RW = DK / 32;  // rows per thread
+    constexpr int KH = ScanSmem<DK>::KH, LD = ScanSmem<DK>::LD;
     extern __shared__ __align__(16) unsigned char scan_smem[];
-    ScanSmem<DK, DV> &sm = *reinterpret_cast<ScanSmem<DK, DV> *>(scan_smem);
+    ScanSmem<DK> &sm = *reinterpret_cast<ScanSmem<DK> *>(scan_smem);
     const int n = blockIdx.x, h = blockIdx.y;
-    const int col = threadIdx.x % kScanCols, rg = threadIdx.x / kScanCols;
-    const int c = blockIdx.z * kScanCols + col;
+    const int cq = threadIdx.x % 8, rg = threadIdx.x / 8;
+    const int c = blockIdx.z * kScanCols + 4 * cq;  // first of this thread's four columns
     const int f = p.seq_first[n];
     const int np = p.seq_first[n + 1] - f;
     if (np <= 1 || f + np > p.P_max) return;
     const int H = p.H;
     const size_t SS = (size_t)DK * DV, MS = (size_t)DK * DK;
     const float *init = p.initial_state ? p.initial_state + ((size_t)n * H + h) * SS : nullptr;
+    // element (row, c) of the state-sized entry of `piece` in `base`
+    auto st_at = [&](size_t piece, int row) { return ((size_t)piece * H + h) * SS + (size_t)row * DV + c; };
 
-    auto load_M = [&](int buf, int piece) {
-        const float4 *src = reinterpret_cast<const float4 *>(p.M + ((size_t)piece * H + h) * MS);
-        float4 *dst = reinterpret_cast<float4 *>(sm.M[buf]);
-        for (int x = threadIdx.x; x < DK * DK / 4; x += 256) {
-            const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst + x));
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(src + x)
+    // one half of M of `piece` -> buffer `half` (one cp.async group)
+    auto load_half = [&](int piece, int half) {
+        const float *src = p.M + ((size_t)piece * H + h) * MS + half * KH;
+        float *dst = sm.M[half];
+        for (int x = threadIdx.x; x < DK * KH / 4; x += kScanThreads) {
+            const int row = x / (KH / 4), c4 = x % (KH / 4);
+            const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst + row * LD + 4 * c4));
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(src + (size_t)row * DK + 4 * c4)
                          : "memory");
         }
         asm volatile("cp.async.commit_group;\n" ::: "memory");
     };
-    if (np > 2) load_M(0, f + 1);
+    if (np > 2) {
+        load_half(f + 1, 0);
+        load_half(f + 1, 1);
+    }
 
 #pragma unroll
     for (int r = 0; r < RW; ++r) {
-        const int i = rg * RW + r;
-        p.Sin[((size_t)f * H + h) * SS + (size_t)i * DV + c] = init ? init[(size_t)i * DV + c] : 0.f;
-        const float z = p.Szero[((size_t)f * H + h) * SS + (size_t)i * DV + c];
-        p.Sin[((size_t)(f + 1) * H + h) * SS + (size_t)i * DV + c] = z;
-        sm.Sp[i][col] = z;
+        const int row = rg + 32 * r;
+        const float4 s0 = init ? *reinterpret_cast<const float4 *>(init + (size_t)row * DV + c)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<float4 *>(p.Sin + st_at(f, row)) = s0;
+        const float4 z = *reinterpret_cast<const float4 *>(p.Szero + st_at(f, row));
+        *reinterpret_cast<float4 *>(p.Sin + st_at(f + 1, row)) = z;
+        sm.Sp[row][cq] = z;
     }
     // S_zero of the piece the next step adds, loaded one step ahead so that
     // its global-memory latency overlaps the current product
-    float zn[RW];
+    float4 zn[RW];
     if (np > 2) {
 #pragma unroll
-        for (int r = 0; r < RW; ++r) zn[r] = p.Szero[((size_t)(f + 1) * H + h) * SS + (size_t)(rg * RW + r) * DV + c];
+        for (int r = 0; r < RW; ++r) zn[r] = *reinterpret_cast<const float4 *>(p.Szero + st_at(f + 1, rg + 32 * r));
     }
     for (int j = 2; j < np; ++j) {
-        const int buf = j & 1;
-        if (j + 1 < np) {
-            load_M(buf ^ 1, f + j);
-            asm volatile("cp.async.wait_group 1;\n" ::: "memory");
-        } else {
-            asm volatile("cp.async.wait_group 0;\n" ::: "memory");
-        }
-        __syncthreads();
-        const float *Ms = sm.M[buf];
-        float acc[RW];
-#pragma unroll
-        for (int r = 0; r < RW; ++r) acc[r] = zn[r];
-        if (j + 1 < np) {
-#pragma unroll
-            for (int r = 0; r < RW; ++r)
-                zn[r] = p.Szero[((size_t)(f + j) * H + h) * SS + (size_t)(rg * RW + r) * DV + c];
-        }
-#pragma unroll 2
-        for (int kk = 0; kk < DK; kk += 4) {  // four k at a time: float4 reads of the M rows
-            const float s0 = sm.Sp[kk][col], s1 = sm.Sp[kk + 1][col];
-            const float s2 = sm.Sp[kk + 2][col], s3 = sm.Sp[kk + 3][col];
-#pragma unroll
-            for (int r = 0; r < RW; ++r) {
-                const float4 m4 = *reinterpret_cast<const float4 *>(&Ms[(rg * RW + r) * DK + kk]);
-                acc[r] = fmaf(m4.x, s0, acc[r]);
-                acc[r] = fmaf(m4.y, s1, acc[r]);
-                acc[r] = fmaf(m4.z, s2, acc[r]);
-                acc[r] = fmaf(m4.w, s3, acc[r]);
-            }
-        }
-        __syncthreads();
+        const bool more = j + 1 < np;
+        float2 acc[RW][2];
 #pragma unroll
         for (int r = 0; r < RW; ++r) {
-            const int i = rg * RW + r;
-            sm.Sp[i][col] = acc[r];
-            p.Sin[((size_t)(f + j) * H + h) * SS + (size_t)i * DV + c] = acc[r];
+            acc[r][0] = make_float2(zn[r].x, zn[r].y);
+            acc[r][1] = make_float2(zn[r].z, zn[r].w);
+        }
+        if (more) {
+#pragma unroll
+            for (int r = 0; r < RW; ++r) zn[r] = *reinterpret_cast<const float4 *>(p.Szero + st_at(f + j, rg + 32 * r));
+        }
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            // in flight: this half, then the other one or the next step's first
+            if (hf == 0 || more) {
+                asm volatile("cp.async.wait_group 1;\n" ::: "memory");
+            } else {
+                asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+            }
+            __syncthreads();  // the half (and the previous step's state) is visible
+            const float *Mh = sm.M[hf];
+#pragma unroll 2
+            for (int kk = 0; kk < KH; kk += 4) {
+                float4 s[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) s[i] = sm.Sp[hf * KH + kk + i][cq];
+#pragma unroll
+                for (int r = 0; r < RW; ++r) {
+                    const float4 m4 = *reinterpret_cast<const float4 *>(Mh + (rg + 32 * r) * LD + kk);
+                    const float mv[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        acc[r][0] = fma2(mv[i], make_float2(s[i].x, s[i].y), acc[r][0]);
+                        acc[r][1] = fma2(mv[i], make_float2(s[i].z, s[i].w), acc[r][1]);
+                    }
+                }
+            }
+            __syncthreads();  // every thread is done with this half (and with the state)
+            if (more) load_half(f + j, hf);
+        }
+#pragma unroll
+        for (int r = 0; r < RW; ++r) {
+            const int row = rg + 32 * r;
+            const float4 v = make_float4(acc[r][0].x, acc[r][0].y, acc[r][1].x, acc[r][1].y);
+            sm.Sp[row][cq] = v;
+            *reinterpret_cast<float4 *>(p.Sin + st_at(f + j, row)) = v;
         }
     }
 }
@@ -189,11 +226,11 @@ cudaError_t launch_plan(const int32_t *cu, int num_seqs, int total_tokens, int p
 
 template <int DK, int DV>
 static cudaError_t launch_scan_t(const PrefillParams &p, cudaStream_t st) {
-    const size_t sm = ScanSmem<DK, DV>::bytes();
+    const size_t sm = ScanSmem<DK>::bytes();
     cudaError_t e = cudaFuncSetAttribute(scan_kernel<DK, DV>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
-    scan_kernel<DK, DV><<<dim3(p.num_seqs, p.H, DV / kScanCols), 256, sm, st>>>(p);
+    scan_kernel<DK, DV><<<dim3(p.num_seqs, p.H, DV / kScanCols), kScanThreads, sm, st>>>(p);
     return cudaGetLastError();
 }
 

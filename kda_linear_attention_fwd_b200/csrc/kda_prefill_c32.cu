@@ -896,7 +896,7 @@ __global__ void __launch_bounds__(kThreads, 1) summary_kernel(PrefillParams p, c
     const int n = pc.x, j = pc.w;
     const int np = p.seq_first[n + 1] - p.seq_first[n];
     const bool want_s = p.summarize_all || j < np - 1;
-    const bool want_m = p.summarize_all || j > 0;
+    const bool want_m = p.summarize_all || (j > 0 && j < np - 1);
     if (!want_s && !want_m) return;
     const size_t ph = (size_t)pi * p.H + h;
     const float *init = (j == 0 && p.initial_state) ? p.initial_state + ((size_t)n * p.H + h) * kD * kD : nullptr;

@@ -22,16 +22,19 @@
 // tensor work, keeping every named-barrier hand-off so that no warp is left
 // waiting.
 //
-// The prep team (warps 4-7) prepares one chunk at a time into one of three
-// stages: cp.async of q, k, g two chunks ahead into a ring of raw tiles and of
-// v into the stage; exp(G) as prefix and suffix products of exp(g) with one
-// thread per key-channel pair and half of the rows; the Gram matrices
-// A = Kd Ki^T and P = Qd Ki^T on two warps in parallel (16x16 tiles are far
-// below the smallest tcgen05 tile, so these use warp-level MMA); the 16x16
-// unit-lower solve in fp32 on one warp; W = Tb Kd split over the four warps
-// by key channel.  Every MMA operand is written in the canonical no-swizzle
-// K-major / MN-major layout.  A stage goes back to the team as soon as the
-// update MMAs that read it have completed.
+// The prep team (the four warps after the state warps: a decay pair and a
+// matrix pair, interleaved over the SM sub-partitions) prepares one chunk at a
+// time into one of three stages: TMA loads of q, k, g up to three chunks ahead
+// into a ring of raw tiles (128-byte swizzle) and cp.async of v into the
+// stage; exp(G) as prefix and suffix products of exp(g), one decay thread per
+// key-channel pair over the 16 rows, rewriting the raw tiles in place into
+// Qd, Kd and Ki and writing Kb^T; the Gram matrices A = Kd Ki^T and
+// P = Qd Ki^T on the two matrix warps in parallel (16x16 tiles are far below
+// the smallest tcgen05 tile, so these use warp-level MMA); the 16x16
+// unit-lower solve in fp32 on one warp; W = Tb Kd split over the two matrix
+// warps by key channel.  Every MMA operand the prep writes is in the
+// canonical no-swizzle K-major / MN-major layout.  A stage goes back to the
+// team as soon as the update MMAs that read it have completed.
 //
 // Sources: the token pipeline and the decay floor -- affta.cn K3 explainer,
 // section "第一关：KDA 解决算得动"; decay as an absolute-position transform over a
@@ -412,11 +415,14 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
             }
         }
         if (active && !ok && lane == 0 && p.err) atomicOr(p.err, 1);
-    } else if (warp < 4 * NWG + 2) {
+    } else if (((warp - 4 * NWG) & 1) == 0) {
         // ------------------------------------------------------------ decay pair
-        // Warps 4-5: thread d owns the key-channel pair (ip, ip + 1) on all 16
-        // rows of a chunk; it runs up to kRaw chunks ahead of the matrix pair.
-        const int d = tid - 128 * NWG, dw = d >> 5, ip = 2 * d;
+        // The first and third warp after the state warps (their warp slots put
+        // them on two different SM sub-partitions, each shared with a matrix
+        // warp rather than with the other decay warp): thread d owns the
+        // key-channel pair (ip, ip + 1) on all 16 rows of a chunk; it runs up
+        // to kRaw chunks ahead of the matrix pair.
+        const int dw = (warp - 4 * NWG) >> 1, d = 32 * dw + lane, ip = 2 * d;
         const bf16 *v = (const bf16 *)p.v, *beta = (const bf16 *)p.beta;
         typename Lay::Prep &pr = sm.pr;
         // beta of chunks c and c + 1 (threads d < 16), kept as raw bf16 bits so
@@ -575,9 +581,9 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
         for (int c = max(nchunks - kStages, 0); c < nchunks; ++c) bar_sync(BAR_EMPTY + c % kStages, kBarCount);
     } else {
         // ----------------------------------------------------------- matrix pair
-        // Warps 6-7: the Gram matrices, the unit-lower solve, W, and the TMA
-        // loads of q, k, g (thread 0).
-        const int m = tid - 128 * NWG - kPair, mw = m >> 5;
+        // The second and fourth warp after the state warps: the Gram matrices,
+        // the unit-lower solve, W, and the TMA loads of q, k, g (thread 0).
+        const int mw = (warp - 4 * NWG) >> 1, m = 32 * mw + lane;
         typename Lay::Prep &pr = sm.pr;
         auto issue_raw = [&](int c) {
             typename Lay::Raw &R = sm.raw[c % kRaw];
@@ -725,8 +731,8 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
 // 0 runs the piece from zero (or from the sequence's initial state for its
 // first piece) into S_zero, warpgroup 1 runs it from the identity without v
 // into the transition M; both share one preparation of every chunk.  A part
-// the scan does not need (S_zero of a sequence's last piece, M of its first)
-// is skipped unless every piece's map is asked for.
+// the scan does not need (both maps of a sequence's last piece, M of its
+// first) is skipped unless every piece's map is asked for.
 template <int DK, bool L2N, bool EXT>
 __global__ void __launch_bounds__(kThreadsOf<2>, 1)
     summary_kernel(PrefillParams p, const __grid_constant__ TmaMaps maps) {
@@ -739,7 +745,7 @@ __global__ void __launch_bounds__(kThreadsOf<2>, 1)
     const int n = pc.x, j = pc.w;
     const int np = p.seq_first[n + 1] - p.seq_first[n];
     const bool want_s = p.summarize_all || j < np - 1;
-    const bool want_m = p.summarize_all || j > 0;
+    const bool want_m = p.summarize_all || (j > 0 && j < np - 1);
     if (!want_s && !want_m) return;
     const size_t ph = (size_t)pi * p.H + h;
     const float *init = (j == 0 && p.initial_state)
