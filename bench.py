@@ -17,6 +17,7 @@ collective); value = tokens over all ranks / max-over-ranks device time.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import ctypes
 import json
 import os
@@ -279,6 +280,9 @@ def main():
                     help="skip the backward measurement")
     ap.add_argument("--out-dir", default=os.path.join(tempfile.gettempdir(), "kda_bench"),
                     help="where the nvidia-smi clock samples of the timed region are written")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="profiling only: run a one-sequence workload at this length (a smaller case "
+                         "of the same kernels); 0 = the workload's own length")
     ap.add_argument("--ref-tokens", type=int, default=0,
                     help="reference arm: tokens per step sample (0 = scale with cores)")
     args = ap.parse_args()
@@ -303,6 +307,10 @@ def main():
 
     # ---------------- prefill ----------------
     w = W.get(args.workload)
+    if args.tokens:
+        if len(w.lengths) != 1:
+            raise SystemExit("--tokens applies to one-sequence workloads only")
+        w = dataclasses.replace(w, lengths=(args.tokens,))
     T, N = w.total_tokens, w.num_seqs
     inp = W.fast_prefill(w, seed=w.seed + 1000 * rank, device=dev)
     out = torch.empty(T, w.H, w.dv, dtype=w.torch_dtype, device=dev)
@@ -340,7 +348,8 @@ def main():
     pflops = prefill_flops(w, T)
     hbm = pk["hbm_gbs"]
     achieved = pbytes / (ms / 1e3) / 1e9
-    traffic, _, traffic_src = measured_traffic(args.workload)
+    traffic, _, traffic_src = (measured_traffic(args.workload) if not args.tokens
+                               else (None, None, "shortened workload"))
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                 "frac": achieved / hbm,
                 "traffic": traffic,

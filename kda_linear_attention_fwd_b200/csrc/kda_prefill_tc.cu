@@ -10,11 +10,12 @@
 //   MMA 1  D1      = V^T [Tb^T | 0]             (M=128, N=32, K=16; A MN-major smem)
 //   MMA 2  D1     += S^T [-W^T | Qd^T]          (K=128; A = bf16 S^T in TMEM)
 //          -> D1[:, 0:16] = U^T, D1[:, 16:32] = (Qd S)^T
+//   WG     (while MMA 1/2 run) S^T scaled in place by the chunk's exp(G_C);
+//          y = gate (.) O of the previous chunk
 //   WG     U^T (bf16) -> shared memory (A operand of the next two)
-//   MMA 3  S^T    += U^T Kb                     (M=128, N=128, K=16; S^T pre-scaled)
+//   MMA 3  S^T    += U^T Kb                     (M=128, N=128, K=16)
 //   MMA 4  D1[16:] += U^T P^T                   (M=128, N=16, K=16) -> O^T
-//   WG     y = gate (.) O;  one pass over S^T: its bf16 copy, and S^T scaled
-//          by the next chunk's exp(G_C) so that its MMA 3 accumulates into it
+//   WG     the bf16 copy of S^T for the next chunk's MMA 2
 //
 // One elected lane issues the MMAs; tcgen05.commit arrives on an mbarrier that
 // the warpgroup waits on with a time bound (2 s): a wait that gives up records
@@ -77,6 +78,8 @@ template <int NWG> constexpr int kBarCountOf = 128 * NWG + kPair;  // FULL and E
 constexpr int kDecCount = 2 * kPair;
 constexpr int NC = 128;        // state columns = TMEM lanes = MMA M
 constexpr uint32_t kTmemColsPerWG = 256;
+constexpr int kAT = 20;        // row stride of the solve's AT matrix: the Gram epilogue's
+                               // scattered stores fall in distinct banks
 
 // TMA descriptors of q, k and g as [T][H][128] bf16 (3-D: channel, head,
 // token); one box = 64 channels x 1 head x 16 tokens, 128-byte swizzle.
@@ -114,7 +117,7 @@ struct Layout {
         alignas(16) float gam[DK];      // exp(G_C) per key channel
     };
     struct Prep {
-        alignas(16) float AT[16 * 16];  // AT[s][r] = beta_r A[r][s], r > s (matrix pair)
+        alignas(16) float AT[16 * kAT];  // AT[s][r] = beta_r A[r][s], r > s (matrix pair)
         float beta[kStages][16];        // beta of the chunk in each stage
         float nk[2][16], nq[2][16];     // per decay warp and row: partial sums of k^2, q^2
         float rk[16], rq[16];           // 1/|k_r| and scale/|q_r| of the chunk being decayed
@@ -260,12 +263,14 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
                         *reinterpret_cast<const uint4 *>(&tile[r * NC + cc * 8]);
             }
         };
-        // One pass over the fp32 state in TMEM (32 columns at a time): its
-        // bf16 copy becomes the A operand of the next chunk's MMA 2, and, when
-        // a next chunk exists, the state is pre-scaled by that chunk's
-        // exp(G_C) so that its MMA 3 can accumulate U^T Kb straight into it.
-        // src: nullptr = read the state from TMEM; else an initial state.
-        auto state_pass = [&](const float *gam_next, bool from_init, float *snap_out) {
+        // One pass over the fp32 state (from TMEM, or the initial state when
+        // from_init): its bf16 copy becomes the A operand of the next chunk's
+        // MMA 2 (not needed after the last chunk, which writes the final state
+        // instead), and with gam_next the fp32 state is stored back scaled by
+        // that chunk's exp(G_C), so that its MMA 3 accumulates U^T Kb straight
+        // into it.  Between chunks the scaling is left to scale_pass, which
+        // runs while the next chunk's MMA 1/2 are in flight.
+        auto state_pass = [&](const float *gam_next, bool from_init, float *snap_out, bool last) {
             // 64 columns per round: both TMEM loads in flight before one wait
 #pragma unroll 1
             for (int cb = 0; cb < DK / 64; ++cb) {
@@ -286,7 +291,7 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
                         for (int e = 0; e < 64; ++e) snap_out[(size_t)(64 * cb + e) * NC + j] = __uint_as_float(d[e]);
                     }
                 }
-                {
+                if (!last) {
                     uint32_t pk[32];
 #pragma unroll
                     for (int e = 0; e < 32; ++e)
@@ -308,13 +313,40 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
                     }
                     tmem_st32(t_s + 64 * cb, *reinterpret_cast<uint32_t(*)[32]>(&d[0]));
                     tmem_st32(t_s + 64 * cb + 32, *reinterpret_cast<uint32_t(*)[32]>(&d[32]));
-                } else if (s_out) {  // after the last chunk: the final state
+                } else if (last && s_out) {  // after the last chunk: the final state
 #pragma unroll
                     for (int e = 0; e < 64; ++e) s_out[(size_t)(64 * cb + e) * NC + j] = __uint_as_float(d[e]);
                 }
             }
             tc_wait_st();
             tc_fence_before();
+        };
+        // The fp32 state scaled in place by the chunk's exp(G_C) (gam), ahead
+        // of the MMA 3 that accumulates into it; the TMEM stores are complete
+        // on return.
+        auto scale_pass = [&](const float *gam) {
+#pragma unroll 1
+            for (int cb = 0; cb < DK / 64; ++cb) {
+                uint32_t d[64];
+                tmem_ld32(t_s + 64 * cb, *reinterpret_cast<uint32_t(*)[32]>(&d[0]));
+                tmem_ld32(t_s + 64 * cb + 32, *reinterpret_cast<uint32_t(*)[32]>(&d[32]));
+                tc_wait_ld();
+#pragma unroll
+                for (int e4 = 0; e4 < 16; ++e4) {
+                    const float4 gm = *reinterpret_cast<const float4 *>(&gam[64 * cb + 4 * e4]);
+                    const float2 a = f2mul(make_float2(__uint_as_float(d[4 * e4]), __uint_as_float(d[4 * e4 + 1])),
+                                           make_float2(gm.x, gm.y));
+                    const float2 b = f2mul(make_float2(__uint_as_float(d[4 * e4 + 2]), __uint_as_float(d[4 * e4 + 3])),
+                                           make_float2(gm.z, gm.w));
+                    d[4 * e4] = __float_as_uint(a.x);
+                    d[4 * e4 + 1] = __float_as_uint(a.y);
+                    d[4 * e4 + 2] = __float_as_uint(b.x);
+                    d[4 * e4 + 3] = __float_as_uint(b.y);
+                }
+                tmem_st32(t_s + 64 * cb, *reinterpret_cast<uint32_t(*)[32]>(&d[0]));
+                tmem_st32(t_s + 64 * cb + 32, *reinterpret_cast<uint32_t(*)[32]>(&d[32]));
+            }
+            tc_wait_st();
         };
 
         if (nchunks == 0) {
@@ -326,7 +358,7 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
             }
         } else {
             bar_sync(BAR_FULL + 0, kBarCount);  // stage of chunk 0: its exp(G_C)
-            if (ok) state_pass(sm.st[0].gam, true, nullptr);
+            if (ok) state_pass(sm.st[0].gam, true, nullptr, false);
         }
         // MMA operand descriptors of stage 0; stages are contiguous, so stage s
         // adds s * sizeof(Stage) / 16 to the start-address field (all of shared
@@ -363,6 +395,7 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
                 }
                 __syncwarp();  // reconverge warp 0 before the aligned TMEM loads below
             }
+            if (c > 0 && ok) scale_pass(sm.st[stg].gam);  // S_{c-1} -> Diag(exp G_C) S_{c-1}
             if (c > 0) finish_chunk(c - 1);
             if (ok) ok = mbar_wait(mb1, c & 1);
             ok = __all_sync(0xffffffffu, ok);
@@ -399,8 +432,7 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
             tc_fence_before();
             bar_arrive(BAR_EMPTY + stg, kBarCount);  // every reader of this stage is done
             if (ok) {
-                state_pass(has_next ? sm.st[(c + 1) % kStages].gam : nullptr, false,
-                           EXT ? snap.at(snap.pos0 + 16 * (c + 1)) : nullptr);
+                state_pass(nullptr, false, EXT ? snap.at(snap.pos0 + 16 * (c + 1)) : nullptr, !has_next);
             } else {
                 tc_fence_before();
             }
@@ -441,7 +473,10 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
                 constexpr int PV = NC / 8;
 #pragma unroll
                 for (int x = d; x < 16 * PV; x += kPair) {
-                    const int r = x / PV, cc = x % PV;
+                    // token fastest: the 16-byte pieces of one warp fill whole
+                    // core matrices (no bank conflicts) and pairs of them whole
+                    // 32-byte sectors of v
+                    const int r = x % 16, cc = x / 16;
                     const bool okr = r < rows;
                     const size_t off = ((size_t)(okr ? tc + r : t0) * H + h) * NC + cc * 8;
                     cp_async16(at_bytes(Sv.v, mnmaj(cc * 8, r, 16)), v + off, okr);
@@ -633,7 +668,7 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
                     for (int e2 = 0; e2 < 8; ++e2) {
                         const int r = r0 + ((e2 & 2) ? 8 : 0);
                         const int sc = c0 + (e2 & 1) + ((e2 & 4) ? 8 : 0);
-                        pr.AT[sc * 16 + r] = sc < r ? bet[r] * vals[e2] : 0.f;
+                        pr.AT[sc * kAT + r] = sc < r ? bet[r] * vals[e2] : 0.f;
                     }
                 } else {
                     auto pv = [&](float x, int r, int sc) { return sc <= r ? x : 0.f; };
@@ -664,7 +699,7 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
                         float at[16];
 #pragma unroll
                         for (int q4 = 0; q4 < 4; ++q4) {
-                            const float4 a4 = *reinterpret_cast<const float4 *>(&pr.AT[r * 16 + 4 * q4]);
+                            const float4 a4 = *reinterpret_cast<const float4 *>(&pr.AT[r * kAT + 4 * q4]);
                             at[4 * q4 + 0] = a4.x; at[4 * q4 + 1] = a4.y;
                             at[4 * q4 + 2] = a4.z; at[4 * q4 + 3] = a4.w;
                         }
