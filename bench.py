@@ -50,17 +50,22 @@ def peaks():
 
 # DRAM traffic of the dominant kernel, per launch: read from the committed
 # ncu summary profiles/traffic.json, which records the figure together with a
-# hash of the CUDA sources it was captured from.  When the sources differ
-# from that hash (a kernel changed since the capture) the figure is stale and
-# `traffic` is reported as null.
+# hash of the sources of the prefill call it was captured from (its entry
+# point, the plan and scan, the chunk kernels and their headers).  When those
+# differ from the hash (a kernel on the path changed since the capture) the
+# figure is stale and `traffic` is reported as null.
+PREFILL_SOURCES = ("kda_api.cu", "kda_args.h", "kda_plan.cu", "kda_prefill_c32.cu", "kda_prefill_mma.cu",
+                   "kda_prefill_simt.cu", "kda_prefill_tc.cu", "kda_common.cuh", "kda_prefill.cuh",
+                   "kda_sm100.cuh")
+
+
 def source_hash():
-    import glob
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "kda_linear_attention_fwd_b200", "csrc")
-    for path in sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh"))):
-        with open(path, "rb") as f:
-            h.update(os.path.basename(path).encode() + b"\0" + f.read())
+    for name in PREFILL_SOURCES:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 
