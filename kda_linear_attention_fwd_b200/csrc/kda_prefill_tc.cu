@@ -10,7 +10,8 @@
 //   MMA 1  D1      = V^T [Tb^T | 0]             (M=128, N=32, K=16; A MN-major smem)
 //   MMA 2  D1     += S^T [-W^T | Qd^T]          (K=128; A = bf16 S^T in TMEM)
 //          -> D1[:, 0:16] = U^T, D1[:, 16:32] = (Qd S)^T
-//   WG     (while MMA 1/2 run) S^T scaled in place by the chunk's exp(G_C);
+//   WG     (while MMA 1/2 run) S^T scaled in place by the chunk's exp(G_C)
+//          (the plain kernels; the others scale it at the end of the previous chunk);
 //          y = gate (.) O of the previous chunk
 //   WG     U^T (bf16) -> shared memory (A operand of the next two)
 //   MMA 3  S^T    += U^T Kb                     (M=128, N=128, K=16)
@@ -268,54 +269,71 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
         // MMA 2 (not needed after the last chunk, which writes the final state
         // instead), and with gam_next the fp32 state is stored back scaled by
         // that chunk's exp(G_C), so that its MMA 3 accumulates U^T Kb straight
-        // into it.  Between chunks the scaling is left to scale_pass, which
-        // runs while the next chunk's MMA 1/2 are in flight.
+        // into it.  Between chunks the plain kernels leave the scaling to
+        // scale_pass, which runs while the next chunk's MMA 1/2 are in flight.
+        // SW state columns per round of a pass: 64 (both TMEM loads in flight
+        // before one wait) in the plain kernels, 32 in the variants with the
+        // norms or the extended features, which have fewer registers to spare
+        constexpr int SW = (L2N || EXT) ? 32 : 64;
+        // the plain kernels scale the state while MMA 1/2 run (scale_pass);
+        // the heavier variants keep the single pass after MMA 3, whose
+        // registers they can afford
+        constexpr bool kSplitPass = !L2N && !EXT;
+        auto ld_round = [&](int cb, uint32_t (&d)[SW]) {
+            tmem_ld32(t_s + SW * cb, *reinterpret_cast<uint32_t(*)[32]>(&d[0]));
+            if constexpr (SW == 64) tmem_ld32(t_s + SW * cb + 32, *reinterpret_cast<uint32_t(*)[32]>(&d[SW - 32]));
+            tc_wait_ld();
+        };
+        auto st_round = [&](int cb, uint32_t (&d)[SW]) {
+            tmem_st32(t_s + SW * cb, *reinterpret_cast<uint32_t(*)[32]>(&d[0]));
+            if constexpr (SW == 64) tmem_st32(t_s + SW * cb + 32, *reinterpret_cast<uint32_t(*)[32]>(&d[SW - 32]));
+        };
+        auto scale_round = [&](const float *gam, int cb, uint32_t (&d)[SW]) {
+#pragma unroll
+            for (int e4 = 0; e4 < SW / 4; ++e4) {
+                const float4 gm = *reinterpret_cast<const float4 *>(&gam[SW * cb + 4 * e4]);
+                const float2 a = f2mul(make_float2(__uint_as_float(d[4 * e4]), __uint_as_float(d[4 * e4 + 1])),
+                                       make_float2(gm.x, gm.y));
+                const float2 b = f2mul(make_float2(__uint_as_float(d[4 * e4 + 2]), __uint_as_float(d[4 * e4 + 3])),
+                                       make_float2(gm.z, gm.w));
+                d[4 * e4] = __float_as_uint(a.x);
+                d[4 * e4 + 1] = __float_as_uint(a.y);
+                d[4 * e4 + 2] = __float_as_uint(b.x);
+                d[4 * e4 + 3] = __float_as_uint(b.y);
+            }
+        };
         auto state_pass = [&](const float *gam_next, bool from_init, float *snap_out, bool last) {
-            // 64 columns per round: both TMEM loads in flight before one wait
 #pragma unroll 1
-            for (int cb = 0; cb < DK / 64; ++cb) {
-                uint32_t d[64];
+            for (int cb = 0; cb < DK / SW; ++cb) {
+                uint32_t d[SW];
                 if (from_init) {
 #pragma unroll
-                    for (int e = 0; e < 64; ++e) {
-                        const int i = 64 * cb + e;
+                    for (int e = 0; e < SW; ++e) {
+                        const int i = SW * cb + e;
                         d[e] = __float_as_uint(identity ? (i == j ? 1.f : 0.f)
                                                         : (s_init ? s_init[(size_t)i * NC + j] : 0.f));
                     }
                 } else {
-                    tmem_ld32(t_s + 64 * cb, *reinterpret_cast<uint32_t(*)[32]>(&d[0]));
-                    tmem_ld32(t_s + 64 * cb + 32, *reinterpret_cast<uint32_t(*)[32]>(&d[32]));
-                    tc_wait_ld();
+                    ld_round(cb, d);
                     if (snap_out) {  // a state snapshot after this chunk
 #pragma unroll
-                        for (int e = 0; e < 64; ++e) snap_out[(size_t)(64 * cb + e) * NC + j] = __uint_as_float(d[e]);
+                        for (int e = 0; e < SW; ++e) snap_out[(size_t)(SW * cb + e) * NC + j] = __uint_as_float(d[e]);
                     }
                 }
                 if (!last) {
-                    uint32_t pk[32];
+                    uint32_t pk[SW / 2];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
+                    for (int e = 0; e < SW / 2; ++e)
                         pk[e] = pack_bf16(__uint_as_float(d[2 * e]), __uint_as_float(d[2 * e + 1]));
-                    tmem_st32(t_as + 32 * cb, pk);
+                    if constexpr (SW == 64) tmem_st32(t_as + 32 * cb, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+                    else tmem_st16(t_as + 16 * cb, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
                 }
                 if (gam_next) {
-#pragma unroll
-                    for (int e4 = 0; e4 < 16; ++e4) {
-                        const float4 gm = *reinterpret_cast<const float4 *>(&gam_next[64 * cb + 4 * e4]);
-                        const float2 a = f2mul(make_float2(__uint_as_float(d[4 * e4]), __uint_as_float(d[4 * e4 + 1])),
-                                               make_float2(gm.x, gm.y));
-                        const float2 b = f2mul(make_float2(__uint_as_float(d[4 * e4 + 2]), __uint_as_float(d[4 * e4 + 3])),
-                                               make_float2(gm.z, gm.w));
-                        d[4 * e4] = __float_as_uint(a.x);
-                        d[4 * e4 + 1] = __float_as_uint(a.y);
-                        d[4 * e4 + 2] = __float_as_uint(b.x);
-                        d[4 * e4 + 3] = __float_as_uint(b.y);
-                    }
-                    tmem_st32(t_s + 64 * cb, *reinterpret_cast<uint32_t(*)[32]>(&d[0]));
-                    tmem_st32(t_s + 64 * cb + 32, *reinterpret_cast<uint32_t(*)[32]>(&d[32]));
+                    scale_round(gam_next, cb, d);
+                    st_round(cb, d);
                 } else if (last && s_out) {  // after the last chunk: the final state
 #pragma unroll
-                    for (int e = 0; e < 64; ++e) s_out[(size_t)(64 * cb + e) * NC + j] = __uint_as_float(d[e]);
+                    for (int e = 0; e < SW; ++e) s_out[(size_t)(SW * cb + e) * NC + j] = __uint_as_float(d[e]);
                 }
             }
             tc_wait_st();
@@ -326,25 +344,11 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
         // on return.
         auto scale_pass = [&](const float *gam) {
 #pragma unroll 1
-            for (int cb = 0; cb < DK / 64; ++cb) {
-                uint32_t d[64];
-                tmem_ld32(t_s + 64 * cb, *reinterpret_cast<uint32_t(*)[32]>(&d[0]));
-                tmem_ld32(t_s + 64 * cb + 32, *reinterpret_cast<uint32_t(*)[32]>(&d[32]));
-                tc_wait_ld();
-#pragma unroll
-                for (int e4 = 0; e4 < 16; ++e4) {
-                    const float4 gm = *reinterpret_cast<const float4 *>(&gam[64 * cb + 4 * e4]);
-                    const float2 a = f2mul(make_float2(__uint_as_float(d[4 * e4]), __uint_as_float(d[4 * e4 + 1])),
-                                           make_float2(gm.x, gm.y));
-                    const float2 b = f2mul(make_float2(__uint_as_float(d[4 * e4 + 2]), __uint_as_float(d[4 * e4 + 3])),
-                                           make_float2(gm.z, gm.w));
-                    d[4 * e4] = __float_as_uint(a.x);
-                    d[4 * e4 + 1] = __float_as_uint(a.y);
-                    d[4 * e4 + 2] = __float_as_uint(b.x);
-                    d[4 * e4 + 3] = __float_as_uint(b.y);
-                }
-                tmem_st32(t_s + 64 * cb, *reinterpret_cast<uint32_t(*)[32]>(&d[0]));
-                tmem_st32(t_s + 64 * cb + 32, *reinterpret_cast<uint32_t(*)[32]>(&d[32]));
+            for (int cb = 0; cb < DK / SW; ++cb) {
+                uint32_t d[SW];
+                ld_round(cb, d);
+                scale_round(gam, cb, d);
+                st_round(cb, d);
             }
             tc_wait_st();
         };
@@ -395,7 +399,7 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
                 }
                 __syncwarp();  // reconverge warp 0 before the aligned TMEM loads below
             }
-            if (c > 0 && ok) scale_pass(sm.st[stg].gam);  // S_{c-1} -> Diag(exp G_C) S_{c-1}
+            if (kSplitPass && c > 0 && ok) scale_pass(sm.st[stg].gam);  // S_{c-1} -> Diag(exp G_C) S_{c-1}
             if (c > 0) finish_chunk(c - 1);
             if (ok) ok = mbar_wait(mb1, c & 1);
             ok = __all_sync(0xffffffffu, ok);
@@ -432,7 +436,8 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
             tc_fence_before();
             bar_arrive(BAR_EMPTY + stg, kBarCount);  // every reader of this stage is done
             if (ok) {
-                state_pass(nullptr, false, EXT ? snap.at(snap.pos0 + 16 * (c + 1)) : nullptr, !has_next);
+                state_pass(kSplitPass || !has_next ? nullptr : sm.st[(c + 1) % kStages].gam, false,
+                           EXT ? snap.at(snap.pos0 + 16 * (c + 1)) : nullptr, !has_next);
             } else {
                 tc_fence_before();
             }
@@ -563,19 +568,18 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
             const float2 invEl = make_float2(__frcp_rn(El.x), __frcp_rn(El.y));
             *reinterpret_cast<float2 *>(&St.gam[ip]) = El;
             uint32_t kb0[8], kb1[8];  // Kb^T rows ip, ip + 1 (token pairs)
-            {   // k: the tile column first (the in-place stores below would otherwise
-                // keep every load behind the previous row's store)
+            if constexpr (!L2N && !EXT) {
+                // plain kernels: each tile column is loaded ahead of the in-place
+                // stores (which would otherwise keep every load behind the
+                // previous row's store); k last row first (the suffix products
+                // run backwards), then q
                 uint32_t kr[16];
 #pragma unroll
                 for (int r = 0; r < 16; ++r) kr[r] = *reinterpret_cast<const uint32_t *>(Wk.k + sw128(r, ip));
                 float2 F = make_float2(1.f, 1.f), kb_hi = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int r = 15; r >= 0; --r) {
-                    float2 kv = unpack_bf16(kr[r]);
-                    if (L2N) {
-                        const float rk = pr.rk[r];
-                        kv = f2mul(kv, make_float2(rk, rk));
-                    }
+                    const float2 kv = unpack_bf16(kr[r]);
                     *reinterpret_cast<uint32_t *>(Wk.k + sw128(r, ip)) = pack_bf16(f2mul(kv, E[r]));
                     *reinterpret_cast<uint32_t *>(Wk.g + sw128(r, ip)) = pack_bf16(f2mul(kv, f2mul(F, invEl)));
                     const float2 kbv = f2mul(kv, F);
@@ -587,16 +591,43 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
                     }
                     F = f2mul(F, e[r]);
                 }
-            }
-            if (OUT) {  // q: needs only the prefix products (and the row norms)
-                uint32_t qr[16];
+                if (OUT) {
+                    uint32_t qr[16];
 #pragma unroll
-                for (int r = 0; r < 16; ++r) qr[r] = *reinterpret_cast<const uint32_t *>(Wk.q + sw128(r, ip));
+                    for (int r = 0; r < 16; ++r) qr[r] = *reinterpret_cast<const uint32_t *>(Wk.q + sw128(r, ip));
 #pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    const float sc = L2N ? pr.rq[r] : p.scale;
-                    *reinterpret_cast<uint32_t *>(Wk.q + sw128(r, ip)) =
-                        pack_bf16(f2mul(f2mul(unpack_bf16(qr[r]), make_float2(sc, sc)), E[r]));
+                    for (int r = 0; r < 16; ++r)
+                        *reinterpret_cast<uint32_t *>(Wk.q + sw128(r, ip)) =
+                            pack_bf16(f2mul(f2mul(unpack_bf16(qr[r]), make_float2(p.scale, p.scale)), E[r]));
+                }
+            } else {
+                // the variants with the norms or the extended features (fewer
+                // registers to spare): k and q row by row in one backward loop
+                float2 F = make_float2(1.f, 1.f), kb_hi = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int r = 15; r >= 0; --r) {
+                    float2 kv = unpack_bf16(*reinterpret_cast<const uint32_t *>(Wk.k + sw128(r, ip)));
+                    float sc = p.scale;
+                    if (L2N) {
+                        const float rk = pr.rk[r];
+                        kv = f2mul(kv, make_float2(rk, rk));
+                        sc = pr.rq[r];
+                    }
+                    *reinterpret_cast<uint32_t *>(Wk.k + sw128(r, ip)) = pack_bf16(f2mul(kv, E[r]));
+                    *reinterpret_cast<uint32_t *>(Wk.g + sw128(r, ip)) = pack_bf16(f2mul(kv, f2mul(F, invEl)));
+                    const float2 kbv = f2mul(kv, F);
+                    if (r & 1) {
+                        kb_hi = kbv;
+                    } else {
+                        kb0[r >> 1] = pack_bf16(kbv.x, kb_hi.x);
+                        kb1[r >> 1] = pack_bf16(kbv.y, kb_hi.y);
+                    }
+                    if (OUT) {
+                        const float2 qv = unpack_bf16(*reinterpret_cast<const uint32_t *>(Wk.q + sw128(r, ip)));
+                        *reinterpret_cast<uint32_t *>(Wk.q + sw128(r, ip)) =
+                            pack_bf16(f2mul(f2mul(qv, make_float2(sc, sc)), E[r]));
+                    }
+                    F = f2mul(F, e[r]);
                 }
             }
             *reinterpret_cast<uint4 *>(at_bytes(St.b2, kmaj(ip, 0, 16))) = make_uint4(kb0[0], kb0[1], kb0[2], kb0[3]);
