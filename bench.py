@@ -108,57 +108,72 @@ def decode_bytes(wd):
 
 
 class Clocks:
-    """nvidia-smi sampler for the timed region."""
+    """nvidia-smi sampler for the timed region: samples every 20 ms, and
+    only those whose timestamps fall between mark_start() and mark_end()
+    count (the region can be shorter than one sample period; then the
+    nearest samples stand in and `samples` says 0)."""
 
     def __init__(self, path):
         self.path = path
         self.proc = None
+        self.t0 = self.t1 = None
 
     def start(self):
         try:
             uuid = "GPU-" + str(torch.cuda.get_device_properties(torch.cuda.current_device()).uuid)
-            q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+            q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
                  "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", uuid, f"--query-gpu={q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "20"],
                                          stdout=self.f, stderr=subprocess.DEVNULL)
-            time.sleep(0.3)
+            deadline = time.time() + 5.0  # until the sampler is live
+            while time.time() < deadline and os.path.getsize(self.path) == 0:
+                time.sleep(0.05)
         except Exception:
             self.proc = None
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
 
     def stop(self):
         if self.proc is None:
             return None
-        time.sleep(0.25)
+        time.sleep(0.1)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
         self.f.close()
-        sm, mx, reasons = [], None, set()
-        names = ["active", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
-                 "sw_power_cap"]
+        from datetime import datetime
+        rows = []
         with open(self.path) as f:
             for line in f:
                 parts = [x.strip() for x in line.split(",")]
-                if len(parts) < 9:
+                if len(parts) < 10:
                     continue
                 try:
-                    sm.append(float(parts[1]))
-                    mx = float(parts[2])
+                    t = datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                    rows.append((t, float(parts[2]), float(parts[3]), parts[6:10]))
                 except ValueError:
                     continue
-                for name, val in zip(names[1:], parts[5:9]):
-                    if val.lower() == "active":
-                        reasons.add(name)
-        if not sm:
+        if not rows:
             return None
-        load = [x for x in sm if mx is None or x > 0.5 * mx] or sm
+        t0 = self.t0 if self.t0 is not None else rows[0][0]
+        t1 = self.t1 if self.t1 is not None else rows[-1][0]
+        inside = [r for r in rows if t0 <= r[0] <= t1]
+        used = inside or sorted(rows, key=lambda r: min(abs(r[0] - t0), abs(r[0] - t1)))[:2]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = {n for r in used for n, v in zip(names, r[3]) if v.lower() == "active"}
+        mx = used[-1][2]
+        load = [r[1] for r in used if r[1] > 0.5 * mx] or [r[1] for r in used]
         return {"sm_mhz": statistics.median(load), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(inside)}
 
 
 def rank_env():
@@ -268,7 +283,7 @@ def run_reference(args, ws, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="long_bf16")
@@ -339,11 +354,13 @@ def main():
     barrier(ws)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks.mark_start()
     e0.record(stream)
     for _ in range(args.steps):
         prefill()
     e1.record(stream)
     torch.cuda.synchronize()
+    clocks.mark_end()
     barrier(ws)
     ms_total = reduce_max(e0.elapsed_time(e1), ws)
     clk = clocks.stop()

@@ -48,3 +48,32 @@ def test_committed_traffic_entries_are_complete():
         assert {"source_hash", "bytes_per_launch", "kernel", "source"} <= set(e), workload
         assert os.path.exists(os.path.join(ROOT, e["source"])), e["source"]
         assert e["bytes_per_launch"] > 0
+
+
+def test_clock_samples_are_taken_inside_the_timed_region(tmp_path):
+    """Only nvidia-smi samples stamped between mark_start and mark_end count;
+    a throttle reason seen there is reported, one outside is not."""
+    import time
+    from datetime import datetime
+    path = tmp_path / "clocks.csv"
+    t = time.time()
+    with open(path, "w") as f:
+        for k in range(10):
+            ts = datetime.fromtimestamp(t + 0.02 * k).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+            sm = 1965 if 2 <= k <= 6 else 1200
+            cap = "Active" if k == 4 else "Not Active"
+            slow = "Active" if k == 8 else "Not Active"
+            f.write(f"{ts}, 0, {sm}, 1965, 700.0, 0x0, {slow}, Not Active, Not Active, {cap}\n")
+
+    class Done:
+        def terminate(self):
+            pass
+
+        def wait(self, timeout=None):
+            pass
+
+    c = bench.Clocks(str(path))
+    c.proc, c.f = Done(), open(os.devnull, "w")
+    c.t0, c.t1 = t + 0.035, t + 0.125
+    r = c.stop()
+    assert r == {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 5}
