@@ -25,12 +25,13 @@
 // waiting.
 //
 // The prep team (the four warps after the state warps: a decay pair and a
-// matrix pair, interleaved over the SM sub-partitions) prepares one chunk at a
-// time into one of three stages: TMA loads of q, k, g up to three chunks ahead
-// into a ring of raw tiles (128-byte swizzle) and cp.async of v into the
-// stage; exp(G) as prefix and suffix products of exp(g), one decay thread per
-// key-channel pair over the 16 rows, rewriting the raw tiles in place into
-// Qd, Kd and Ki and writing Kb^T; the Gram matrices A = Kd Ki^T and
+// matrix pair, interleaved over the SM sub-partitions in the plain kernels)
+// prepares one chunk at a time into one of three stages: TMA loads of q, k, g
+// up to three chunks ahead into a ring of raw tiles (128-byte swizzle) and
+// cp.async of v into the stage; exp(G) as prefix and suffix products of
+// exp(g), one decay thread per key-channel pair over the 16 rows, rewriting
+// the raw tiles in place into Qd, Kd and Ki and writing Kb^T; the Gram
+// matrices A = Kd Ki^T and
 // P = Qd Ki^T on the two matrix warps in parallel (16x16 tiles are far below
 // the smallest tcgen05 tile, so these use warp-level MMA); the 16x16
 // unit-lower solve in fp32 on one warp; W = Tb Kd split over the two matrix
@@ -167,6 +168,8 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int H = p.H;
     const int nchunks = (len + 15) / 16;
+    // decay and matrix warps alternate over the warp slots (plain kernels)
+    constexpr bool kInterleave = !L2N && !EXT;
 
     // ---- set-up: TMEM columns and the two MMA-completion barriers
     if (warp == 0) {
@@ -452,14 +455,16 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
             }
         }
         if (active && !ok && lane == 0 && p.err) atomicOr(p.err, 1);
-    } else if (((warp - 4 * NWG) & 1) == 0) {
+    } else if (kInterleave ? ((warp - 4 * NWG) & 1) == 0 : warp < 4 * NWG + 2) {
         // ------------------------------------------------------------ decay pair
-        // The first and third warp after the state warps (their warp slots put
-        // them on two different SM sub-partitions, each shared with a matrix
-        // warp rather than with the other decay warp): thread d owns the
-        // key-channel pair (ip, ip + 1) on all 16 rows of a chunk; it runs up
-        // to kRaw chunks ahead of the matrix pair.
-        const int dw = (warp - 4 * NWG) >> 1, d = 32 * dw + lane, ip = 2 * d;
+        // In the plain kernels the first and third warp after the state warps
+        // (their warp slots put them on two different SM sub-partitions, each
+        // shared with a matrix warp); in the heavier variants, whose decay
+        // work is longer, the first two (measured faster there).  Thread d
+        // owns the key-channel pair (ip, ip + 1) on all 16 rows of a chunk; it
+        // runs up to kRaw chunks ahead of the matrix pair.
+        const int d = kInterleave ? 32 * ((warp - 4 * NWG) >> 1) + lane : tid - 128 * NWG;
+        const int dw = d >> 5, ip = 2 * d;
         const bf16 *v = (const bf16 *)p.v, *beta = (const bf16 *)p.beta;
         typename Lay::Prep &pr = sm.pr;
         // beta of chunks c and c + 1 (threads d < 16), kept as raw bf16 bits so
@@ -647,9 +652,10 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
         for (int c = max(nchunks - kStages, 0); c < nchunks; ++c) bar_sync(BAR_EMPTY + c % kStages, kBarCount);
     } else {
         // ----------------------------------------------------------- matrix pair
-        // The second and fourth warp after the state warps: the Gram matrices,
-        // the unit-lower solve, W, and the TMA loads of q, k, g (thread 0).
-        const int mw = (warp - 4 * NWG) >> 1, m = 32 * mw + lane;
+        // The other two warps after the state warps: the Gram matrices, the
+        // unit-lower solve, W, and the TMA loads of q, k, g (thread 0).
+        const int m = kInterleave ? 32 * ((warp - 4 * NWG) >> 1) + lane : tid - 128 * NWG - kPair;
+        const int mw = m >> 5;
         typename Lay::Prep &pr = sm.pr;
         auto issue_raw = [&](int c) {
             typename Lay::Raw &R = sm.raw[c % kRaw];
