@@ -93,6 +93,15 @@ size_t kda_chunk_fwd_workspace_size(int32_t total_tokens, int32_t num_seqs, int3
 int kda_chunk_fwd_plan(int32_t total_tokens, int32_t num_seqs, int32_t H, int32_t *piece_len,
                        int32_t *max_pieces, int32_t *launches);
 
+/* Sub-pieces of the same plan (bf16, dk = dv = 128, the 16-token tcgen05
+ * kernels): the summary pass cuts every piece that has a successor into this
+ * many equal parts, summarised by separate CTAs so that the pass's waves fill
+ * the GPU, and composes their affine maps into the piece's before the scan
+ * (the piece states of the prefix scan, Kimi K3 report explainer, affta.cn,
+ * section "KDA 上下文并行，让上下文的交接变薄", at two levels).  1 = none.
+ * Returns the count (>= 1) or KDA_ERR_INVALID_ARG. */
+int32_t kda_chunk_fwd_sub_pieces(int32_t total_tokens, int32_t num_seqs, int32_t H);
+
 /*
  * Prefill: the layer over packed variable-length sequences, computed in
  * 16-token chunks (within a chunk by whole-block matrix products, between

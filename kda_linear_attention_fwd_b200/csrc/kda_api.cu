@@ -17,6 +17,7 @@ cudaError_t launch_decode(bool bf16, int dk, int dv, const void *q, const void *
 cudaError_t launch_plan(const int32_t *cu, int num_seqs, int total_tokens, int piece_len, int P_max,
                         int32_t *header, int32_t *seq_first, int4 *pieces, cudaStream_t st);
 cudaError_t launch_scan(const PrefillParams &p, int dk, int dv, cudaStream_t st);
+cudaError_t launch_subfold_tc(const SubFoldParams &p, int32_t *err, cudaStream_t st);
 cudaError_t launch_prefill_chunks(const PrefillParams &p, bool bf16, int dk, int dv,
                                   bool summaries, cudaStream_t st);
 
@@ -68,14 +69,29 @@ int sm_count() {
     return cache[dev];
 }
 
-int choose_piece_len(long total_tokens, int num_seqs, int H, bool c32,
-                     const int32_t *cu_host = nullptr) {
-    const kda::PlanModel pm = c32 ? kda::plan_model_chunk32(sm_count()) : kda::plan_model_chunk16(sm_count());
-    return kda::plan_piece_len(total_tokens, num_seqs, H, pm, cu_host);
+enum class Path { chunk16, tc5, chunk32 };  // kernel families with their own plans
+
+// The plan of a call on one kernel family: sub-pieces only for the 16-token
+// tcgen05 kernels.
+kda::PlanChoice choose_plan(long total_tokens, int num_seqs, int H, Path path,
+                            const int32_t *cu_host = nullptr) {
+    kda::PlanModel pm = path == Path::chunk32 ? kda::plan_model_chunk32(sm_count())
+                                              : kda::plan_model_chunk16(sm_count());
+    if (path != Path::tc5) pm.sub_max = 1;
+    kda::PlanChoice c = kda::plan_choose(total_tokens, num_seqs, H, pm, cu_host);
+    if (c.sub > 1 && total_tokens <= c.piece_len) c.sub = 1;  // one piece per sequence: nothing to fold
+    return c;
 }
 
-long max_pieces(long total_tokens, int num_seqs, int piece_len) {
-    return (long)num_seqs + (total_tokens + piece_len - 1) / piece_len;
+long max_pieces(long total_tokens, int num_seqs, long piece_len) {
+    return kda::max_pieces_of(total_tokens, num_seqs, piece_len);
+}
+
+kda::WorkspaceLayout layout_of(const kda::PlanChoice &c, long total_tokens, int num_seqs, int H, int dk,
+                               int dv) {
+    const long P = max_pieces(total_tokens, num_seqs, c.piece_len);
+    const long Ps = c.sub > 1 ? max_pieces(total_tokens, num_seqs, c.piece_len / c.sub) : 0;
+    return kda::workspace_layout(P, num_seqs, H, dk, dv, Ps);
 }
 
 }  // namespace
@@ -99,22 +115,37 @@ size_t kda_chunk_fwd_workspace_size(int32_t total_tokens, int32_t num_seqs, int3
                                     int32_t dv, kda_dtype dtype) {
     if (total_tokens < 0 || num_seqs < 0 || H < 1 || !dim_ok(dk) || !dim_ok(dv)) return 0;
     if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return 0;
-    // enough for either plan (the extended features run in 16-token chunks)
-    long P = max_pieces(total_tokens, num_seqs, choose_piece_len(total_tokens, num_seqs, H, false));
-    if (dtype == KDA_DTYPE_BF16 && dk == 128 && dv == 128)
-        P = std::max(P, max_pieces(total_tokens, num_seqs, choose_piece_len(total_tokens, num_seqs, H, true)));
-    return kda::workspace_layout(P, num_seqs, H, dk, dv).total;
+    // enough for the plan of every kernel family the call may run (the
+    // extended features and forced paths change the family)
+    size_t total = layout_of(choose_plan(total_tokens, num_seqs, H, Path::chunk16), total_tokens, num_seqs, H,
+                             dk, dv).total;
+    if (dtype == KDA_DTYPE_BF16 && dk == 128 && dv == 128) {
+        for (Path path : {Path::tc5, Path::chunk32})
+            total = std::max(total, layout_of(choose_plan(total_tokens, num_seqs, H, path), total_tokens, num_seqs,
+                                              H, dk, dv).total);
+    }
+    return total;
 }
 
 int kda_chunk_fwd_plan(int32_t total_tokens, int32_t num_seqs, int32_t H, int32_t *piece_len,
                        int32_t *max_pieces_out, int32_t *launches) {
     if (total_tokens < 0 || num_seqs < 0 || H < 1) return KDA_ERR_INVALID_ARG;
-    const int L = choose_piece_len(total_tokens, num_seqs, H, kda::prefill_impl_forced() == 1);
+    const int f = kda::prefill_impl_forced();
+    const kda::PlanChoice c = choose_plan(total_tokens, num_seqs, H,
+                                          f == 1 ? Path::chunk32 : (f == 3 || f == 4 ? Path::chunk16 : Path::tc5));
+    const long L = c.piece_len;
     const long P = max_pieces(total_tokens, num_seqs, L);
-    if (piece_len) *piece_len = L;
+    if (piece_len) *piece_len = (int32_t)L;
     if (max_pieces_out) *max_pieces_out = (int32_t)(P > 0x7fffffffL ? 0x7fffffffL : P);
-    if (launches) *launches = num_seqs == 0 ? 0 : (total_tokens > L ? 4 : 2);
+    if (launches) *launches = num_seqs == 0 ? 0 : (total_tokens > L ? (c.sub > 1 ? 6 : 4) : 2);
     return KDA_OK;
+}
+
+int32_t kda_chunk_fwd_sub_pieces(int32_t total_tokens, int32_t num_seqs, int32_t H) {
+    if (total_tokens < 0 || num_seqs < 0 || H < 1) return KDA_ERR_INVALID_ARG;
+    const int f = kda::prefill_impl_forced();
+    if (f == 1 || f == 3 || f == 4) return 1;
+    return choose_plan(total_tokens, num_seqs, H, Path::tc5).sub;
 }
 
 int kda_chunk_fwd_ex(const void *q, const void *k, const void *v, const void *g, const void *beta,
@@ -138,13 +169,20 @@ int kda_chunk_fwd_ex(const void *q, const void *k, const void *v, const void *g,
                                     total_tokens, H, dk, dv, dtype, initial_state, final_state, workspace,
                                     &empty);
     if (rc != KDA_OK || empty) return rc;
-    // the piece length with the real lengths, when known, is never shorter
+    // the plan with the real lengths, when known, never needs more workspace
     // than the length-blind one the workspace was sized for
-    const bool c32 = kda::chunk32_eligible(dtype == KDA_DTYPE_BF16, dk, dv, flags, snapshot_tokens);
-    const int L = choose_piece_len(total_tokens, num_seqs, H, c32, cu_seqlens_host);
+    const bool bf16 = dtype == KDA_DTYPE_BF16;
+    const Path path = kda::chunk32_eligible(bf16, dk, dv, flags, snapshot_tokens)
+                          ? Path::chunk32
+                          : (kda::tc5_path(bf16, dk, dv, flags, snapshot_tokens) ? Path::tc5 : Path::chunk16);
+    const kda::PlanChoice plan = choose_plan(total_tokens, num_seqs, H, path, cu_seqlens_host);
+    const long L = plan.piece_len;
+    const int sub = plan.sub;
     const long P_max = max_pieces(total_tokens, num_seqs, L);
-    if (P_max > (1L << 30) || (long)H * P_max > (1L << 31)) return KDA_ERR_UNSUPPORTED;
-    const kda::WorkspaceLayout WL = kda::workspace_layout(P_max, num_seqs, H, dk, dv);
+    const long P_sub_max = sub > 1 ? max_pieces(total_tokens, num_seqs, L / sub) : 0;
+    if (L > (1L << 30) || P_max > (1L << 30) || (long)H * P_max > (1L << 31) || (long)H * P_sub_max > (1L << 31))
+        return KDA_ERR_UNSUPPORTED;
+    const kda::WorkspaceLayout WL = kda::workspace_layout(P_max, num_seqs, H, dk, dv, P_sub_max);
     if (!workspace || workspace_bytes < WL.total) return KDA_ERR_WORKSPACE;
 
     char *ws = (char *)workspace;
@@ -169,24 +207,54 @@ int kda_chunk_fwd_ex(const void *q, const void *k, const void *v, const void *g,
     p.snap_tokens = snapshot_tokens;
     p.snapshots = snapshot_tokens > 0 ? snapshots : nullptr;
     p.snap_offsets = snapshot_tokens > 0 ? snapshot_offsets : nullptr;
-    p.piece_len = L;
+    p.piece_len = (int)L;
 
-    const bool bf16 = dtype == KDA_DTYPE_BF16;
-    cudaError_t e = kda::launch_plan(cu_seqlens, num_seqs, total_tokens, L, (int)P_max,
+    cudaError_t e = kda::launch_plan(cu_seqlens, num_seqs, total_tokens, (int)L, (int)P_max,
                                      (int32_t *)(ws + WL.off_header),
                                      (int32_t *)(ws + WL.off_seq_first),
                                      (int4 *)(ws + WL.off_pieces), stream);
     if (e != cudaSuccess) return KDA_ERR_CUDA;
+    const bool multi = total_tokens > L;  // some sequence may have >1 piece
+    // the summary pass over sub-pieces: its own plan tables and maps
+    kda::PrefillParams ps = p;
+    if (multi && sub > 1) {
+        e = kda::launch_plan(cu_seqlens, num_seqs, total_tokens, (int)(L / sub), (int)P_sub_max,
+                             (int32_t *)(ws + WL.off_header_sub), (int32_t *)(ws + WL.off_seq_first_sub),
+                             (int4 *)(ws + WL.off_pieces_sub), stream);
+        if (e != cudaSuccess) return KDA_ERR_CUDA;
+        ps.seq_first = (const int32_t *)(ws + WL.off_seq_first_sub);
+        ps.pieces = (const int4 *)(ws + WL.off_pieces_sub);
+        ps.M = (float *)(ws + WL.off_M_sub);
+        ps.Szero = (float *)(ws + WL.off_Szero_sub);
+        ps.P_max = (int)P_sub_max;
+        ps.piece_len = (int)(L / sub);
+        ps.sub = sub;
+    }
 #ifdef KDA_CHECK_G
-    // after the plan kernel, which clears the error word
+    // after the plan kernels, which clear the error word
     e = kda::launch_check_g(g, bf16, (long)total_tokens * H * dk, (flags & kda::FLAG_CLAMP_G) ? 1 : 0,
                             p.err, stream);
     if (e != cudaSuccess) return KDA_ERR_CUDA;
 #endif
-    const bool multi = total_tokens > L;  // some sequence may have >1 piece
     if (multi) {
-        e = kda::launch_prefill_chunks(p, bf16, dk, dv, true, stream);
+        e = kda::launch_prefill_chunks(ps, bf16, dk, dv, true, stream);
         if (e != cudaSuccess) return KDA_ERR_CUDA;
+        if (sub > 1) {
+            kda::SubFoldParams f{};
+            f.pieces = p.pieces;
+            f.seq_first = p.seq_first;
+            f.seq_first_sub = ps.seq_first;
+            f.M_sub = ps.M;
+            f.Z_sub = ps.Szero;
+            f.M = p.M;
+            f.Z = p.Szero;
+            f.H = H;
+            f.P_max = (int)P_max;
+            f.P_sub_max = (int)P_sub_max;
+            f.sub = sub;
+            e = kda::launch_subfold_tc(f, p.err, stream);
+            if (e != cudaSuccess) return KDA_ERR_CUDA;
+        }
         e = kda::launch_scan(p, dk, dv, stream);
         if (e != cudaSuccess) return KDA_ERR_CUDA;
     }

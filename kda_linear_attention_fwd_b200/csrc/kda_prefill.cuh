@@ -21,6 +21,11 @@
 //   scan     -> incoming state of every piece (sequences with >1 piece)
 //   output   -> every piece from its incoming state: y, and the final state
 // When no sequence can have more than one piece, only plan and output run.
+// With sub-pieces (the 16-token tcgen05 kernels, when the plan asks for
+// them) the summary runs over pieces cut into `sub` equal parts, which fills
+// the summary pass's waves better, and a fold composes each piece's sub-piece
+// maps into the piece's (M, S_zero) before the scan:
+//   plan, plan of the sub-pieces, summary (sub-pieces), fold, scan, output.
 #pragma once
 
 #include <stdint.h>
@@ -40,13 +45,16 @@ constexpr int kChunk = 16;
 //   fp32  M           [P_max][H][dk][dk]   transition of each piece
 //   fp32  Szero       [P_max][H][dk][dv]   state each piece makes from zero
 //   fp32  Sin         [P_max][H][dk][dv]   incoming state of each piece
+// and, with sub-pieces (P_sub_max > 0), the same plan sections and the two
+// maps once more for the sub-pieces.
 struct WorkspaceLayout {
-    size_t off_header, off_seq_first, off_pieces, off_M, off_Szero, off_Sin, total;
+    size_t off_header, off_seq_first, off_pieces, off_M, off_Szero, off_Sin;
+    size_t off_header_sub, off_seq_first_sub, off_pieces_sub, off_M_sub, off_Szero_sub, total;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-inline WorkspaceLayout workspace_layout(long P_max, int num_seqs, int H, int dk, int dv) {
+inline WorkspaceLayout workspace_layout(long P_max, int num_seqs, int H, int dk, int dv, long P_sub_max = 0) {
     WorkspaceLayout L;
     size_t o = 0;
     L.off_header = o;    o = align256(o + 64 * sizeof(int32_t));
@@ -55,6 +63,14 @@ inline WorkspaceLayout workspace_layout(long P_max, int num_seqs, int H, int dk,
     L.off_M = o;         o = align256(o + (size_t)P_max * H * dk * dk * sizeof(float));
     L.off_Szero = o;     o = align256(o + (size_t)P_max * H * dk * dv * sizeof(float));
     L.off_Sin = o;       o = align256(o + (size_t)P_max * H * dk * dv * sizeof(float));
+    L.off_header_sub = L.off_seq_first_sub = L.off_pieces_sub = L.off_M_sub = L.off_Szero_sub = o;
+    if (P_sub_max > 0) {
+        L.off_header_sub = o;    o = align256(o + 64 * sizeof(int32_t));
+        L.off_seq_first_sub = o; o = align256(o + (size_t)(num_seqs + 1) * sizeof(int32_t));
+        L.off_pieces_sub = o;    o = align256(o + (size_t)P_sub_max * 4 * sizeof(int32_t));
+        L.off_M_sub = o;         o = align256(o + (size_t)P_sub_max * H * dk * dk * sizeof(float));
+        L.off_Szero_sub = o;     o = align256(o + (size_t)P_sub_max * H * dk * dv * sizeof(float));
+    }
     L.total = o;
     return L;
 }
@@ -65,30 +81,45 @@ inline WorkspaceLayout workspace_layout(long P_max, int num_seqs, int H, int dk,
 // `slots_out` CTAs.  A sequence of p > 1 pieces costs an output pass over all
 // p pieces, a summary pass over pieces 0..p-2 (one CTA per (piece, head)
 // computes both the zero-start state and the transition; waves of
-// `slots_sum`) and p - 1 steps of the prefix scan.  With equal-length
-// sequences (the lengths are not known on the host in general) the model is
-//   cost(L) = waves(output) * chunks(L) + sum_ratio * waves(summary) * chunks(L)
-//             + scan_cost * (pieces - 1)
+// `slots_sum`) and p - 1 steps of the prefix scan.  With sub-pieces, each
+// summarised piece is cut into `sub` equal parts summarised by separate CTAs
+// (shorter CTAs fill the summary's waves better) and `sub` - 1 fold steps
+// compose their maps.  With equal-length sequences (the lengths are not known
+// on the host in general) the model is
+//   cost(L, sub) = waves(output) * chunks(L)
+//                  + sum_ratio * waves(summary units) * chunks(L) / sub
+//                  + scan_cost * (pieces - 1) + fold_cost * (sub - 1)
 // in units of one chunk step of the output pass.  When the host copy of the
-// offsets is given, the real lengths are used, and only piece lengths at
-// least as long as the length-blind choice are considered, so that the
-// workspace sized without the lengths still fits.
+// offsets is given, the real lengths are used, and only plans whose tables fit
+// the workspace sized for the length-blind choice are considered.
 struct PlanModel {
     int chunk;          // tokens per chunk step (16 or 32); pieces are multiples of it
     long slots_out;     // output-pass CTAs resident at once
     long slots_sum;     // summary-pass CTAs resident at once
     double sum_ratio;   // summary chunk step / output chunk step
     double scan_cost;   // one scan step, in output chunk steps
+    int sub_max;        // most sub-pieces a summarised piece may be cut into (1 = none)
+    double fold_cost;   // one fold step, in output chunk steps
 };
 // The 16-token kernels: output pass two CTAs per SM, the paired summary one;
 // 0.67 is the measured ratio of their per-chunk periods at full occupancy
 // (about 2.96 K and 4.44 K SM cycles), a scan step about two output chunk
-// steps.
-inline PlanModel plan_model_chunk16(int sms) { return PlanModel{16, 2L * sms, (long)sms, 0.67, 2.0}; }
+// steps, a fold step about three.  Sub-pieces are for the tcgen05 kernels
+// only (the caller clears sub_max for the others).
+inline PlanModel plan_model_chunk16(int sms) { return PlanModel{16, 2L * sms, (long)sms, 0.67, 2.0, 4, 3.0}; }
 // The 32-token kernels (bf16, dk = dv = 128): both passes one CTA per SM.
-inline PlanModel plan_model_chunk32(int sms) { return PlanModel{32, (long)sms, (long)sms, 1.0, 6.0}; }
+inline PlanModel plan_model_chunk32(int sms) { return PlanModel{32, (long)sms, (long)sms, 1.0, 6.0, 1, 0.0}; }
 
-inline double plan_cost(long L, int num_seqs, int H, const PlanModel &pm, const int32_t *cu_host,
+struct PlanChoice {
+    long piece_len;
+    int sub;  // sub-pieces per summarised piece (1 = none)
+};
+
+inline long max_pieces_of(long total_tokens, int num_seqs, long piece_len) {
+    return (long)num_seqs + (total_tokens + piece_len - 1) / piece_len;
+}
+
+inline double plan_cost(long L, int sub, int num_seqs, int H, const PlanModel &pm, const int32_t *cu_host,
                         long total_tokens) {
     long out = 0, sum = 0, max_chunks = 0, max_pieces = 1;
     for (int n = 0; n < (cu_host ? num_seqs : 1); ++n) {
@@ -97,7 +128,7 @@ inline double plan_cost(long L, int num_seqs, int H, const PlanModel &pm, const 
         const long pcs = len <= 0 ? 1 : (len + L - 1) / L;
         const long mult = cu_host ? 1 : num_seqs;
         out += mult * pcs;
-        sum += mult * (pcs - 1);
+        sum += mult * (pcs - 1) * sub;
         const long ch = (std::min(len, L) + pm.chunk - 1) / pm.chunk;
         if (ch > max_chunks) max_chunks = ch;
         if (pcs > max_pieces) max_pieces = pcs;
@@ -105,8 +136,9 @@ inline double plan_cost(long L, int num_seqs, int H, const PlanModel &pm, const 
     const long w_out = (out * H + pm.slots_out - 1) / pm.slots_out;
     const long sum_slots = std::max(pm.slots_sum, 1L);
     const long w_sum = (sum * H + sum_slots - 1) / sum_slots;
-    return (double)w_out * max_chunks + pm.sum_ratio * (double)w_sum * max_chunks +
-           pm.scan_cost * (double)(max_pieces - 1);
+    return (double)w_out * max_chunks + pm.sum_ratio * (double)w_sum * (double)((max_chunks + sub - 1) / sub) +
+           pm.scan_cost * (double)(max_pieces - 1) +
+           (sub > 1 && max_pieces > 1 ? pm.fold_cost * (double)(sub - 1) : 0.0);
 }
 
 inline long env_positive(const char *name) {
@@ -117,33 +149,65 @@ inline long env_positive(const char *name) {
     return (end && *end == 0 && v > 0) ? v : 0;
 }
 
-inline int plan_piece_len(long total_tokens, int num_seqs, int H, const PlanModel &pm_in,
-                          const int32_t *cu_host) {
+// KDA_PIECE_LEN forces the piece length (rounded up to whole chunks, and to
+// whole sub-pieces); KDA_SUB_PIECES forces the number of sub-pieces (at most
+// sub_max).
+inline PlanChoice plan_choose(long total_tokens, int num_seqs, int H, const PlanModel &pm_in,
+                              const int32_t *cu_host) {
     const long C = pm_in.chunk;
+    const int sub_max = std::max(pm_in.sub_max, 1);
+    const long forced_sub = std::min<long>(env_positive("KDA_SUB_PIECES"), sub_max);
     const long forced = env_positive("KDA_PIECE_LEN");
-    if (forced > 0) return (int)(((forced + C - 1) / C) * C);
+    if (forced > 0) {
+        const long m = forced_sub > 0 ? forced_sub : 1;
+        return PlanChoice{((forced + C * m - 1) / (C * m)) * C * m, (int)m};
+    }
     PlanModel pm = pm_in;
     if (env_positive("KDA_SLOTS")) pm.slots_out = env_positive("KDA_SLOTS");
-    if (num_seqs <= 0 || total_tokens <= 0) return 256;
-    auto search = [&](const int32_t *cu, long Lref, long L_floor) {
-        long best_L = std::max<long>(((Lref + C - 1) / C) * C, 256);
-        best_L = std::max(best_L, L_floor);
-        double best = plan_cost(best_L, num_seqs, H, pm, cu, total_tokens);
-        for (int pcs = 2; pcs <= 128; ++pcs) {
-            long L = ((Lref + pcs - 1) / pcs + C - 1) / C * C;
-            if (L < 256 || L < L_floor) break;
-            const double c = plan_cost(L, num_seqs, H, pm, cu, total_tokens);
-            if (c < best) { best = c; best_L = L; }
+    if (num_seqs <= 0 || total_tokens <= 0) return PlanChoice{256, 1};
+    // floors: the chosen tables must fit the workspace of the length-blind plan
+    auto search = [&](const int32_t *cu, long Lref, const PlanChoice *floor) {
+        PlanChoice best{0, 1};
+        double best_cost = 0;
+        for (int m = 1; m <= sub_max; m *= 2) {
+            if (forced_sub > 0 && m != forced_sub) continue;
+            if (floor && m > 1 && floor->sub == 1) continue;  // no sub-piece tables in the workspace
+            for (int pcs = 1; pcs <= 128; ++pcs) {
+                long L = ((Lref + pcs - 1) / pcs + C * m - 1) / (C * m) * (C * m);
+                L = std::max<long>(L, ((256 + C * m - 1) / (C * m)) * C * m);
+                if (floor) {
+                    if (L < floor->piece_len) break;
+                    if (m > 1 && L / m < floor->piece_len / floor->sub) break;
+                }
+                const double c = plan_cost(L, m, num_seqs, H, pm, cu, total_tokens);
+                if (best.piece_len == 0 || c < best_cost) {
+                    best = PlanChoice{L, m};
+                    best_cost = c;
+                }
+                if (L <= ((256 + C * m - 1) / (C * m)) * C * m) break;
+            }
         }
-        return best_L;
+        if (best.piece_len == 0) best = floor ? *floor : PlanChoice{std::max<long>(((Lref + C - 1) / C) * C, 256), 1};
+        return best;
     };
     const long Lavg = (total_tokens + num_seqs - 1) / num_seqs;
-    const long L_blind = search(nullptr, Lavg, 0);
+    PlanChoice blind = search(nullptr, Lavg, nullptr);
+    blind.piece_len = std::min<long>(blind.piece_len, 1L << 30);
     // the exact model walks every sequence per candidate: only for modest N
-    if (!cu_host || num_seqs > 8192) return (int)std::min<long>(L_blind, 1L << 30);
+    if (!cu_host || num_seqs > 8192) return blind;
     long Lmax = 0;
     for (int n = 0; n < num_seqs; ++n) Lmax = std::max<long>(Lmax, (long)cu_host[n + 1] - cu_host[n]);
-    return (int)std::min<long>(search(cu_host, std::max(Lmax, L_blind), L_blind), 1L << 30);
+    PlanChoice c = search(cu_host, std::max(Lmax, blind.piece_len), &blind);
+    c.piece_len = std::min<long>(c.piece_len, 1L << 30);
+    return c;
+}
+
+// The plan without sub-pieces (callers whose kernels do not take them).
+inline int plan_piece_len(long total_tokens, int num_seqs, int H, const PlanModel &pm_in,
+                          const int32_t *cu_host) {
+    PlanModel pm = pm_in;
+    pm.sub_max = 1;
+    return (int)plan_choose(total_tokens, num_seqs, H, pm, cu_host).piece_len;
 }
 
 struct PrefillParams {
@@ -172,6 +236,20 @@ struct PrefillParams {
     int summarize_all;
     // piece length of the plan (tokens): the 32-token kernels need a multiple of 32
     int piece_len;
+    // summary launches over sub-pieces: the pieces table holds sub-pieces,
+    // `sub` of them per piece of the output pass (0 or 1 = plain pieces)
+    int sub;
+};
+
+// The fold of sub-piece maps into piece maps (plans with sub-pieces): the
+// output pass's piece table and the sub-piece table in, the sub-piece maps
+// in, the piece maps (what the scan reads) out.
+struct SubFoldParams {
+    const int4 *pieces;
+    const int32_t *seq_first, *seq_first_sub;
+    const float *M_sub, *Z_sub;
+    float *M, *Z;
+    int H, P_max, P_sub_max, sub;
 };
 
 // The 32-token kernels (bf16, dk = dv = 128, none of the extended features)
@@ -191,6 +269,12 @@ inline int prefill_impl_forced() {
 inline bool chunk32_eligible(bool bf16, int dk, int dv, int flags, int snap_tokens) {
     const int f = prefill_impl_forced();
     return bf16 && dk == 128 && dv == 128 && flags == 0 && snap_tokens == 0 && f == 1;
+}
+// The call runs the 16-token tcgen05 kernels (the only ones that summarise
+// sub-pieces).
+inline bool tc5_path(bool bf16, int dk, int dv, int flags, int snap_tokens) {
+    const int f = prefill_impl_forced();
+    return bf16 && dk == 128 && dv == 128 && f != 3 && f != 4 && !chunk32_eligible(bf16, dk, dv, flags, snap_tokens);
 }
 
 // Where the output pass of one (piece, head) writes state snapshots.

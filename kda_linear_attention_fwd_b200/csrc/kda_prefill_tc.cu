@@ -804,7 +804,8 @@ __device__ void run_piece(const PrefillParams &p, const TmaMaps &maps, int t0, i
 // first piece) into S_zero, warpgroup 1 runs it from the identity without v
 // into the transition M; both share one preparation of every chunk.  A part
 // the scan does not need (both maps of a sequence's last piece, M of its
-// first) is skipped unless every piece's map is asked for.
+// first) is skipped unless every piece's map is asked for.  The same holds
+// for sub-pieces, piece by piece of the output pass.
 template <int DK, bool L2N, bool EXT>
 __global__ void __launch_bounds__(kThreadsOf<2>, 1)
     summary_kernel(PrefillParams p, const __grid_constant__ TmaMaps maps) {
@@ -815,9 +816,15 @@ __global__ void __launch_bounds__(kThreadsOf<2>, 1)
     const int4 pc = p.pieces[pi];
     if (pc.x < 0) return;
     const int n = pc.x, j = pc.w;
+    // with sub-pieces, j counts sub-pieces and `sub` of them make one piece of
+    // the output pass; a (sub-)piece is summarised when the output piece it
+    // lies in has a successor, its transition too unless it starts the
+    // sequence (the fold composes the sub-piece maps of each piece)
+    const int sub = p.sub > 1 ? p.sub : 1;
     const int np = p.seq_first[n + 1] - p.seq_first[n];
-    const bool want_s = p.summarize_all || j < np - 1;
-    const bool want_m = p.summarize_all || (j > 0 && j < np - 1);
+    const bool needed = j / sub < (np + sub - 1) / sub - 1;
+    const bool want_s = p.summarize_all || needed;
+    const bool want_m = p.summarize_all || (needed && j > 0);
     if (!want_s && !want_m) return;
     const size_t ph = (size_t)pi * p.H + h;
     const float *init = (j == 0 && p.initial_state)

@@ -24,7 +24,7 @@ EXPORTS = ("kda_status_string", "kda_chunk_fwd_workspace_size", "kda_chunk_fwd_p
            "kda_chunk_fwd", "kda_decode_step", "kda_chunk_fwd_ex", "kda_decode_step_ex",
            "kda_chunk_fwd_summary", "kda_state_compose", "kda_bwd_workspace_size", "kda_bwd",
            "kda_chunk_fwd_check", "kda_build_checks_g", "kda_chunk_fwd_noalloc",
-           "kda_chunk_fwd_noalloc_check")
+           "kda_chunk_fwd_noalloc_check", "kda_chunk_fwd_sub_pieces")
 
 # flags of the extended entry points (include/kda.h)
 FLAG_QK_L2NORM, FLAG_BETA_LOGITS, FLAG_GATE_LOGITS, FLAG_CLAMP_DECAY = 1, 2, 4, 8
@@ -70,6 +70,8 @@ def _open(path):
     lib.kda_chunk_fwd_workspace_size.restype = sz
     lib.kda_chunk_fwd_plan.argtypes = [i32, i32, i32, P, P, P]
     lib.kda_chunk_fwd_plan.restype = ctypes.c_int
+    lib.kda_chunk_fwd_sub_pieces.argtypes = [i32, i32, i32]
+    lib.kda_chunk_fwd_sub_pieces.restype = ctypes.c_int32
     lib.kda_chunk_fwd.argtypes = [P, P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32,
                                   ctypes.c_int, f32, i32, P, P, P, sz, P]
     lib.kda_chunk_fwd.restype = ctypes.c_int
@@ -142,11 +144,16 @@ def workspace_size(total_tokens, num_seqs, H, dk, dv, dtype=torch.bfloat16) -> i
 
 
 def plan(total_tokens, num_seqs, H) -> dict:
-    """Piece length, piece bound and launch count of one kda_chunk_fwd call."""
+    """Piece length, piece bound, launch count and sub-pieces of one
+    kda_chunk_fwd call (bf16, dk = dv = 128)."""
     L, P, n = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
-    _check("kda_chunk_fwd_plan", load().kda_chunk_fwd_plan(
+    lib = load()
+    _check("kda_chunk_fwd_plan", lib.kda_chunk_fwd_plan(
         total_tokens, num_seqs, H, ctypes.byref(L), ctypes.byref(P), ctypes.byref(n)))
-    return dict(piece_len=L.value, max_pieces=P.value, launches=n.value)
+    sub = int(lib.kda_chunk_fwd_sub_pieces(total_tokens, num_seqs, H))
+    if sub < 1:
+        _check("kda_chunk_fwd_sub_pieces", sub)
+    return dict(piece_len=L.value, max_pieces=P.value, launches=n.value, sub_pieces=sub)
 
 
 def _flags(qk_l2norm, beta_logits, gate_logits, clamp_decay):

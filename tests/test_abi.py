@@ -252,15 +252,19 @@ def test_chunk_fwd_check_validation(lib):
 def test_plan_choices_on_148_sms(lib, monkeypatch):
     """The piece plan's cost model on a 148-SM device (without a device the
     library assumes 148 SMs).  Default (16-token kernels): waves of the output
-    pass at two CTAs per SM and of the paired summary pass at one, plus scan
-    steps.  With the 32-token kernels (KDA_PREFILL_IMPL=c32): both passes one
+    pass at two CTAs per SM and of the paired summary pass at one -- over
+    sub-pieces where they fill its waves better -- plus scan and fold steps.
+    With the 32-token kernels (KDA_PREFILL_IMPL=c32): both passes one
     CTA per SM, pieces a multiple of 32 tokens."""
     import torch
     if torch.cuda.is_available() and torch.cuda.get_device_properties(0).multi_processor_count != 148:
         pytest.skip("plan depends on the SM count")
-    assert kda.plan(131072, 1, 32)["piece_len"] == 14576  # 9 pieces per head: 288 CTAs, one wave
-    assert kda.plan(8192, 2, 16)["piece_len"] == 464      # 9 pieces per sequence
-    assert kda.plan(256, 1, 2) == {"piece_len": 256, "max_pieces": 2, "launches": 2}  # one piece
+    long = kda.plan(131072, 1, 32)  # 9 pieces per head: 288 output CTAs, one wave; summary over
+    assert (long["piece_len"], long["sub_pieces"], long["launches"]) == (14592, 4, 6)  # 4 sub-pieces each
+    assert kda.plan(8192, 2, 16)["piece_len"] == 464      # 9 pieces per sequence, no sub-pieces
+    assert kda.plan(8192, 2, 16)["sub_pieces"] == 1
+    assert kda.plan(256, 1, 2) == {"piece_len": 256, "max_pieces": 2, "launches": 2,
+                                   "sub_pieces": 1}  # one piece
     monkeypatch.setenv("KDA_PREFILL_IMPL", "c32")
     assert kda.plan(131072, 1, 32)["piece_len"] == 14592  # 9 pieces per head: 288 CTAs, 2 waves
     assert kda.plan(8192, 2, 16)["piece_len"] == 1024     # 4 pieces per sequence

@@ -150,6 +150,36 @@ def test_length_blind_plan_bf16_128_matches_oracle(cuda_lib):
     compare(inp, y, S, yr, Sr, "bf16", heads=heads, what="length-blind plan")
 
 
+SUB_CASES = [
+    # lengths, forced piece length, sub-pieces per summarised piece
+    ((3000, 700, 1, 1500), 512, 2),
+    ((4111, 300, 0, 2049), 1024, 4),
+    ((2600,), 768, 3),
+]
+
+
+@pytest.mark.parametrize("case", SUB_CASES, ids=[f"p{c[1]}-sub{c[2]}" for c in SUB_CASES])
+def test_sub_pieces_match_oracle(cuda_lib, monkeypatch, case):
+    """bf16, dk = dv = 128 with the summary pass over sub-pieces and the fold
+    of their maps (forced plans: several pieces per sequence, partial last
+    pieces, an empty and a one-token sequence, initial states): y and the
+    final states against the oracle, identical with and without the host
+    copy of the offsets."""
+    lengths, piece, sub = case
+    monkeypatch.setenv("KDA_PIECE_LEN", str(piece))
+    monkeypatch.setenv("KDA_SUB_PIECES", str(sub))
+    T, N, H = sum(lengths), len(lengths), 3
+    assert kda.plan(T, N, H)["sub_pieces"] == sub
+    w = W.custom(dtype="bf16", H=H, dk=128, dv=128, lengths=lengths, init_state=True,
+                 seed=700 + SUB_CASES.index(case))
+    inp = W.pack_prefill(w, device="cuda")
+    y1, S1 = run(inp, host_cu=True)
+    y2, S2 = run(inp, host_cu=False)
+    assert np.array_equal(y1, y2) and np.array_equal(S1, S2)
+    yr, Sr = oracle_prefill(inp)
+    compare(inp, y1, S1, yr, Sr, "bf16", what=f"sub-pieces {case}")
+
+
 def test_beta_zero_closed_form(cuda_lib):
     """beta = 0: o_t = S0^T (q_t exp(G_t)), S_L = Diag(exp G_L) S0 -- checked
     against the closed form itself, not the oracle."""
