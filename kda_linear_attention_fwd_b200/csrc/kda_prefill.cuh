@@ -104,9 +104,11 @@ struct PlanModel {
 // The 16-token kernels: output pass two CTAs per SM, the paired summary one;
 // 0.67 is the measured ratio of their per-chunk periods at full occupancy
 // (about 2.96 K and 4.44 K SM cycles), a scan step about two output chunk
-// steps, a fold step about three.  Sub-pieces are for the tcgen05 kernels
-// only (the caller clears sub_max for the others).
-inline PlanModel plan_model_chunk16(int sms) { return PlanModel{16, 2L * sms, (long)sms, 0.67, 2.0, 4, 3.0}; }
+// steps, a fold step about thirteen (measured: 87 us for the three steps of
+// 256 piece-head chains, one output chunk step being about 2.2 us).
+// Sub-pieces are for the tcgen05 kernels only (the caller clears sub_max for
+// the others).
+inline PlanModel plan_model_chunk16(int sms) { return PlanModel{16, 2L * sms, (long)sms, 0.67, 2.0, 4, 13.0}; }
 // The 32-token kernels (bf16, dk = dv = 128): both passes one CTA per SM.
 inline PlanModel plan_model_chunk32(int sms) { return PlanModel{32, (long)sms, (long)sms, 1.0, 6.0, 1, 0.0}; }
 
