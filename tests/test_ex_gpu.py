@@ -51,11 +51,15 @@ def _preprocessed(inp):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("bf16", 64), ("f32", 64)])
-def test_prefill_preprocessing_flags(cuda_lib, dtype, d):
+@pytest.mark.parametrize("dtype,d,piece,sub", [("bf16", 128, None, None), ("bf16", 64, None, None),
+                                              ("f32", 64, None, None), ("bf16", 128, 128, 4)])
+def test_prefill_preprocessing_flags(cuda_lib, monkeypatch, dtype, d, piece, sub):
     """beta and gate as logits, g clamped at the floor, q/k normalised in the
     kernel (bf16 d=128: tcgen05 kernel; bf16 d=64: warp-MMA kernel; fp32: CUDA
-    cores)."""
+    cores); the last case on a forced plan whose summary runs over sub-pieces."""
+    if piece:
+        monkeypatch.setenv("KDA_PIECE_LEN", str(piece))
+        monkeypatch.setenv("KDA_SUB_PIECES", str(sub))
     w = W.custom(dtype=dtype, H=2, dk=d, dv=d, lengths=(37, 300), init_state=True, seed=41)
     inp = _logit_inputs(W.pack_prefill(w, device="cuda"), dtype, seed=42)
     cu = inp["cu_seqlens"].tolist()
@@ -121,13 +125,17 @@ def _snapshot_refs(inp, B):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("dtype,d,piece", [("bf16", 128, None), ("bf16", 128, 256),
-                                            ("bf16", 64, 256), ("f32", 64, 256)])
-def test_snapshots(cuda_lib, monkeypatch, dtype, d, piece):
+@pytest.mark.parametrize("dtype,d,piece,sub", [("bf16", 128, None, None), ("bf16", 128, 256, None),
+                                                ("bf16", 64, 256, None), ("f32", 64, 256, None),
+                                                ("bf16", 128, 256, 2)])
+def test_snapshots(cuda_lib, monkeypatch, dtype, d, piece, sub):
     """State snapshots every 64 tokens: single-piece and forced multi-piece
-    plans (the snapshots of later pieces start from the scanned state)."""
+    plans (the snapshots of later pieces start from the scanned state), one of
+    them with the summary over sub-pieces."""
     if piece:
         monkeypatch.setenv("KDA_PIECE_LEN", str(piece))
+    if sub:
+        monkeypatch.setenv("KDA_SUB_PIECES", str(sub))
     B = 64
     w = W.custom(dtype=dtype, H=2, dk=d, dv=d, lengths=(0, 5, 64, 300, 701), init_state=True,
                  seed=61)
@@ -143,9 +151,8 @@ def test_snapshots(cuda_lib, monkeypatch, dtype, d, piece):
     assert snaps.shape[0] == ref.shape[0] == offs[-1]
     assert_close(np32(snaps), ref, dtype, "snapshots")
     # the plain outputs are unchanged by asking for snapshots: the same call
-    # without them on the kernels that take snapshots (for bf16 128 x 128
-    # plain calls otherwise run the 32-token kernels, which round differently)
-    # is bit-identical, and both match the oracle
+    # without them, on the same 16-token kernels (the ones that take
+    # snapshots), is bit-identical, and both match the oracle
     if dtype == "bf16" and d == 128:
         monkeypatch.setenv("KDA_PREFILL_IMPL", "tc5")
     y2, S2 = kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["gate"],
