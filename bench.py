@@ -520,9 +520,10 @@ def main():
                             "fp32 gradients, final-state gradient given",
                 "roofline": {"bound": "hbm", "achieved": bgbs, "peak": hbm, "unit": "GB/s",
                              "frac": bgbs / hbm, "traffic": None,
-                             "kernel": "bwd_kernel<128,bf16> (checkpointed reverse recurrence)",
+                             "kernel": "kda_bwd call (prep, forward chain, reverse chain, "
+                                       "per-chunk gradients)",
                              "peak_source": f"{pk_kind} hbm_gbs"},
-                "gpu_launches": args.steps}
+                "gpu_launches": 4 * args.steps}
         del bi, dyb, dsfb, gq, gk, gg, gv, ggt, gbt, gs0, wsb
 
     # ---------------- decode ----------------

@@ -311,14 +311,19 @@ int kda_state_compose(const float *transitions, const float *zero_states, int32_
  *   L = sum dy (.) y + sum d_final_state (.) final_state.
  * The pages state the forward only (Kimi K3 report explainer, affta.cn,
  * section "第一关：KDA 解决算得动": forget, corrective write with an update
- * strength, read, output gate); this is that recurrence differentiated by the
- * chain rule, token by token in reverse, with the states recomputed from
- * checkpoints every 16 tokens.  fp32 arithmetic; results are deterministic up
- * to the order of fp32 atomic additions across 8-column slices of dv.
+ * strength, read, output gate); this is its 16-token chunk form
+ * (prism.simon-ai.net, section "计算范式演进：从递归低效到 GPU 友好的 Chunk
+ * Recurrent") differentiated by the chain rule: per-chunk operands in
+ * parallel, a forward pass over the chunks storing the state entering each,
+ * a reverse pass carrying dL/dS, then the per-chunk gradients in parallel
+ * (four launches on `stream`).  fp32 arithmetic; every output element is
+ * written once, so results are deterministic.
  *
  * kda_bwd_workspace_size: bytes of workspace kda_bwd needs (0 for
- *   unsupported sizes): checkpoints ((total_tokens / 16 + num_seqs) * H * dk
- *   * dv floats) plus per-(sequence, head, 8 columns) scratch of 16 states.
+ *   unsupported sizes).  With ch = (total_tokens / 16 + num_seqs) * H chunk
+ *   slots: ch * (49 dk + 16 dv + 256 + 2 dk dv + 32 dv) floats (per-chunk
+ *   operands, the state entering and dL/d(state leaving) each chunk, U and
+ *   dL/dU), each region rounded up to 256 bytes.
  *
  * kda_bwd:
  *   q, k, g       device [total_tokens][H][dk], dtype; v, gate, dy device

@@ -3,364 +3,676 @@
 //
 // The pages give the forward only (Kimi K3 report explainer, affta.cn,
 // section "第一关：KDA 解决算得动": forget, corrective write with an update
-// strength, read, output gate).  The reverse recurrence is that forward
-// differentiated step by step; per token t, going backwards, with S_{t-1} the
-// state before the token, alpha = exp(g_t) and dS = dL/dS_t:
-//   S' = Diag(alpha) S_{t-1};  a = S'^T k;  u = beta (v - a);  S_t = S' + k u^T
-//   o = S_t^T (scale q);  do = gate (.) dy;  dgate = dy (.) o
-//   dS += scale q do^T;   dq = scale S_t do
-//   du = dS^T k;  dv = beta du;  dbeta = du . (v - a);  da = -beta du
-//   dk = dS u + S' da;  dS' = dS + k da^T;  dg = rowsum(dS' (.) S')
-//   dS <- Diag(alpha) dS'
+// strength, read, output gate).  This is its 16-token chunk form
+// (prism.simon-ai.net, section "计算范式演进：从递归低效到 GPU 友好的 Chunk
+// Recurrent"; the decay as a transform inside a 16-token tile, section
+// "数值稳定性与 Co-Design：BF16 约束下的衰减控制策略") differentiated by the
+// chain rule.  Per chunk of C = 16 rows (rows past a sequence's end are zero,
+// with g = 0), G = the inclusive running sum of g over the chunk's rows,
+// E = exp(G), s = scale, S = the state entering the chunk:
+//   Kd = K (.) E,  Ki = K (.) E^-1,  Qd = s Q (.) E,  Kb = K (.) exp(G_C - G)
+//   A = strict_tril(Kd Ki^T),  P = tril(Qd Ki^T),  X = (I + Diag(beta) A)^-1
+//   T = X Diag(beta),  W = T Kd,  U0 = T V
+//   U = U0 - W S,  O = Qd S + P U,  y = gate (.) O
+//   S' = Diag(gamma_C) S + Kb^T U        (G_C = G of the last row, gamma_C = exp(G_C))
+// Going backwards, with dS' = dL/dS' and dO = gate (.) dy:
+//   dU = P^T dO + Kb dS',   dS = Qd^T dO + Diag(gamma_C) dS' - W^T dU    (the chain)
+//   dQd = dO S^T,  dW = -dU S^T,  dKb = U dS'^T,  dgamma_C = rowsum(dS' (.) S)
+//   dP = tril(dO U^T),  dT = dU V^T + dW Kd^T,  dV = T^T dU,  dKd = T^T dW
+//   M = X^T dT Diag(beta),  dL = -M X^T
+//   dbeta = colsum(X (.) dT) + rowsum(strict(dL) (.) A),  dA = Diag(beta) strict(dL)
+//   dKd += dA Ki,  dKi = dA^T Kd + dP^T Qd,  dQd += dP Ki
+//   dK = dKd (.) E + dKi (.) E^-1 + dKb (.) exp(G_C - G),  dQ = s dQd (.) E
+//   dG = dKd (.) Kd - dKi (.) Ki + dQd (.) Qd - dKb (.) Kb; the last row adds
+//        colsum(dKb (.) Kb) + dgamma_C (.) gamma_C;  dg = suffix sums of dG over the rows
 //
-// Layout of the work: the columns of the state are independent in every step
-// except through the row sums (dq, dk, dg) and dbeta, so one CTA owns one
-// (sequence, head, 8-column slice of dv) and adds its share of those sums
-// into fp32 outputs with atomics; dv, dgate and the initial-state gradient are
-// per column and stored directly.  Thread i (one per key channel) holds row i
-// of the state slice and of dS in registers; sums over the key channels (a, o,
-// du) are a warp reduce-scatter plus a shared-memory combine across warps.
-//
-// States going backwards: a forward sweep stores the state every kBlk tokens
-// (checkpoints); the reverse sweep re-runs each block forwards from its
-// checkpoint, keeping the block's states in per-CTA scratch, then walks the
-// block backwards.  Every state row is written and read back by the thread
-// that owns it.  fp32 throughout; the inputs are bf16 or fp32.
+// Four launches, all fp32 arithmetic on bf16 or fp32 inputs:
+//   prep_kernel   per (chunk, head), parallel: W, Qd, Kb, U0, P, gamma_C -> workspace
+//   fwd_chain     per (sequence, head, 16 state columns), chunks in order: the
+//                 state entering each chunk and U -> workspace; dgate = dy (.) O
+//   rev_chain     per (sequence, head, 16 columns), chunks in reverse: dS' and
+//                 dU -> workspace; dL/d(initial state)
+//   grad_kernel   per (chunk, head), parallel: the other gradients from the
+//                 chunk's inputs, S, dS', U and dU
+// Every output element is written by exactly one thread (no atomics), so the
+// results do not depend on scheduling.
 #include "kda.h"
 #include "kda_common.cuh"
+#include "kda_sm100.cuh"
 
 namespace kda {
 namespace {
 
-constexpr int kBlk = 16;   // tokens between checkpoints (a block's states stay L2-resident)
-constexpr int kAhead = 8;  // tokens ahead whose lines are prefetched into L2
-constexpr int kCols = 8;   // state columns per CTA (NC below)
-constexpr int NC = kCols;
+using sm100::cp_async16;
+using sm100::cp_async_commit;
+using sm100::cp_async_wait;
+
+constexpr int C = 16;          // tokens per chunk
+constexpr int kThreads = 256;  // every launch
+constexpr int kWarps = kThreads / 32;
+constexpr int NC = 16;         // state columns of one chain CTA
 
 struct BwdParams {
     const void *q, *k, *v, *g, *beta, *gate, *dy;
     const int32_t *cu;
     const float *s0, *dsT;
     float *dq, *dk, *dv, *dg, *dbeta, *dgate, *ds0;
-    float *ckpt, *scratch;
-    int N, H, DV, T;
+    float *prep;  // per (slot, head): the prep block (Blk below)
+    float *Sst;   // per (slot, head): the state entering the chunk, [DK][DV]
+    float *dSst;  // per (slot, head): dL/d(state leaving the chunk), [DK][DV]
+    float *Ust;   // per (slot, head): U, [C][DV]
+    float *dUst;  // per (slot, head): dL/dU, [C][DV]
+    int N, H, T;
     float scale;
 };
 
-// x[c] (c < NC) summed over the 32 lanes of the warp; lane l returns column
-// l % NC.  With NC < 32 the lanes 16 (and 8) apart are added first.  Then
-// recursive halving: at width s a lane keeps the half of its columns selected
-// by bit s of its lane id and adds the partner's copy of that half.
-KDA_DEVICE float reduce_scatter(float (&x)[NC], int lane) {
-    static_assert(NC == 8 || NC == 16 || NC == 32, "slice width");
-    if constexpr (NC <= 16) {
-#pragma unroll
-        for (int c = 0; c < NC; ++c) x[c] += __shfl_xor_sync(0xffffffffu, x[c], 16);
-    }
-    if constexpr (NC <= 8) {
-#pragma unroll
-        for (int c = 0; c < NC; ++c) x[c] += __shfl_xor_sync(0xffffffffu, x[c], 8);
-    }
-#pragma unroll
-    for (int s = NC / 2; s >= 1; s >>= 1) {
-        const bool up = lane & s;
-#pragma unroll
-        for (int m = 0; m < s; ++m) {
-            const float send = up ? x[m] : x[m + s];
-            const float keep = up ? x[m + s] : x[m];
-            x[m] = keep + __shfl_xor_sync(0xffffffffu, send, s);
-        }
-    }
-    return x[0];
-}
-
-// Column sums over all key channels of the CTA: out[c] = sum_i x_i[c].
-// Two barriers: the first also publishes the token's shared inputs.
-template <int NW>
-KDA_DEVICE void col_sum(float (&x)[NC], float *red, float *out, int warp, int lane) {
-    const float sx = reduce_scatter(x, lane);
-    if (lane < NC) red[warp * NC + lane] = sx;
-    __syncthreads();
-    if (warp == 0 && lane < NC) {
-        float t = 0.f;
-#pragma unroll
-        for (int w = 0; w < NW; ++w) t += red[w * NC + lane];
-        out[lane] = t;
-    }
-    __syncthreads();
-}
-
-// Three column sums and one scalar sum in one exchange: out[0, NC) = sum x,
-// out[NC, 2 NC) = sum y, out[2 NC, 3 NC) = sum z, out[3 NC] = sum w.
-constexpr int kRed3 = 3 * NC + 1;
-template <int NW>
-KDA_DEVICE void col_sum3(float (&x)[NC], float (&y)[NC], float (&z)[NC], float w, float *red,
-                         float *out, int warp, int lane) {
-    const float sx = reduce_scatter(x, lane);
-    const float sy = reduce_scatter(y, lane);
-    const float sz = reduce_scatter(z, lane);
-    const float sw = warp_sum(w);
-    float *r = red + warp * kRed3;
-    if (lane < NC) {
-        r[lane] = sx;
-        r[NC + lane] = sy;
-        r[2 * NC + lane] = sz;
-    }
-    if (lane == 0) r[3 * NC] = sw;
-    __syncthreads();
-    for (int e = threadIdx.x; e < kRed3; e += 32 * NW) {
-        float t = 0.f;
-#pragma unroll
-        for (int q = 0; q < NW; ++q) t += red[q * kRed3 + e];
-        out[e] = t;
-    }
-    __syncthreads();
-}
-
-KDA_DEVICE void prefetch_l2(const void *ptr) {
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
-}
-
-struct FwdIn {  // one token's inputs to the forward step (v: column i, i < NC)
-    float k, g, beta, v;
-};
-struct RevIn {  // one token's inputs to the reverse step (v, gate, dy: column i, i < NC)
-    float k, q, g, beta, v, gate, dy;
+// Offsets (floats) inside one prep block: W, Qd, Kb [C][DK], U0 [C][DV],
+// P [C][C], gamma_C [DK].  Every offset and the block size are multiples of
+// four floats (dk, dv in {64, 128}), so 16-byte copies stay aligned.
+template <int DK, int DV> struct Blk {
+    static constexpr int W = 0, QD = C * DK, KB = 2 * C * DK, U0 = 3 * C * DK;
+    static constexpr int P = U0 + C * DV, GC = P + C * C, size = GC + DK;
 };
 
-template <int DK, typename T>
-// 512 threads per SM at least (four 128-thread CTAs): more chains share each SM
-__global__ void __launch_bounds__(DK, 512 / DK) bwd_kernel(BwdParams p) {
-    constexpr int NW = DK / 32;
-    // per-token shared data, double-buffered by token parity so that a fast
-    // thread writing the next token never overwrites what a slow one still
-    // reads (the barriers of one token separate uses two tokens apart)
-    __shared__ float red[NW * kRed3];
-    __shared__ float cv[2][NC], cgt[2][NC], cdy[2][NC];
-    __shared__ float ca[2][NC], cs[2][kRed3];
+// Chunk slots: chunk c of sequence n is slot cu[n] / C + n + c.  A sequence of
+// L tokens has ceil(L / C) chunks, and the slots of different sequences do
+// not overlap; all fit below total_tokens / C + num_seqs.
+struct Seq {
+    int bos, len, nb;
+    long slot0;
+};
 
-    const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
-    const int nh = blockIdx.x, n = nh / p.H, h = nh % p.H;
-    const int j0 = blockIdx.y * kCols;
-    const int H = p.H, DV = p.DV;
-    // offsets clamped into [0, T]: any offsets keep every access in bounds
-    const int bos = min(max(p.cu[n], 0), p.T);
-    const int eos = min(max(p.cu[n + 1], bos), p.T);
-    const int L = eos - bos;
-    const int nb = (L + kBlk - 1) / kBlk;
-    const long ck0 = bos / kBlk + n;  // first checkpoint slot of the sequence
-    const T *q = (const T *)p.q, *k = (const T *)p.k, *v = (const T *)p.v, *g = (const T *)p.g;
-    const T *beta = (const T *)p.beta, *gate = (const T *)p.gate, *dy = (const T *)p.dy;
-    const float scale = p.scale;
-    float *scr = p.scratch + ((size_t)(nh * gridDim.y + blockIdx.y) * kBlk * DK + i) * kCols;
-    auto ck_row = [&](int b) { return p.ckpt + (((size_t)(ck0 + b) * H + h) * DK + i) * DV + j0; };
-    auto save = [](float *dst, const float (&x)[NC]) {
-#pragma unroll
-        for (int c = 0; c < NC; c += 4)
-            *reinterpret_cast<float4 *>(dst + c) = make_float4(x[c], x[c + 1], x[c + 2], x[c + 3]);
-    };
-    auto load = [](const float *src, float (&x)[NC]) {
-#pragma unroll
-        for (int c = 0; c < NC; c += 4) {
-            const float4 f = *reinterpret_cast<const float4 *>(src + c);
-            x[c] = f.x; x[c + 1] = f.y; x[c + 2] = f.z; x[c + 3] = f.w;
-        }
-    };
-    auto load_fwd = [&](int t) {
-        const size_t r = (size_t)t * H + h;
-        FwdIn x;
-        x.k = ld(k + r * DK + i);
-        x.g = ld(g + r * DK + i);
-        x.beta = ld(beta + r);
-        x.v = i < NC ? ld(v + r * DV + j0 + i) : 0.f;
-        return x;
-    };
-    auto load_rev = [&](int t) {
-        const size_t r = (size_t)t * H + h;
-        RevIn x;
-        x.k = ld(k + r * DK + i);
-        x.q = ld(q + r * DK + i);
-        x.g = ld(g + r * DK + i);
-        x.beta = ld(beta + r);
-        x.v = x.gate = x.dy = 0.f;
-        if (i < NC) {
-            const size_t rc = r * DV + j0 + i;
-            x.v = ld(v + rc);
-            x.gate = gate ? ld(gate + rc) : 1.f;
-            x.dy = ld(dy + rc);
-        }
-        return x;
-    };
+KDA_DEVICE int clamp_off(const BwdParams &p, int n) { return min(max(p.cu[n], 0), p.T); }
 
-    // L2 prefetch of token t's input lines (one thread per 128-byte line of a
-    // row; t must be a token of this sequence)
-    constexpr int kLine = 128 / (int)sizeof(T);
-    auto prefetch_in = [&](int t, bool rev) {
-        const size_t r = (size_t)t * H + h;
-        if (i % kLine == 0) {
-            prefetch_l2(k + r * DK + i);
-            prefetch_l2(g + r * DK + i);
-            if (rev) prefetch_l2(q + r * DK + i);
-        }
-        if (i == 0) {
-            prefetch_l2(beta + r);
-            prefetch_l2(v + r * DV + j0);
-            if (rev) {
-                prefetch_l2(dy + r * DV + j0);
-                if (gate) prefetch_l2(gate + r * DV + j0);
-            }
-        }
-    };
+KDA_DEVICE Seq seq_of(const BwdParams &p, int n) {
+    Seq s;
+    s.bos = clamp_off(p, n);
+    const int eos = min(max(p.cu[n + 1], s.bos), p.T);
+    s.len = eos - s.bos;
+    s.nb = (s.len + C - 1) / C;
+    s.slot0 = s.bos / C + n;
+    return s;
+}
 
-    // S <- the state after token t (S holds the state before it)
-    auto fwd_step = [&](int t, const FwdIn &in, float (&S)[NC]) {
-        const int par = t & 1;
-        const float al = __expf(in.g);
-        if (i < NC) cv[par][i] = in.v;
-        float x[NC];
-#pragma unroll
-        for (int c = 0; c < NC; ++c) {
-            S[c] *= al;
-            x[c] = S[c] * in.k;
-        }
-        col_sum<NW>(x, red, ca[par], warp, lane);
-#pragma unroll
-        for (int c = 0; c < NC; ++c) S[c] += in.k * (in.beta * (cv[par][c] - ca[par][c]));
-    };
-    // forward over tokens [t0, t1) with the next token's inputs in flight
-    auto fwd_run = [&](int t0, int t1, float (&S)[NC], bool keep) {
-        if (t0 >= t1) return;
-        FwdIn cur = load_fwd(t0);
-        for (int t = t0; t < t0 + kAhead && t < t1; ++t) prefetch_in(t, false);
-        for (int t = t0; t < t1; ++t) {
-            if (t + kAhead < t1) prefetch_in(t + kAhead, false);
-            if (keep) save(scr + (size_t)(t - t0) * DK * kCols, S);
-            else if ((t - bos) % kBlk == 0) save(ck_row((t - bos) / kBlk), S);
-            const FwdIn nxt = t + 1 < t1 ? load_fwd(t + 1) : cur;
-            fwd_step(t, cur, S);
-            cur = nxt;
-        }
-    };
-
-    // ---- forward sweep: a checkpoint at the start of every block
-    float S[NC];
-#pragma unroll
-    for (int c = 0; c < NC; ++c) S[c] = p.s0 ? p.s0[((size_t)nh * DK + i) * DV + j0 + c] : 0.f;
-    if (nb > 0) {
-        fwd_run(bos, bos + (nb - 1) * kBlk, S, false);
-        save(ck_row(nb - 1), S);
+// The sequence and chunk of a slot (false: no chunk uses it).  Offsets are
+// clamped as in seq_of, so any offsets keep every access in bounds.
+KDA_DEVICE bool chunk_of_slot(const BwdParams &p, long slot, Seq &s, int &c) {
+    int lo = 0, hi = p.N - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if ((long)(clamp_off(p, mid) / C) + mid <= slot) lo = mid;
+        else hi = mid - 1;
     }
+    s = seq_of(p, lo);
+    const long cc = slot - s.slot0;
+    if (cc < 0 || cc >= s.nb) return false;
+    c = (int)cc;
+    return true;
+}
 
-    // ---- reverse sweep
-    float dS[NC];
+KDA_DEVICE float dot4(float4 a, float4 b, float acc) {
+    acc = fmaf(a.x, b.x, acc);
+    acc = fmaf(a.y, b.y, acc);
+    acc = fmaf(a.z, b.z, acc);
+    return fmaf(a.w, b.w, acc);
+}
+
+// ---- the chunk's operands in shared memory (prep_kernel and grad_kernel)
+template <int DK, int DV> struct alignas(16) PrepSm {
+    static constexpr int LK = DK + 4;                        // padded row strides (floats)
+    static constexpr int LM = (DK > DV ? DK : DV) + 4;
+    float kd[C][LK], ki[C][LK], qd[C][LK], kb[C][LK], gs[C][LK];  // gs: G
+    float vs[C][LM];                                         // V (grad_kernel: then dKd)
+    float A[C][C + 1], P[C][C + 1], X[C][C + 1], Tm[C][C + 1];
+    float beta[C];
+    float gc[DK];                                            // gamma_C
+};
+
+// Loads the chunk (rows t0 .. t0 + n - 1 of head h; the rest zero) and forms
+// G, Kd, Ki, Qd, Kb, gamma_C, A, P, X and T in shared memory.
+template <int DK, int DV, typename T>
+KDA_DEVICE void prep_chunk(const BwdParams &p, PrepSm<DK, DV> &sm, int h, int t0, int n) {
+    const int tid = threadIdx.x, H = p.H;
+    const T *q = (const T *)p.q, *k = (const T *)p.k, *g = (const T *)p.g;
+    const T *v = (const T *)p.v, *beta = (const T *)p.beta;
+    for (int e = tid; e < C * DK; e += kThreads) {
+        const int r = e / DK, i = e % DK;
+        float kv = 0.f, qv = 0.f, gv = 0.f;
+        if (r < n) {
+            const size_t o = ((size_t)(t0 + r) * H + h) * DK + i;
+            kv = ld(k + o);
+            qv = ld(q + o);
+            gv = ld(g + o);
+        }
+        sm.kd[r][i] = kv;
+        sm.qd[r][i] = qv;
+        sm.gs[r][i] = gv;
+    }
+    for (int e = tid; e < C * DV; e += kThreads) {
+        const int r = e / DV, j = e % DV;
+        sm.vs[r][j] = r < n ? ld(v + ((size_t)(t0 + r) * H + h) * DV + j) : 0.f;
+    }
+    if (tid < C) sm.beta[tid] = tid < n ? ld(beta + (size_t)(t0 + tid) * H + h) : 0.f;
+    __syncthreads();
+    if (tid < DK) {  // decay: one thread per key channel, down the rows
+        const int i = tid;
+        float G = 0.f;
 #pragma unroll
-    for (int c = 0; c < NC; ++c) dS[c] = p.dsT ? p.dsT[((size_t)nh * DK + i) * DV + j0 + c] : 0.f;
-    for (int b = nb - 1; b >= 0; --b) {
-        const int tb = bos + b * kBlk, te = min(eos, tb + kBlk);
-        // the last token walked (tb + kBlk of the previous block, or the
-        // forward sweep's) may share a buffer parity with the first one below
+        for (int r = 0; r < C; ++r) {
+            G += sm.gs[r][i];
+            sm.gs[r][i] = G;
+        }
+        const float GC = G;
+        sm.gc[i] = expf(GC);
+#pragma unroll 4
+        for (int r = 0; r < C; ++r) {
+            const float Gr = sm.gs[r][i], kv = sm.kd[r][i];
+            const float e = expf(Gr);
+            sm.kd[r][i] = kv * e;
+            sm.ki[r][i] = kv * expf(-Gr);
+            sm.qd[r][i] = p.scale * sm.qd[r][i] * e;
+            sm.kb[r][i] = kv * expf(GC - Gr);
+        }
+    }
+    __syncthreads();
+    {  // A and P: thread (r, s)
+        const int r = tid >> 4, s = tid & 15;
+        const float4 *kd4 = reinterpret_cast<const float4 *>(sm.kd[r]);
+        const float4 *qd4 = reinterpret_cast<const float4 *>(sm.qd[r]);
+        const float4 *ki4 = reinterpret_cast<const float4 *>(sm.ki[s]);
+        float a = 0.f, pp = 0.f;
+#pragma unroll 8
+        for (int c4 = 0; c4 < DK / 4; ++c4) {
+            const float4 x = ki4[c4];
+            a = dot4(kd4[c4], x, a);
+            pp = dot4(qd4[c4], x, pp);
+        }
+        sm.A[r][s] = r > s ? a : 0.f;
+        sm.P[r][s] = r >= s ? pp : 0.f;
+    }
+    __syncthreads();
+    if (tid < C) {  // X = (I + Diag(beta) A)^-1 by forward substitution, column s per lane
+        const int s = tid;
+        float x[C];
+#pragma unroll
+        for (int r = 0; r < C; ++r) {
+            float acc = 0.f;
+#pragma unroll
+            for (int m = 0; m < r; ++m) acc = fmaf(sm.A[r][m], x[m], acc);
+            x[r] = r < s ? 0.f : (r == s ? 1.f : -sm.beta[r] * acc);
+        }
+        const float bs = sm.beta[s];
+#pragma unroll
+        for (int r = 0; r < C; ++r) {
+            sm.X[r][s] = x[r];
+            sm.Tm[r][s] = x[r] * bs;
+        }
+    }
+    __syncthreads();
+}
+
+template <int DK, int DV, typename T>
+__global__ void __launch_bounds__(kThreads) prep_kernel(BwdParams p) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    auto &sm = *reinterpret_cast<PrepSm<DK, DV> *>(smem_raw);
+    using B = Blk<DK, DV>;
+    const long slot = blockIdx.x;
+    const int h = blockIdx.y, tid = threadIdx.x;
+    Seq s;
+    int c;
+    if (!chunk_of_slot(p, slot, s, c)) return;
+    prep_chunk<DK, DV, T>(p, sm, h, s.bos + c * C, min(C, s.len - c * C));
+    float *out = p.prep + ((size_t)slot * p.H + h) * B::size;
+    for (int e = tid; e < C * DK; e += kThreads) {
+        const int r = e / DK, i = e % DK;
+        float w = 0.f;
+#pragma unroll
+        for (int m = 0; m < C; ++m) w = fmaf(sm.Tm[r][m], sm.kd[m][i], w);  // T is lower triangular
+        out[B::W + e] = w;
+        out[B::QD + e] = sm.qd[r][i];
+        out[B::KB + e] = sm.kb[r][i];
+    }
+    for (int e = tid; e < C * DV; e += kThreads) {
+        const int r = e / DV, j = e % DV;
+        float u = 0.f;
+#pragma unroll
+        for (int m = 0; m < C; ++m) u = fmaf(sm.Tm[r][m], sm.vs[m][j], u);
+        out[B::U0 + e] = u;
+    }
+    out[B::P + tid] = sm.P[tid >> 4][tid & 15];
+    for (int i = tid; i < DK; i += kThreads) out[B::GC + i] = sm.gc[i];
+}
+
+// ---- the sequential passes: one CTA per (sequence, head, NC state columns).
+// Thread t owns column j = t % 16 of the slice and rows rg R .. rg R + R - 1
+// (rg = t / 16, R = DK / 16) of the state (or of its gradient) in registers;
+// for the chunk's [C][NC] outputs it is thread (r, j) with r = rg.  Sums over
+// the key channels: the two row groups of a warp are added with one shuffle,
+// then the eight warps through shared memory.
+template <int DK> struct alignas(16) ChainSm {
+    struct Buf {                   // one chunk's prep block (the rows this CTA needs)
+        float wqk[3 * C * DK];     // W, Qd, Kb: [C][DK] each
+        float pg[C * C + DK];      // P [C][C], gamma_C [DK]
+        float u0[C * NC];          // forward pass: U0 columns of this CTA
+        KDA_DEVICE const float *w() const { return wqk; }
+        KDA_DEVICE const float *qd() const { return wqk + C * DK; }
+        KDA_DEVICE const float *kb() const { return wqk + 2 * C * DK; }
+        KDA_DEVICE const float *pm() const { return pg; }
+        KDA_DEVICE const float *gc() const { return pg + C * C; }
+    } buf[2];
+    float red[kWarps][C][32];      // partial sums per warp
+    float xs[2][C][NC];            // reverse pass: dO of the chunk (by iteration parity)
+    float us[C][NC];               // U (forward) or dU (reverse) of the chunk
+};
+
+// cp.async of chunk prep block `blk` into `b` (one group).
+template <int DK, int DV>
+KDA_DEVICE void fetch_prep(typename ChainSm<DK>::Buf &b, const float *blk, int j0, bool with_u0) {
+    using B = Blk<DK, DV>;
+    const int tid = threadIdx.x;
+    for (int e = tid; e < 3 * C * DK / 4; e += kThreads) cp_async16(b.wqk + 4 * e, blk + B::W + 4 * e, true);
+    for (int e = tid; e < (C * C + DK) / 4; e += kThreads) cp_async16(b.pg + 4 * e, blk + B::P + 4 * e, true);
+    if (with_u0 && tid < C * NC / 4) {
+        const int r = tid / (NC / 4), c4 = tid % (NC / 4);
+        cp_async16(b.u0 + r * NC + 4 * c4, blk + B::U0 + r * DV + j0 + 4 * c4, true);
+    }
+    cp_async_commit();
+}
+
+// x[0..R) . row segment (R consecutive floats of shared memory, 16-byte aligned)
+template <int R> KDA_DEVICE float dot_rows(const float *seg, const float (&x)[R]) {
+    float a = 0.f;
+#pragma unroll
+    for (int m4 = 0; m4 < R / 4; ++m4) {
+        const float4 w = *reinterpret_cast<const float4 *>(seg + 4 * m4);
+        a = fmaf(w.x, x[4 * m4], a);
+        a = fmaf(w.y, x[4 * m4 + 1], a);
+        a = fmaf(w.z, x[4 * m4 + 2], a);
+        a = fmaf(w.w, x[4 * m4 + 3], a);
+    }
+    return a;
+}
+
+// x[0..R) += c * row segment
+template <int R> KDA_DEVICE void axpy_rows(const float *seg, float c, float (&x)[R]) {
+#pragma unroll
+    for (int m4 = 0; m4 < R / 4; ++m4) {
+        const float4 w = *reinterpret_cast<const float4 *>(seg + 4 * m4);
+        x[4 * m4] = fmaf(w.x, c, x[4 * m4]);
+        x[4 * m4 + 1] = fmaf(w.y, c, x[4 * m4 + 1]);
+        x[4 * m4 + 2] = fmaf(w.z, c, x[4 * m4 + 2]);
+        x[4 * m4 + 3] = fmaf(w.w, c, x[4 * m4 + 3]);
+    }
+}
+
+// Forward pass over the chunks of one sequence: stores the state entering
+// each chunk and U; dgate = dy (.) O.
+template <int DK, int DV, typename T>
+__global__ void __launch_bounds__(kThreads) fwd_chain(BwdParams p) {
+    constexpr int R = DK / 16;
+    using B = Blk<DK, DV>;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    auto &sm = *reinterpret_cast<ChainSm<DK> *>(smem_raw);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int j = tid & 15, rg = tid >> 4, i0 = rg * R;
+    const int nh = blockIdx.x, n = nh / p.H, h = nh % p.H, H = p.H;
+    const int j0 = blockIdx.y * NC;
+    const Seq s = seq_of(p, n);
+    const T *dy = (const T *)p.dy;
+    float S[R];
+#pragma unroll
+    for (int m = 0; m < R; ++m) S[m] = p.s0 ? p.s0[((size_t)nh * DK + i0 + m) * DV + j0 + j] : 0.f;
+    if (s.nb == 0) return;
+    auto blk = [&](int c) { return p.prep + ((size_t)(s.slot0 + c) * H + h) * B::size; };
+    auto load_dy = [&](int c) {
+        const int r = c * C + rg;
+        return (p.dgate && r < s.len) ? ld(dy + ((size_t)(s.bos + r) * H + h) * DV + j0 + j) : 0.f;
+    };
+    fetch_prep<DK, DV>(sm.buf[0], blk(0), j0, true);
+    float dyv = load_dy(0);
+    for (int c = 0; c < s.nb; ++c) {
+        const auto &b = sm.buf[c & 1];
+        cp_async_wait<0>();
         __syncthreads();
-        load(ck_row(b), S);
-        // the block's states S_{t-1} into scratch (the last one saved, not stepped)
-        fwd_run(tb, te - 1, S, true);
-        save(scr + (size_t)(te - 1 - tb) * DK * kCols, S);
-
-        RevIn cur = load_rev(te - 1);
-        float Sp[NC];
-        load(scr + (size_t)(te - 1 - tb) * DK * kCols, Sp);
-        for (int t = te - 1; t >= tb && t >= te - kAhead; --t) {
-            prefetch_in(t, true);
-            prefetch_l2(scr + (size_t)(t - tb) * DK * kCols);
+        if (c + 1 < s.nb) fetch_prep<DK, DV>(sm.buf[(c + 1) & 1], blk(c + 1), j0, true);
+        const size_t idx = (size_t)(s.slot0 + c) * H + h;
+        float *Sg = p.Sst + idx * DK * DV + (size_t)i0 * DV + j0 + j;
+#pragma unroll
+        for (int m = 0; m < R; ++m) Sg[(size_t)m * DV] = S[m];
+        // rows of W S and Qd S over this thread's key channels; lanes 0-15
+        // keep the U sums of the warp's two row groups, lanes 16-31 the Qd S sums
+        const bool hi = lane >= 16;
+#pragma unroll
+        for (int r = 0; r < C; ++r) {
+            const float pu = dot_rows<R>(b.w() + r * DK + i0, S);
+            const float pq = dot_rows<R>(b.qd() + r * DK + i0, S);
+            const float send = hi ? pu : pq, keep = hi ? pq : pu;
+            sm.red[warp][r][lane] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
         }
-        for (int t = te - 1; t >= tb; --t) {
-            const int par = t & 1;
-            const size_t r = (size_t)t * H + h;
-            if (t - kAhead >= tb) {
-                prefetch_in(t - kAhead, true);
-                prefetch_l2(scr + (size_t)(t - kAhead - tb) * DK * kCols);
-            }
-            RevIn nxt = cur;
-            float Sn[NC];
-            if (t > tb) {
-                nxt = load_rev(t - 1);
-                load(scr + (size_t)(t - 1 - tb) * DK * kCols, Sn);
-            }
-            const float al = __expf(cur.g);
-            if (i < NC) {
-                cv[par][i] = cur.v;
-                cgt[par][i] = cur.gate;
-                cdy[par][i] = cur.dy;
-            }
-            // one exchange: a = S'^T k, b = S'^T q, c = dS^T k (dS = dL/dS_t
-            // without this token's read) and k.q
-            float x[NC], y[NC], z[NC];
+        __syncthreads();
+        float u = 0.f, qs = 0.f;
 #pragma unroll
-            for (int c = 0; c < NC; ++c) {
-                Sp[c] *= al;
-                x[c] = Sp[c] * cur.k;
-                y[c] = Sp[c] * cur.q;
-                z[c] = dS[c] * cur.k;
-            }
-            col_sum3<NW>(x, y, z, cur.k * cur.q, red, cs[par], warp, lane);
-            const float *A = cs[par], *Bq = cs[par] + NC, *C = cs[par] + 2 * NC;
-            const float kq = cs[par][3 * NC], bt = cur.beta;
-            if (i < NC) {  // per column: u, o (= scale (b + (k.q) u)), du, dv, dgate
-                const float u = bt * (cur.v - A[i]);
-                const float o = scale * (Bq[i] + kq * u);
-                const float du = C[i] + scale * kq * (cur.gate * cur.dy);
-                p.dv[r * DV + j0 + i] = bt * du;
-                if (p.dgate) p.dgate[r * DV + j0 + i] = cur.dy * o;
-            }
-            if (i == 0) {
-                float db = 0.f;
+        for (int w = 0; w < kWarps; ++w) {
+            u += sm.red[w][rg][j];
+            qs += sm.red[w][rg][16 + j];
+        }
+        u = b.u0[rg * NC + j] - u;
+        sm.us[rg][j] = u;
+        p.Ust[idx * C * DV + (size_t)rg * DV + j0 + j] = u;
+        __syncthreads();
+        float o = qs;  // O = Qd S + P U (P is zero above the diagonal)
 #pragma unroll
-                for (int c = 0; c < NC; ++c) {
-                    const float du = C[c] + scale * kq * (cgt[par][c] * cdy[par][c]);
-                    db += du * (cv[par][c] - A[c]);
-                }
-                atomicAdd(p.dbeta + r, db);
-            }
-            float dqi = 0.f, dki = 0.f, dgi = 0.f;
+        for (int r2 = 0; r2 < C; ++r2) o = fmaf(b.pm()[rg * C + r2], sm.us[r2][j], o);
+        if (p.dgate && c * C + rg < s.len)
+            p.dgate[((size_t)(s.bos + c * C + rg) * H + h) * DV + j0 + j] = dyv * o;
+        if (c + 1 < s.nb) dyv = load_dy(c + 1);
+        // S <- Diag(gamma_C) S + Kb^T U
+        const float *gc = b.gc() + i0;
 #pragma unroll
-            for (int c = 0; c < NC; ++c) {
-                const float doc = cgt[par][c] * cdy[par][c];
-                const float uc = bt * (cv[par][c] - A[c]);
-                dqi += (Sp[c] + cur.k * uc) * doc;              // S_t do
-                const float dsc = dS[c] + scale * cur.q * doc;  // dL/dS_t
-                const float da = -bt * (C[c] + scale * kq * doc);
-                dki += dsc * uc + Sp[c] * da;
-                const float dsp = dsc + cur.k * da;              // dL/dS'
-                dgi += dsp * Sp[c];
-                dS[c] = al * dsp;                                // dL/dS_{t-1}
-            }
-            atomicAdd(p.dq + r * DK + i, scale * dqi);
-            atomicAdd(p.dk + r * DK + i, dki);
-            atomicAdd(p.dg + r * DK + i, dgi);
-            cur = nxt;
+        for (int m = 0; m < R; ++m) S[m] *= gc[m];
 #pragma unroll
-            for (int c = 0; c < NC; ++c) Sp[c] = Sn[c];
+        for (int r = 0; r < C; ++r) axpy_rows<R>(b.kb() + r * DK + i0, sm.us[r][j], S);
+    }
+}
+
+// Reverse pass over the chunks of one sequence: stores dL/d(state leaving
+// each chunk) and dU; writes dL/d(initial state).
+template <int DK, int DV, typename T>
+__global__ void __launch_bounds__(kThreads) rev_chain(BwdParams p) {
+    constexpr int R = DK / 16;
+    using B = Blk<DK, DV>;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    auto &sm = *reinterpret_cast<ChainSm<DK> *>(smem_raw);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int j = tid & 15, rg = tid >> 4, i0 = rg * R;
+    const int nh = blockIdx.x, n = nh / p.H, h = nh % p.H, H = p.H;
+    const int j0 = blockIdx.y * NC;
+    const Seq s = seq_of(p, n);
+    const T *dy = (const T *)p.dy, *gate = (const T *)p.gate;
+    float dS[R];
+#pragma unroll
+    for (int m = 0; m < R; ++m) dS[m] = p.dsT ? p.dsT[((size_t)nh * DK + i0 + m) * DV + j0 + j] : 0.f;
+    auto blk = [&](int c) { return p.prep + ((size_t)(s.slot0 + c) * H + h) * B::size; };
+    auto load_do = [&](int c) {
+        const int r = c * C + rg;
+        if (r >= s.len) return 0.f;
+        const size_t o = ((size_t)(s.bos + r) * H + h) * DV + j0 + j;
+        const float d = ld(dy + o);
+        return gate ? ld(gate + o) * d : d;
+    };
+    if (s.nb > 0) fetch_prep<DK, DV>(sm.buf[0], blk(s.nb - 1), j0, false);
+    float dov = s.nb > 0 ? load_do(s.nb - 1) : 0.f;
+    for (int it = 0; it < s.nb; ++it) {
+        const int c = s.nb - 1 - it;
+        const auto &b = sm.buf[it & 1];
+        cp_async_wait<0>();
+        __syncthreads();
+        if (c > 0) fetch_prep<DK, DV>(sm.buf[(it + 1) & 1], blk(c - 1), j0, false);
+        sm.xs[it & 1][rg][j] = dov;
+        const size_t idx = (size_t)(s.slot0 + c) * H + h;
+        float *dSg = p.dSst + idx * DK * DV + (size_t)i0 * DV + j0 + j;
+#pragma unroll
+        for (int m = 0; m < R; ++m) dSg[(size_t)m * DV] = dS[m];
+        // rows of Kb dS'; lanes 0-15 keep rows 0-7 of the warp's two row
+        // groups, lanes 16-31 rows 8-15
+        const bool hi = lane >= 16;
+        float pk[C];
+#pragma unroll
+        for (int r = 0; r < C; ++r) pk[r] = dot_rows<R>(b.kb() + r * DK + i0, dS);
+#pragma unroll
+        for (int m = 0; m < C / 2; ++m) {
+            const float send = hi ? pk[m] : pk[m + 8], keep = hi ? pk[m + 8] : pk[m];
+            sm.red[warp][m][lane] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+        }
+        __syncthreads();
+        float du = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) du += sm.red[w][rg & 7][(rg >> 3) * 16 + j];
+#pragma unroll
+        for (int r2 = 0; r2 < C; ++r2) du = fmaf(b.pm()[r2 * C + rg], sm.xs[it & 1][r2][j], du);  // P^T dO
+        sm.us[rg][j] = du;
+        p.dUst[idx * C * DV + (size_t)rg * DV + j0 + j] = du;
+        if (c > 0) dov = load_do(c - 1);
+        __syncthreads();
+        // dS <- Diag(gamma_C) dS + Qd^T dO - W^T dU
+        const float *gc = b.gc() + i0;
+#pragma unroll
+        for (int m = 0; m < R; ++m) dS[m] *= gc[m];
+#pragma unroll
+        for (int r = 0; r < C; ++r) {
+            axpy_rows<R>(b.qd() + r * DK + i0, sm.xs[it & 1][r][j], dS);
+            axpy_rows<R>(b.w() + r * DK + i0, -sm.us[r][j], dS);
         }
     }
     if (p.ds0) {
 #pragma unroll
-        for (int c = 0; c < NC; ++c) p.ds0[((size_t)nh * DK + i) * DV + j0 + c] = dS[c];
+        for (int m = 0; m < R; ++m) p.ds0[((size_t)nh * DK + i0 + m) * DV + j0 + j] = dS[m];
     }
 }
 
-template <int DK, typename T>
-cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t st) {
-    bwd_kernel<DK, T><<<dim3((unsigned)(p.N * p.H), (unsigned)(p.DV / kCols)), DK, 0, st>>>(p);
+// ---- the per-chunk gradients: one CTA per (chunk, head)
+template <int DK, int DV> struct alignas(16) GradSm {
+    static constexpr int LK = DK + 4, LV = DV + 4, LM = PrepSm<DK, DV>::LM;
+    PrepSm<DK, DV> pr;
+    float us[C][LM];                   // U, then dKi
+    float dus[C][LV], dos[C][LV];      // dU, dO
+    float dqd[C][LK], dw[C][LK], dkb[C][LK];
+    float dP[C][C + 1], dT[C][C + 1], M[C][C + 1], dL[C][C + 1];
+    float dgc[DK];                     // dgamma_C (.) gamma_C
+};
+
+template <int DK, int DV, typename T>
+__global__ void __launch_bounds__(kThreads, 2) grad_kernel(BwdParams p) {
+    constexpr int TPC = kThreads / DK;  // threads per key channel in the products with S
+    constexpr int JW = DV / TPC;        // their columns each
+    constexpr int RPT = C / TPC;        // rows per thread in the row-wise steps
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    auto &sm = *reinterpret_cast<GradSm<DK, DV> *>(smem_raw);
+    auto &pr = sm.pr;
+    const long slot = blockIdx.x;
+    const int h = blockIdx.y, tid = threadIdx.x, H = p.H;
+    Seq s;
+    int c;
+    if (!chunk_of_slot(p, slot, s, c)) return;
+    const int t0 = s.bos + c * C, n = min(C, s.len - c * C);
+    const size_t idx = (size_t)slot * H + h;
+    const T *dy = (const T *)p.dy, *gate = (const T *)p.gate;
+
+    // U, dU (workspace) and dO = gate (.) dy
+    for (int e = tid; e < C * DV; e += kThreads) {
+        const int r = e / DV, jj = e % DV;
+        sm.us[r][jj] = p.Ust[idx * C * DV + e];
+        sm.dus[r][jj] = p.dUst[idx * C * DV + e];
+        float d = 0.f;
+        if (r < n) {
+            const size_t o = ((size_t)(t0 + r) * H + h) * DV + jj;
+            d = ld(dy + o);
+            if (gate) d *= ld(gate + o);
+        }
+        sm.dos[r][jj] = d;
+    }
+    prep_chunk<DK, DV, T>(p, pr, h, t0, n);  // ends with a barrier
+
+    {  // dQd = dO S^T, dW = -dU S^T, dKb = U dS'^T, dgamma_C = rowsum(dS' (.) S)
+        // the TPC threads of a channel take interleaved 4-column groups
+        const int i = tid / TPC, part = tid % TPC;
+        const float4 *S4 = reinterpret_cast<const float4 *>(p.Sst + idx * DK * DV + (size_t)i * DV);
+        const float4 *D4 = reinterpret_cast<const float4 *>(p.dSst + idx * DK * DV + (size_t)i * DV);
+        float aq[C], aw[C], ab[C], ag = 0.f;
+#pragma unroll
+        for (int r = 0; r < C; ++r) aq[r] = aw[r] = ab[r] = 0.f;
+#pragma unroll 2
+        for (int c4 = 0; c4 < JW / 4; ++c4) {
+            const int j4 = c4 * TPC + part, jj = 4 * j4;
+            const float4 s4 = __ldg(S4 + j4), d4 = __ldg(D4 + j4);
+            ag = dot4(s4, d4, ag);
+#pragma unroll
+            for (int r = 0; r < C; ++r) {
+                aq[r] = dot4(*reinterpret_cast<const float4 *>(&sm.dos[r][jj]), s4, aq[r]);
+                aw[r] = dot4(*reinterpret_cast<const float4 *>(&sm.dus[r][jj]), s4, aw[r]);
+                ab[r] = dot4(*reinterpret_cast<const float4 *>(&sm.us[r][jj]), d4, ab[r]);
+            }
+        }
+#pragma unroll
+        for (int o = 1; o < TPC; o <<= 1) {
+            ag += __shfl_xor_sync(0xffffffffu, ag, o);
+#pragma unroll
+            for (int r = 0; r < C; ++r) {
+                aq[r] += __shfl_xor_sync(0xffffffffu, aq[r], o);
+                aw[r] += __shfl_xor_sync(0xffffffffu, aw[r], o);
+                ab[r] += __shfl_xor_sync(0xffffffffu, ab[r], o);
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < C; ++r) {
+            if (r % TPC == part) {
+                sm.dqd[r][i] = aq[r];
+                sm.dw[r][i] = -aw[r];
+                sm.dkb[r][i] = ab[r];
+            }
+        }
+        if (part == 0) sm.dgc[i] = ag * pr.gc[i];
+    }
+    __syncthreads();
+    {  // dP = tril(dO U^T), dT = dU V^T + dW Kd^T: thread (r, s)
+        const int r = tid >> 4, s2 = tid & 15;
+        float dp = 0.f, dt = 0.f;
+#pragma unroll 8
+        for (int c4 = 0; c4 < DV / 4; ++c4) {
+            dp = dot4(*reinterpret_cast<const float4 *>(&sm.dos[r][4 * c4]),
+                      *reinterpret_cast<const float4 *>(&sm.us[s2][4 * c4]), dp);
+            dt = dot4(*reinterpret_cast<const float4 *>(&sm.dus[r][4 * c4]),
+                      *reinterpret_cast<const float4 *>(&pr.vs[s2][4 * c4]), dt);
+        }
+#pragma unroll 8
+        for (int c4 = 0; c4 < DK / 4; ++c4)
+            dt = dot4(*reinterpret_cast<const float4 *>(&sm.dw[r][4 * c4]),
+                      *reinterpret_cast<const float4 *>(&pr.kd[s2][4 * c4]), dt);
+        sm.dP[r][s2] = r >= s2 ? dp : 0.f;
+        sm.dT[r][s2] = dt;
+    }
+    __syncthreads();
+    {  // M = X^T dT Diag(beta): thread (r, s)
+        const int r = tid >> 4, s2 = tid & 15;
+        float m = 0.f;
+#pragma unroll
+        for (int q = 0; q < C; ++q) m = fmaf(pr.X[q][r], sm.dT[q][s2], m);
+        sm.M[r][s2] = m * pr.beta[s2];
+    }
+    // dV = T^T dU (rows < n)
+    for (int e = tid; e < C * DV; e += kThreads) {
+        const int r = e / DV, jj = e % DV;
+        float d = 0.f;
+#pragma unroll
+        for (int q = 0; q < C; ++q) d = fmaf(pr.Tm[q][r], sm.dus[q][jj], d);
+        if (r < n) p.dv[((size_t)(t0 + r) * H + h) * DV + jj] = d;
+    }
+    __syncthreads();
+    {  // dL = -M X^T: thread (r, s)
+        const int r = tid >> 4, s2 = tid & 15;
+        float l = 0.f;
+#pragma unroll
+        for (int q = 0; q < C; ++q) l = fmaf(sm.M[r][q], pr.X[s2][q], l);
+        sm.dL[r][s2] = -l;
+    }
+    __syncthreads();
+    if (tid < n) {  // dbeta = colsum(X (.) dT) + rowsum(strict(dL) (.) A)
+        const int r = tid;
+        float db = 0.f;
+#pragma unroll
+        for (int q = 0; q < C; ++q) db = fmaf(pr.X[q][r], sm.dT[q][r], db);
+#pragma unroll
+        for (int q = 0; q < C; ++q) db = fmaf(sm.dL[r][q], pr.A[r][q], db);  // A is strictly lower
+        p.dbeta[(size_t)(t0 + r) * H + h] = db;
+    }
+    {  // dKd = T^T dW + dA Ki, dKi = dA^T Kd + dP^T Qd, dQd += dP Ki; dA = Diag(beta) strict(dL)
+        const int i = tid % DK, r0 = (tid / DK) * RPT;
+#pragma unroll
+        for (int rr = 0; rr < RPT; ++rr) {
+            const int r = r0 + rr;
+            float dkd = 0.f, dki = 0.f, dqd = sm.dqd[r][i];
+#pragma unroll
+            for (int q = 0; q < C; ++q) {
+                dkd = fmaf(pr.Tm[q][r], sm.dw[q][i], dkd);
+                const float a_rq = q < r ? pr.beta[r] * sm.dL[r][q] : 0.f;   // dA[r][q]
+                const float a_qr = q > r ? pr.beta[q] * sm.dL[q][r] : 0.f;   // dA[q][r]
+                dkd = fmaf(a_rq, pr.ki[q][i], dkd);
+                dki = fmaf(a_qr, pr.kd[q][i], dki);
+                dki = fmaf(sm.dP[q][r], pr.qd[q][i], dki);
+                dqd = fmaf(sm.dP[r][q], pr.ki[q][i], dqd);
+            }
+            pr.vs[r][i] = dkd;  // V is no longer needed
+            sm.us[r][i] = dki;  // nor U
+            sm.dqd[r][i] = dqd;
+        }
+    }
+    __syncthreads();
+    if (tid < DK) {  // dq, dk, dg down the rows from the bottom
+        const int i = tid;
+        const float GC = pr.gs[C - 1][i];
+        float acc = sm.dgc[i];
+#pragma unroll
+        for (int r = 0; r < C; ++r) acc = fmaf(sm.dkb[r][i], pr.kb[r][i], acc);
+        for (int r = C - 1; r >= 0; --r) {
+            const float Gr = pr.gs[r][i];
+            const float dkd = pr.vs[r][i], dki = sm.us[r][i], dqd = sm.dqd[r][i], dkb = sm.dkb[r][i];
+            acc += dkd * pr.kd[r][i] - dki * pr.ki[r][i] + dqd * pr.qd[r][i] - dkb * pr.kb[r][i];
+            if (r < n) {
+                const size_t o = ((size_t)(t0 + r) * H + h) * DK + i;
+                const float e = expf(Gr);
+                p.dk[o] = dkd * e + dki * expf(-Gr) + dkb * expf(GC - Gr);
+                p.dq[o] = p.scale * dqd * e;
+                p.dg[o] = acc;
+            }
+        }
+    }
+}
+
+template <typename K> cudaError_t set_smem(K kernel, size_t bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+template <int DK, int DV, typename T>
+cudaError_t launch_bwd_t(const BwdParams &p, long slots, cudaStream_t st) {
+    static_assert(C * C == kThreads, "prep_kernel writes P with one thread per entry");
+    const dim3 per_chunk((unsigned)slots, (unsigned)p.H), per_seq((unsigned)(p.N * p.H), DV / NC);
+    cudaError_t e;
+    if ((e = set_smem(prep_kernel<DK, DV, T>, sizeof(PrepSm<DK, DV>))) != cudaSuccess) return e;
+    if ((e = set_smem(fwd_chain<DK, DV, T>, sizeof(ChainSm<DK>))) != cudaSuccess) return e;
+    if ((e = set_smem(rev_chain<DK, DV, T>, sizeof(ChainSm<DK>))) != cudaSuccess) return e;
+    if ((e = set_smem(grad_kernel<DK, DV, T>, sizeof(GradSm<DK, DV>))) != cudaSuccess) return e;
+    if (slots > 0) prep_kernel<DK, DV, T><<<per_chunk, kThreads, sizeof(PrepSm<DK, DV>), st>>>(p);
+    fwd_chain<DK, DV, T><<<per_seq, kThreads, sizeof(ChainSm<DK>), st>>>(p);
+    rev_chain<DK, DV, T><<<per_seq, kThreads, sizeof(ChainSm<DK>), st>>>(p);
+    if (slots > 0) grad_kernel<DK, DV, T><<<per_chunk, kThreads, sizeof(GradSm<DK, DV>), st>>>(p);
     return cudaGetLastError();
+}
+
+template <int DK, typename T>
+cudaError_t launch_bwd_dk(const BwdParams &p, int dv, long slots, cudaStream_t st) {
+    return dv == 128 ? launch_bwd_t<DK, 128, T>(p, slots, st) : launch_bwd_t<DK, 64, T>(p, slots, st);
 }
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-size_t ckpt_bytes(long T, long N, long H, long dk, long dv) {
-    return align256((size_t)(T / kBlk + N) * H * dk * dv * sizeof(float));
-}
+long slots_of(long T, long N) { return T / C + N; }
 
-size_t scratch_bytes(long N, long H, long dk, long dv) {
-    return align256((size_t)N * H * dv * kBlk * dk * sizeof(float));
+// Workspace regions (bytes, each 256-byte aligned): prep blocks, S, dS', U, dU.
+struct WsLayout {
+    size_t prep, S, dS, U, dU, total;
+};
+
+WsLayout ws_layout(long T, long N, long H, long dk, long dv) {
+    const size_t ch = (size_t)slots_of(T, N) * H;
+    const size_t blk = 3 * C * dk + C * dv + C * C + dk;
+    WsLayout w;
+    w.prep = 0;
+    w.S = w.prep + align256(ch * blk * sizeof(float));
+    w.dS = w.S + align256(ch * dk * dv * sizeof(float));
+    w.U = w.dS + align256(ch * dk * dv * sizeof(float));
+    w.dU = w.U + align256(ch * C * dv * sizeof(float));
+    w.total = w.dU + align256(ch * C * dv * sizeof(float));
+    return w;
 }
 
 bool ok_dim(int d) { return d == 64 || d == 128; }
@@ -373,8 +685,7 @@ extern "C" {
 size_t kda_bwd_workspace_size(int32_t total_tokens, int32_t num_seqs, int32_t H, int32_t dk,
                               int32_t dv) {
     if (total_tokens < 0 || num_seqs < 0 || H < 1 || !kda::ok_dim(dk) || !kda::ok_dim(dv)) return 0;
-    return kda::ckpt_bytes(total_tokens, num_seqs, H, dk, dv) +
-           kda::scratch_bytes(num_seqs, H, dk, dv);
+    return kda::ws_layout(total_tokens, num_seqs, H, dk, dv).total;
 }
 
 int kda_bwd(const void *q, const void *k, const void *v, const void *g, const void *beta,
@@ -407,37 +718,37 @@ int kda_bwd(const void *q, const void *k, const void *v, const void *g, const vo
                          d_final_state};
     for (const void *ptr : out)
         if (ptr && (uintptr_t)ptr % 4) return KDA_ERR_ALIGNMENT;
-    if ((long)num_seqs * H > 0x7fffffffL) return KDA_ERR_UNSUPPORTED;
+    if ((long)num_seqs * H > 0x7fffffffL || kda::slots_of(total_tokens, num_seqs) > 0x7fffffffL)
+        return KDA_ERR_UNSUPPORTED;
     const size_t need = kda_bwd_workspace_size(total_tokens, num_seqs, H, dk, dv);
     if (!workspace || workspace_bytes < need) return KDA_ERR_WORKSPACE;
     if ((uintptr_t)workspace % 256) return KDA_ERR_ALIGNMENT;
 
-    cudaStream_t st = (cudaStream_t)stream;
-    // the row sums and dbeta are accumulated across column slices
-    const size_t tk = (size_t)total_tokens * H;
-    if (tk > 0) {
-        if (cudaMemsetAsync(dq, 0, tk * dk * sizeof(float), st) != cudaSuccess ||
-            cudaMemsetAsync(dk_out, 0, tk * dk * sizeof(float), st) != cudaSuccess ||
-            cudaMemsetAsync(dg, 0, tk * dk * sizeof(float), st) != cudaSuccess ||
-            cudaMemsetAsync(dbeta, 0, tk * sizeof(float), st) != cudaSuccess)
-            return KDA_ERR_CUDA;
-    }
+    const kda::WsLayout w = kda::ws_layout(total_tokens, num_seqs, H, dk, dv);
+    char *ws = (char *)workspace;
     kda::BwdParams p{};
     p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.gate = gate; p.dy = dy;
     p.cu = cu_seqlens;
     p.s0 = initial_state; p.dsT = d_final_state;
     p.dq = dq; p.dk = dk_out; p.dv = dv_out; p.dg = dg; p.dbeta = dbeta; p.dgate = dgate;
     p.ds0 = d_initial_state;
-    p.ckpt = (float *)workspace;
-    p.scratch = (float *)((char *)workspace + kda::ckpt_bytes(total_tokens, num_seqs, H, dk, dv));
-    p.N = num_seqs; p.H = H; p.DV = dv; p.T = total_tokens;
+    p.prep = (float *)(ws + w.prep);
+    p.Sst = (float *)(ws + w.S);
+    p.dSst = (float *)(ws + w.dS);
+    p.Ust = (float *)(ws + w.U);
+    p.dUst = (float *)(ws + w.dU);
+    p.N = num_seqs; p.H = H; p.T = total_tokens;
     p.scale = scale;
+    const long slots = total_tokens > 0 ? kda::slots_of(total_tokens, num_seqs) : 0;
+    cudaStream_t st = (cudaStream_t)stream;
     cudaError_t e;
     const bool bf = dtype == KDA_DTYPE_BF16;
     if (dk == 128)
-        e = bf ? kda::launch_bwd_t<128, __nv_bfloat16>(p, st) : kda::launch_bwd_t<128, float>(p, st);
+        e = bf ? kda::launch_bwd_dk<128, __nv_bfloat16>(p, dv, slots, st)
+               : kda::launch_bwd_dk<128, float>(p, dv, slots, st);
     else
-        e = bf ? kda::launch_bwd_t<64, __nv_bfloat16>(p, st) : kda::launch_bwd_t<64, float>(p, st);
+        e = bf ? kda::launch_bwd_dk<64, __nv_bfloat16>(p, dv, slots, st)
+               : kda::launch_bwd_dk<64, float>(p, dv, slots, st);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
