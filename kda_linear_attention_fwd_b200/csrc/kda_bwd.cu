@@ -33,7 +33,8 @@
 //   rev_chain     per (sequence, head, 16 columns), chunks in reverse: dS' and
 //                 dU -> workspace; dL/d(initial state)
 //   grad_kernel   per (chunk, head), parallel: the other gradients from the
-//                 chunk's inputs, S, dS', U and dU
+//                 chunk's inputs, S, dS', U and dU; its three products with a
+//                 whole state run on split-tf32 tensor-core tiles
 // Every output element is written by exactly one thread (no atomics), so the
 // results do not depend on scheduling.
 #include "kda.h"
@@ -67,8 +68,9 @@ struct BwdParams {
 };
 
 // Offsets (floats) inside one prep block: W, Qd, Kb [C][DK], U0 [C][DV],
-// P [C][C], gamma_C [DK].  Every offset and the block size are multiples of
-// four floats (dk, dv in {64, 128}), so 16-byte copies stay aligned.
+// P [C][C], gamma_C [DK].  Every offset and the block size are
+// multiples of four floats (dk, dv in {64, 128}), so 16-byte copies stay
+// aligned.
 template <int DK, int DV> struct Blk {
     static constexpr int W = 0, QD = C * DK, KB = 2 * C * DK, U0 = 3 * C * DK;
     static constexpr int P = U0 + C * DV, GC = P + C * C, size = GC + DK;
@@ -241,6 +243,36 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(BwdParams p) {
     }
     out[B::P + tid] = sm.P[tid >> 4][tid & 15];
     for (int i = tid; i < DK; i += kThreads) out[B::GC + i] = sm.gc[i];
+}
+
+// ---- split-tf32 tensor-core tiles (mma.sync m16n8k8) for the products of
+// grad_kernel that run over a whole state: fp32 accuracy from tf32 tiles by
+// splitting each operand as x = hi + lo and forming hi*hi + hi*lo + lo*hi
+// with fp32 accumulation (what is dropped is below 2^-20 relative).
+
+// x = hi + lo: hi = x with the 13 low mantissa bits cleared (a tf32 value), lo
+// = the exact remainder, of which the tensor core reads the tf32 part
+// (|lo| < 2^-10 |x|, so the representation error is below 2^-20 |x|)
+KDA_DEVICE void split_tf32(float x, uint32_t &hi, uint32_t &lo) {
+    hi = __float_as_uint(x) & 0xffffe000u;
+    lo = __float_as_uint(x - __uint_as_float(hi));
+}
+
+KDA_DEVICE void mma_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// d += A B for A = ah + al and B = (b0, b1) split here
+KDA_DEVICE void mma3(float (&d)[4], const uint32_t (&ah)[4], const uint32_t (&al)[4], float b0, float b1) {
+    uint32_t bh0, bl0, bh1, bl1;
+    split_tf32(b0, bh0, bl0);
+    split_tf32(b1, bh1, bl1);
+    mma_tf32(d, al, bh0, bh1);
+    mma_tf32(d, ah, bl0, bl1);
+    mma_tf32(d, ah, bh0, bh1);
 }
 
 // ---- the sequential passes: one CTA per (sequence, head, NC state columns).
@@ -452,22 +484,24 @@ __global__ void __launch_bounds__(kThreads) rev_chain(BwdParams p) {
 
 // ---- the per-chunk gradients: one CTA per (chunk, head)
 template <int DK, int DV> struct alignas(16) GradSm {
-    static constexpr int LK = DK + 4, LV = DV + 4, LM = PrepSm<DK, DV>::LM;
-    PrepSm<DK, DV> pr;
-    float us[C][LM];                   // U, then dKi
-    float dus[C][LV], dos[C][LV];      // dU, dO
+    static constexpr int LK = DK + 4;
+    static constexpr int NB = kThreads / DK;   // threads per key channel
+    static constexpr int LV = DV + 4;
+    PrepSm<DK, DV> pr;                         // its vs holds dV once V is used
+    float us[C][LV], dus[C][LV], dos[C][LV];   // U, dU, dO
     float dqd[C][LK], dw[C][LK], dkb[C][LK];
-    float dP[C][C + 1], dT[C][C + 1], M[C][C + 1], dL[C][C + 1];
-    float dgc[DK];                     // dgamma_C (.) gamma_C
+    float dP[C][C], dT[C][C], M[C][C], dLs[C][C], dA[C][C];
+    float dgc[DK];                             // dgamma_C (.) gamma_C
+    float bs[NB][DK], ks[NB][DK];              // per row block: sum of dG, colsum of dKb (.) Kb
 };
 
 template <int DK, int DV, typename T>
 __global__ void __launch_bounds__(kThreads, 2) grad_kernel(BwdParams p) {
-    constexpr int TPC = kThreads / DK;  // threads per key channel in the products with S
-    constexpr int JW = DV / TPC;        // their columns each
-    constexpr int RPT = C / TPC;        // rows per thread in the row-wise steps
+    using Sm = GradSm<DK, DV>;
+    constexpr int NB = Sm::NB;
+    constexpr int RPT = C / NB;  // rows per thread in the row-wise steps
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    auto &sm = *reinterpret_cast<GradSm<DK, DV> *>(smem_raw);
+    auto &sm = *reinterpret_cast<Sm *>(smem_raw);
     auto &pr = sm.pr;
     const long slot = blockIdx.x;
     const int h = blockIdx.y, tid = threadIdx.x, H = p.H;
@@ -493,45 +527,61 @@ __global__ void __launch_bounds__(kThreads, 2) grad_kernel(BwdParams p) {
     }
     prep_chunk<DK, DV, T>(p, pr, h, t0, n);  // ends with a barrier
 
-    {  // dQd = dO S^T, dW = -dU S^T, dKb = U dS'^T, dgamma_C = rowsum(dS' (.) S)
-        // the TPC threads of a channel take interleaved 4-column groups
-        const int i = tid / TPC, part = tid % TPC;
-        const float4 *S4 = reinterpret_cast<const float4 *>(p.Sst + idx * DK * DV + (size_t)i * DV);
-        const float4 *D4 = reinterpret_cast<const float4 *>(p.dSst + idx * DK * DV + (size_t)i * DV);
-        float aq[C], aw[C], ab[C], ag = 0.f;
+    {  // dQd = dO S^T, dW = -dU S^T, dKb = U dS'^T on tensor-core tiles (B[j][i] = S[i][j],
+       // the same split-tf32 products as the chains); warp w takes key channels
+       // 8 w NTG .. 8 (w + 1) NTG - 1; dgamma_C = rowsum(dS' (.) S) from the same loads
+        constexpr int NTG = DK / 8 / (kThreads / 32);
+        const int lane = tid & 31, warp = tid >> 5, g = lane >> 2, t = lane & 3;
+        const float *Sb = p.Sst + idx * DK * DV, *Db = p.dSst + idx * DK * DV;
+        float aq[NTG][4], aw[NTG][4], ab[NTG][4], ag[NTG];
 #pragma unroll
-        for (int r = 0; r < C; ++r) aq[r] = aw[r] = ab[r] = 0.f;
+        for (int nt = 0; nt < NTG; ++nt) {
+            ag[nt] = 0.f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) aq[nt][e] = aw[nt][e] = ab[nt][e] = 0.f;
+        }
 #pragma unroll 2
-        for (int c4 = 0; c4 < JW / 4; ++c4) {
-            const int j4 = c4 * TPC + part, jj = 4 * j4;
-            const float4 s4 = __ldg(S4 + j4), d4 = __ldg(D4 + j4);
-            ag = dot4(s4, d4, ag);
+        for (int kt = 0; kt < DV / 8; ++kt) {
+            const int j = 8 * kt + t;
+            uint32_t oh[4], ol[4], dh[4], dl[4], uh[4], ul[4];
+            split_tf32(sm.dos[g][j], oh[0], ol[0]);
+            split_tf32(sm.dos[g + 8][j], oh[1], ol[1]);
+            split_tf32(sm.dos[g][j + 4], oh[2], ol[2]);
+            split_tf32(sm.dos[g + 8][j + 4], oh[3], ol[3]);
+            split_tf32(sm.dus[g][j], dh[0], dl[0]);
+            split_tf32(sm.dus[g + 8][j], dh[1], dl[1]);
+            split_tf32(sm.dus[g][j + 4], dh[2], dl[2]);
+            split_tf32(sm.dus[g + 8][j + 4], dh[3], dl[3]);
+            split_tf32(sm.us[g][j], uh[0], ul[0]);
+            split_tf32(sm.us[g + 8][j], uh[1], ul[1]);
+            split_tf32(sm.us[g][j + 4], uh[2], ul[2]);
+            split_tf32(sm.us[g + 8][j + 4], uh[3], ul[3]);
 #pragma unroll
-            for (int r = 0; r < C; ++r) {
-                aq[r] = dot4(*reinterpret_cast<const float4 *>(&sm.dos[r][jj]), s4, aq[r]);
-                aw[r] = dot4(*reinterpret_cast<const float4 *>(&sm.dus[r][jj]), s4, aw[r]);
-                ab[r] = dot4(*reinterpret_cast<const float4 *>(&sm.us[r][jj]), d4, ab[r]);
+            for (int nt = 0; nt < NTG; ++nt) {
+                const size_t row = (size_t)(8 * (warp * NTG + nt) + g) * DV;
+                const float s0 = __ldg(Sb + row + j), s1 = __ldg(Sb + row + j + 4);
+                const float d0 = __ldg(Db + row + j), d1 = __ldg(Db + row + j + 4);
+                ag[nt] = fmaf(s0, d0, fmaf(s1, d1, ag[nt]));
+                mma3(aq[nt], oh, ol, s0, s1);
+                mma3(aw[nt], dh, dl, s0, s1);
+                mma3(ab[nt], uh, ul, d0, d1);
             }
         }
 #pragma unroll
-        for (int o = 1; o < TPC; o <<= 1) {
-            ag += __shfl_xor_sync(0xffffffffu, ag, o);
+        for (int nt = 0; nt < NTG; ++nt) {
+            const int ib = 8 * (warp * NTG + nt);
 #pragma unroll
-            for (int r = 0; r < C; ++r) {
-                aq[r] += __shfl_xor_sync(0xffffffffu, aq[r], o);
-                aw[r] += __shfl_xor_sync(0xffffffffu, aw[r], o);
-                ab[r] += __shfl_xor_sync(0xffffffffu, ab[r], o);
+            for (int e = 0; e < 4; ++e) {
+                const int r = g + 8 * (e >> 1), i = ib + 2 * t + (e & 1);
+                sm.dqd[r][i] = aq[nt][e];
+                sm.dw[r][i] = -aw[nt][e];
+                sm.dkb[r][i] = ab[nt][e];
             }
+            float a = ag[nt];  // row ib + g: the four lanes t hold interleaved columns
+            a += __shfl_xor_sync(0xffffffffu, a, 1);
+            a += __shfl_xor_sync(0xffffffffu, a, 2);
+            if (t == 0) sm.dgc[ib + g] = a * pr.gc[ib + g];
         }
-#pragma unroll
-        for (int r = 0; r < C; ++r) {
-            if (r % TPC == part) {
-                sm.dqd[r][i] = aq[r];
-                sm.dw[r][i] = -aw[r];
-                sm.dkb[r][i] = ab[r];
-            }
-        }
-        if (part == 0) sm.dgc[i] = ag * pr.gc[i];
     }
     __syncthreads();
     {  // dP = tril(dO U^T), dT = dU V^T + dW Kd^T: thread (r, s)
@@ -548,7 +598,8 @@ __global__ void __launch_bounds__(kThreads, 2) grad_kernel(BwdParams p) {
         for (int c4 = 0; c4 < DK / 4; ++c4)
             dt = dot4(*reinterpret_cast<const float4 *>(&sm.dw[r][4 * c4]),
                       *reinterpret_cast<const float4 *>(&pr.kd[s2][4 * c4]), dt);
-        sm.dP[r][s2] = r >= s2 ? dp : 0.f;
+        const float dpm = r >= s2 ? dp : 0.f;
+        sm.dP[r][s2] = dpm;
         sm.dT[r][s2] = dt;
     }
     __syncthreads();
@@ -559,74 +610,97 @@ __global__ void __launch_bounds__(kThreads, 2) grad_kernel(BwdParams p) {
         for (int q = 0; q < C; ++q) m = fmaf(pr.X[q][r], sm.dT[q][s2], m);
         sm.M[r][s2] = m * pr.beta[s2];
     }
-    // dV = T^T dU (rows < n)
-    for (int e = tid; e < C * DV; e += kThreads) {
+    for (int e = tid; e < C * DV; e += kThreads) {  // dV = T^T dU into vs (V is used up)
         const int r = e / DV, jj = e % DV;
         float d = 0.f;
 #pragma unroll
         for (int q = 0; q < C; ++q) d = fmaf(pr.Tm[q][r], sm.dus[q][jj], d);
-        if (r < n) p.dv[((size_t)(t0 + r) * H + h) * DV + jj] = d;
+        pr.vs[r][jj] = d;
     }
     __syncthreads();
-    {  // dL = -M X^T: thread (r, s)
+    {  // dL = -M X^T (strictly lower part); dA = Diag(beta) strict(dL): thread (r, s)
         const int r = tid >> 4, s2 = tid & 15;
         float l = 0.f;
 #pragma unroll
         for (int q = 0; q < C; ++q) l = fmaf(sm.M[r][q], pr.X[s2][q], l);
-        sm.dL[r][s2] = -l;
+        const float ls = r > s2 ? -l : 0.f;
+        sm.dLs[r][s2] = ls;
+        sm.dA[r][s2] = pr.beta[r] * ls;
     }
     __syncthreads();
     if (tid < n) {  // dbeta = colsum(X (.) dT) + rowsum(strict(dL) (.) A)
         const int r = tid;
         float db = 0.f;
 #pragma unroll
-        for (int q = 0; q < C; ++q) db = fmaf(pr.X[q][r], sm.dT[q][r], db);
-#pragma unroll
-        for (int q = 0; q < C; ++q) db = fmaf(sm.dL[r][q], pr.A[r][q], db);  // A is strictly lower
+        for (int q = 0; q < C; ++q) {
+            db = fmaf(pr.X[q][r], sm.dT[q][r], db);
+            db = fmaf(sm.dLs[r][q], pr.A[r][q], db);
+        }
         p.dbeta[(size_t)(t0 + r) * H + h] = db;
     }
-    {  // dKd = T^T dW + dA Ki, dKi = dA^T Kd + dP^T Qd, dQd += dP Ki; dA = Diag(beta) strict(dL)
-        const int i = tid % DK, r0 = (tid / DK) * RPT;
+    for (int e = tid; e < C * DV; e += kThreads) {
+        const int r = e / DV, jj = e % DV;
+        if (r < n) p.dv[((size_t)(t0 + r) * H + h) * DV + jj] = pr.vs[r][jj];
+    }
+    {  // dKd = T^T dW + dA Ki, dKi = dA^T Kd + dP^T Qd, dQd += dP Ki for rows
+       // r0 .. r0 + RPT - 1 of channel i; then dq, dk, dg
+        const int i = tid % DK, rb = tid / DK, r0 = rb * RPT;
+        float dkd[RPT], dki[RPT], dqd[RPT];
+#pragma unroll
+        for (int rr = 0; rr < RPT; ++rr) {
+            dkd[rr] = dki[rr] = 0.f;
+            dqd[rr] = sm.dqd[r0 + rr][i];
+        }
+#pragma unroll 4
+        for (int q = 0; q < C; ++q) {
+            const float dwq = sm.dw[q][i], kiq = pr.ki[q][i], kdq = pr.kd[q][i], qdq = pr.qd[q][i];
+#pragma unroll
+            for (int rr = 0; rr < RPT; ++rr) {  // r is the same across a warp: broadcast reads
+                const int r = r0 + rr;
+                dkd[rr] = fmaf(pr.Tm[q][r], dwq, dkd[rr]);  // T^T dW
+                dkd[rr] = fmaf(sm.dA[r][q], kiq, dkd[rr]);  // dA Ki
+                dki[rr] = fmaf(sm.dA[q][r], kdq, dki[rr]);  // dA^T Kd
+                dki[rr] = fmaf(sm.dP[q][r], qdq, dki[rr]);  // dP^T Qd
+                dqd[rr] = fmaf(sm.dP[r][q], kiq, dqd[rr]);  // dP Ki
+            }
+        }
+        float dG[RPT], bsum = 0.f, ksum = 0.f;
 #pragma unroll
         for (int rr = 0; rr < RPT; ++rr) {
             const int r = r0 + rr;
-            float dkd = 0.f, dki = 0.f, dqd = sm.dqd[r][i];
-#pragma unroll
-            for (int q = 0; q < C; ++q) {
-                dkd = fmaf(pr.Tm[q][r], sm.dw[q][i], dkd);
-                const float a_rq = q < r ? pr.beta[r] * sm.dL[r][q] : 0.f;   // dA[r][q]
-                const float a_qr = q > r ? pr.beta[q] * sm.dL[q][r] : 0.f;   // dA[q][r]
-                dkd = fmaf(a_rq, pr.ki[q][i], dkd);
-                dki = fmaf(a_qr, pr.kd[q][i], dki);
-                dki = fmaf(sm.dP[q][r], pr.qd[q][i], dki);
-                dqd = fmaf(sm.dP[r][q], pr.ki[q][i], dqd);
-            }
-            pr.vs[r][i] = dkd;  // V is no longer needed
-            sm.us[r][i] = dki;  // nor U
-            sm.dqd[r][i] = dqd;
+            const float kb = pr.kb[r][i], dkb = sm.dkb[r][i];
+            dG[rr] = dkd[rr] * pr.kd[r][i] - dki[rr] * pr.ki[r][i] + dqd[rr] * pr.qd[r][i] - dkb * kb;
+            bsum += dG[rr];
+            ksum = fmaf(dkb, kb, ksum);
         }
-    }
-    __syncthreads();
-    if (tid < DK) {  // dq, dk, dg down the rows from the bottom
-        const int i = tid;
-        const float GC = pr.gs[C - 1][i];
+        sm.bs[rb][i] = bsum;
+        sm.ks[rb][i] = ksum;
+        __syncthreads();
+        // dg_r = dgamma_C gamma_C + colsum(dKb (.) Kb) + sum of dG over rows >= r
         float acc = sm.dgc[i];
 #pragma unroll
-        for (int r = 0; r < C; ++r) acc = fmaf(sm.dkb[r][i], pr.kb[r][i], acc);
-        for (int r = C - 1; r >= 0; --r) {
-            const float Gr = pr.gs[r][i];
-            const float dkd = pr.vs[r][i], dki = sm.us[r][i], dqd = sm.dqd[r][i], dkb = sm.dkb[r][i];
-            acc += dkd * pr.kd[r][i] - dki * pr.ki[r][i] + dqd * pr.qd[r][i] - dkb * pr.kb[r][i];
+        for (int b = 0; b < NB; ++b) {
+            acc += sm.ks[b][i];
+            if (b > rb) acc += sm.bs[b][i];
+        }
+        const float GC = pr.gs[C - 1][i];
+#pragma unroll
+        for (int rr = RPT - 1; rr >= 0; --rr) {
+            const int r = r0 + rr;
+            acc += dG[rr];
             if (r < n) {
+                const float Gr = pr.gs[r][i], e = expf(Gr);
                 const size_t o = ((size_t)(t0 + r) * H + h) * DK + i;
-                const float e = expf(Gr);
-                p.dk[o] = dkd * e + dki * expf(-Gr) + dkb * expf(GC - Gr);
-                p.dq[o] = p.scale * dqd * e;
+                p.dk[o] = dkd[rr] * e + dki[rr] * expf(-Gr) + sm.dkb[r][i] * expf(GC - Gr);
+                p.dq[o] = p.scale * dqd[rr] * e;
                 p.dg[o] = acc;
             }
         }
     }
 }
+
+// two CTAs of grad_kernel per SM (228 KB of shared memory, 1 KB reserved per CTA)
+static_assert(sizeof(GradSm<128, 128>) + 1024 <= 228 * 1024 / 2, "grad_kernel: two CTAs per SM");
 
 template <typename K> cudaError_t set_smem(K kernel, size_t bytes) {
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
