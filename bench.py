@@ -520,10 +520,10 @@ def main():
                             "fp32 gradients, final-state gradient given",
                 "roofline": {"bound": "hbm", "achieved": bgbs, "peak": hbm, "unit": "GB/s",
                              "frac": bgbs / hbm, "traffic": None,
-                             "kernel": "kda_bwd call (prep, forward chain, reverse chain, "
-                                       "per-chunk gradients)",
+                             "kernel": "kda_bwd call (per-chunk operands, the forward and "
+                                       "reverse chains in one launch, per-chunk gradients)",
                              "peak_source": f"{pk_kind} hbm_gbs"},
-                "gpu_launches": 4 * args.steps}
+                "gpu_launches": 3 * args.steps}
         del bi, dyb, dsfb, gq, gk, gg, gv, ggt, gbt, gs0, wsb
 
     # ---------------- decode ----------------

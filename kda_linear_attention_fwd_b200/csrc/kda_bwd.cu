@@ -26,11 +26,12 @@
 //   dG = dKd (.) Kd - dKi (.) Ki + dQd (.) Qd - dKb (.) Kb; the last row adds
 //        colsum(dKb (.) Kb) + dgamma_C (.) gamma_C;  dg = suffix sums of dG over the rows
 //
-// Four launches, all fp32 arithmetic on bf16 or fp32 inputs:
+// Three launches, all fp32 arithmetic on bf16 or fp32 inputs:
 //   prep_kernel   per (chunk, head), parallel: W, Qd, Kb, U0, P, gamma_C -> workspace
-//   fwd_chain     per (sequence, head, 16 state columns), chunks in order: the
+//   chain_kernel  two independent sequential passes side by side:
+//     fwd_chain   per (sequence, head, 16 state columns), chunks in order: the
 //                 state entering each chunk and U -> workspace; dgate = dy (.) O
-//   rev_chain     per (sequence, head, 16 columns), chunks in reverse: dS' and
+//     rev_chain   per (sequence, head, 16 columns), chunks in reverse: dS' and
 //                 dU -> workspace; dL/d(initial state)
 //   grad_kernel   per (chunk, head), parallel: the other gradients from the
 //                 chunk's inputs, S, dS', U and dU; its three products with a
@@ -340,11 +341,9 @@ template <int R> KDA_DEVICE void axpy_rows(const float *seg, float c, float (&x)
 // Forward pass over the chunks of one sequence: stores the state entering
 // each chunk and U; dgate = dy (.) O.
 template <int DK, int DV, typename T>
-__global__ void __launch_bounds__(kThreads) fwd_chain(BwdParams p) {
+KDA_DEVICE void fwd_chain(const BwdParams &p, ChainSm<DK> &sm) {
     constexpr int R = DK / 16;
     using B = Blk<DK, DV>;
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    auto &sm = *reinterpret_cast<ChainSm<DK> *>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int j = tid & 15, rg = tid >> 4, i0 = rg * R;
     const int nh = blockIdx.x, n = nh / p.H, h = nh % p.H, H = p.H;
@@ -410,11 +409,9 @@ __global__ void __launch_bounds__(kThreads) fwd_chain(BwdParams p) {
 // Reverse pass over the chunks of one sequence: stores dL/d(state leaving
 // each chunk) and dU; writes dL/d(initial state).
 template <int DK, int DV, typename T>
-__global__ void __launch_bounds__(kThreads) rev_chain(BwdParams p) {
+KDA_DEVICE void rev_chain(const BwdParams &p, ChainSm<DK> &sm) {
     constexpr int R = DK / 16;
     using B = Blk<DK, DV>;
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    auto &sm = *reinterpret_cast<ChainSm<DK> *>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int j = tid & 15, rg = tid >> 4, i0 = rg * R;
     const int nh = blockIdx.x, n = nh / p.H, h = nh % p.H, H = p.H;
@@ -480,6 +477,17 @@ __global__ void __launch_bounds__(kThreads) rev_chain(BwdParams p) {
 #pragma unroll
         for (int m = 0; m < R; ++m) p.ds0[((size_t)nh * DK + i0 + m) * DV + j0 + j] = dS[m];
     }
+}
+
+// The two passes are independent (the reverse one needs the prep blocks and
+// dO, not the forward states), so one launch runs both: blockIdx.z = 0 the
+// forward pass, 1 the reverse pass.
+template <int DK, int DV, typename T>
+__global__ void __launch_bounds__(kThreads) chain_kernel(BwdParams p) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    auto &sm = *reinterpret_cast<ChainSm<DK> *>(smem_raw);
+    if (blockIdx.z == 0) fwd_chain<DK, DV, T>(p, sm);
+    else rev_chain<DK, DV, T>(p, sm);
 }
 
 // ---- the per-chunk gradients: one CTA per (chunk, head)
@@ -709,15 +717,13 @@ template <typename K> cudaError_t set_smem(K kernel, size_t bytes) {
 template <int DK, int DV, typename T>
 cudaError_t launch_bwd_t(const BwdParams &p, long slots, cudaStream_t st) {
     static_assert(C * C == kThreads, "prep_kernel writes P with one thread per entry");
-    const dim3 per_chunk((unsigned)slots, (unsigned)p.H), per_seq((unsigned)(p.N * p.H), DV / NC);
+    const dim3 per_chunk((unsigned)slots, (unsigned)p.H), per_seq((unsigned)(p.N * p.H), DV / NC, 2);
     cudaError_t e;
     if ((e = set_smem(prep_kernel<DK, DV, T>, sizeof(PrepSm<DK, DV>))) != cudaSuccess) return e;
-    if ((e = set_smem(fwd_chain<DK, DV, T>, sizeof(ChainSm<DK>))) != cudaSuccess) return e;
-    if ((e = set_smem(rev_chain<DK, DV, T>, sizeof(ChainSm<DK>))) != cudaSuccess) return e;
+    if ((e = set_smem(chain_kernel<DK, DV, T>, sizeof(ChainSm<DK>))) != cudaSuccess) return e;
     if ((e = set_smem(grad_kernel<DK, DV, T>, sizeof(GradSm<DK, DV>))) != cudaSuccess) return e;
     if (slots > 0) prep_kernel<DK, DV, T><<<per_chunk, kThreads, sizeof(PrepSm<DK, DV>), st>>>(p);
-    fwd_chain<DK, DV, T><<<per_seq, kThreads, sizeof(ChainSm<DK>), st>>>(p);
-    rev_chain<DK, DV, T><<<per_seq, kThreads, sizeof(ChainSm<DK>), st>>>(p);
+    chain_kernel<DK, DV, T><<<per_seq, kThreads, sizeof(ChainSm<DK>), st>>>(p);
     if (slots > 0) grad_kernel<DK, DV, T><<<per_chunk, kThreads, sizeof(GradSm<DK, DV>), st>>>(p);
     return cudaGetLastError();
 }
