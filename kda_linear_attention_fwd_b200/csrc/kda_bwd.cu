@@ -499,7 +499,7 @@ template <int DK, int DV> struct alignas(16) GradSm {
     float us[C][LV], dus[C][LV], dos[C][LV];   // U, dU, dO
     float dqd[C][LK], dw[C][LK], dkb[C][LK];
     float dP[C][C], dT[C][C], M[C][C], dLs[C][C], dA[C][C];
-    float dgc[DK];                             // dgamma_C (.) gamma_C
+    float dgc[DK];                             // dgamma_C
     float bs[NB][DK], ks[NB][DK];              // per row block: sum of dG, colsum of dKb (.) Kb
 };
 
@@ -533,14 +533,25 @@ __global__ void __launch_bounds__(kThreads, 2) grad_kernel(BwdParams p) {
         }
         sm.dos[r][jj] = d;
     }
-    prep_chunk<DK, DV, T>(p, pr, h, t0, n);  // ends with a barrier
-
-    {  // dQd = dO S^T, dW = -dU S^T, dKb = U dS'^T on tensor-core tiles (B[j][i] = S[i][j],
-       // the same split-tf32 products as the chains); warp w takes key channels
-       // 8 w NTG .. 8 (w + 1) NTG - 1; dgamma_C = rowsum(dS' (.) S) from the same loads
+    // dQd = dO S^T, dW = -dU S^T, dKb = U dS'^T on split-tf32 tensor-core tiles
+    // (B[j][i] = S[i][j]); warp w takes key channels 8 w NTG .. 8 (w + 1) NTG - 1;
+    // dgamma_C = rowsum(dS' (.) S) from the same operands.  This runs before the
+    // chunk's own operands are formed: their shared memory meanwhile stages S
+    // and dS' in blocks of 16 columns (cp.async, two blocks in flight).
+    {
         constexpr int NTG = DK / 8 / (kThreads / 32);
-        const int lane = tid & 31, warp = tid >> 5, g = lane >> 2, t = lane & 3;
+        constexpr int JB = 16, LS = JB + 4;  // columns per staged block; row stride (floats)
+        static_assert(2 * 2 * DK * LS * sizeof(float) <= sizeof(PrepSm<DK, DV>), "staging fits");
+        float(*stage)[2][DK][LS] = reinterpret_cast<float(*)[2][DK][LS]>(&pr);  // [buffer][S, dS'][i][j]
         const float *Sb = p.Sst + idx * DK * DV, *Db = p.dSst + idx * DK * DV;
+        auto fetch = [&](int blk, int buf) {
+            for (int e = tid; e < 2 * DK * JB / 4; e += kThreads) {
+                const int m = e / (DK * JB / 4), i = (e / (JB / 4)) % DK, c4 = e % (JB / 4);
+                cp_async16(&stage[buf][m][i][4 * c4], (m ? Db : Sb) + (size_t)i * DV + blk * JB + 4 * c4, true);
+            }
+            cp_async_commit();
+        };
+        const int lane = tid & 31, warp = tid >> 5, g = lane >> 2, t = lane & 3;
         float aq[NTG][4], aw[NTG][4], ab[NTG][4], ag[NTG];
 #pragma unroll
         for (int nt = 0; nt < NTG; ++nt) {
@@ -548,31 +559,38 @@ __global__ void __launch_bounds__(kThreads, 2) grad_kernel(BwdParams p) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) aq[nt][e] = aw[nt][e] = ab[nt][e] = 0.f;
         }
-#pragma unroll 2
-        for (int kt = 0; kt < DV / 8; ++kt) {
-            const int j = 8 * kt + t;
-            uint32_t oh[4], ol[4], dh[4], dl[4], uh[4], ul[4];
-            split_tf32(sm.dos[g][j], oh[0], ol[0]);
-            split_tf32(sm.dos[g + 8][j], oh[1], ol[1]);
-            split_tf32(sm.dos[g][j + 4], oh[2], ol[2]);
-            split_tf32(sm.dos[g + 8][j + 4], oh[3], ol[3]);
-            split_tf32(sm.dus[g][j], dh[0], dl[0]);
-            split_tf32(sm.dus[g + 8][j], dh[1], dl[1]);
-            split_tf32(sm.dus[g][j + 4], dh[2], dl[2]);
-            split_tf32(sm.dus[g + 8][j + 4], dh[3], dl[3]);
-            split_tf32(sm.us[g][j], uh[0], ul[0]);
-            split_tf32(sm.us[g + 8][j], uh[1], ul[1]);
-            split_tf32(sm.us[g][j + 4], uh[2], ul[2]);
-            split_tf32(sm.us[g + 8][j + 4], uh[3], ul[3]);
+        fetch(0, 0);
+        for (int blk = 0; blk < DV / JB; ++blk) {
+            cp_async_wait<0>();
+            __syncthreads();  // block blk landed; buffer (blk + 1) & 1 is free
+            if (blk + 1 < DV / JB) fetch(blk + 1, (blk + 1) & 1);
+            const auto &st = stage[blk & 1];
 #pragma unroll
-            for (int nt = 0; nt < NTG; ++nt) {
-                const size_t row = (size_t)(8 * (warp * NTG + nt) + g) * DV;
-                const float s0 = __ldg(Sb + row + j), s1 = __ldg(Sb + row + j + 4);
-                const float d0 = __ldg(Db + row + j), d1 = __ldg(Db + row + j + 4);
-                ag[nt] = fmaf(s0, d0, fmaf(s1, d1, ag[nt]));
-                mma3(aq[nt], oh, ol, s0, s1);
-                mma3(aw[nt], dh, dl, s0, s1);
-                mma3(ab[nt], uh, ul, d0, d1);
+            for (int kk = 0; kk < JB / 8; ++kk) {
+                const int j = blk * JB + 8 * kk + t, jl = 8 * kk + t;
+                uint32_t oh[4], ol[4], dh[4], dl[4], uh[4], ul[4];
+                split_tf32(sm.dos[g][j], oh[0], ol[0]);
+                split_tf32(sm.dos[g + 8][j], oh[1], ol[1]);
+                split_tf32(sm.dos[g][j + 4], oh[2], ol[2]);
+                split_tf32(sm.dos[g + 8][j + 4], oh[3], ol[3]);
+                split_tf32(sm.dus[g][j], dh[0], dl[0]);
+                split_tf32(sm.dus[g + 8][j], dh[1], dl[1]);
+                split_tf32(sm.dus[g][j + 4], dh[2], dl[2]);
+                split_tf32(sm.dus[g + 8][j + 4], dh[3], dl[3]);
+                split_tf32(sm.us[g][j], uh[0], ul[0]);
+                split_tf32(sm.us[g + 8][j], uh[1], ul[1]);
+                split_tf32(sm.us[g][j + 4], uh[2], ul[2]);
+                split_tf32(sm.us[g + 8][j + 4], uh[3], ul[3]);
+#pragma unroll
+                for (int nt = 0; nt < NTG; ++nt) {
+                    const int i = 8 * (warp * NTG + nt) + g;
+                    const float s0 = st[0][i][jl], s1 = st[0][i][jl + 4];
+                    const float d0 = st[1][i][jl], d1 = st[1][i][jl + 4];
+                    ag[nt] = fmaf(s0, d0, fmaf(s1, d1, ag[nt]));
+                    mma3(aq[nt], oh, ol, s0, s1);
+                    mma3(aw[nt], dh, dl, s0, s1);
+                    mma3(ab[nt], uh, ul, d0, d1);
+                }
             }
         }
 #pragma unroll
@@ -588,9 +606,11 @@ __global__ void __launch_bounds__(kThreads, 2) grad_kernel(BwdParams p) {
             float a = ag[nt];  // row ib + g: the four lanes t hold interleaved columns
             a += __shfl_xor_sync(0xffffffffu, a, 1);
             a += __shfl_xor_sync(0xffffffffu, a, 2);
-            if (t == 0) sm.dgc[ib + g] = a * pr.gc[ib + g];
+            if (t == 0) sm.dgc[ib + g] = a;  // times gamma_C once the operands are formed
         }
     }
+    __syncthreads();  // the staging area becomes the chunk's operands
+    prep_chunk<DK, DV, T>(p, pr, h, t0, n);  // ends with a barrier
     __syncthreads();
     {  // dP = tril(dO U^T), dT = dU V^T + dW Kd^T: thread (r, s)
         const int r = tid >> 4, s2 = tid & 15;
@@ -685,7 +705,7 @@ __global__ void __launch_bounds__(kThreads, 2) grad_kernel(BwdParams p) {
         sm.ks[rb][i] = ksum;
         __syncthreads();
         // dg_r = dgamma_C gamma_C + colsum(dKb (.) Kb) + sum of dG over rows >= r
-        float acc = sm.dgc[i];
+        float acc = sm.dgc[i] * pr.gc[i];
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
             acc += sm.ks[b][i];
