@@ -138,24 +138,40 @@ KDA_DEVICE void prep_chunk(const BwdParams &p, PrepSm<DK, DV> &sm, int h, int t0
     const int tid = threadIdx.x, H = p.H;
     const T *q = (const T *)p.q, *k = (const T *)p.k, *g = (const T *)p.g;
     const T *v = (const T *)p.v, *beta = (const T *)p.beta;
-    for (int e = tid; e < C * DK; e += kThreads) {
-        const int r = e / DK, i = e % DK;
-        float kv = 0.f, qv = 0.f, gv = 0.f;
+    // all of a thread's loads are issued before its first shared-memory store
+    constexpr int NK = C * DK / kThreads, NV = C * DV / kThreads;
+    static_assert(NK * kThreads == C * DK && NV * kThreads == C * DV, "whole rows per pass");
+    float kv[NK], qv[NK], gv[NK], vv[NV];
+#pragma unroll
+    for (int u = 0; u < NK; ++u) {
+        const int e = tid + u * kThreads, r = e / DK, i = e % DK;
+        kv[u] = qv[u] = gv[u] = 0.f;
         if (r < n) {
             const size_t o = ((size_t)(t0 + r) * H + h) * DK + i;
-            kv = ld(k + o);
-            qv = ld(q + o);
-            gv = ld(g + o);
+            kv[u] = ld(k + o);
+            qv[u] = ld(q + o);
+            gv[u] = ld(g + o);
         }
-        sm.kd[r][i] = kv;
-        sm.qd[r][i] = qv;
-        sm.gs[r][i] = gv;
     }
-    for (int e = tid; e < C * DV; e += kThreads) {
-        const int r = e / DV, j = e % DV;
-        sm.vs[r][j] = r < n ? ld(v + ((size_t)(t0 + r) * H + h) * DV + j) : 0.f;
+#pragma unroll
+    for (int u = 0; u < NV; ++u) {
+        const int e = tid + u * kThreads, r = e / DV, j = e % DV;
+        vv[u] = r < n ? ld(v + ((size_t)(t0 + r) * H + h) * DV + j) : 0.f;
     }
-    if (tid < C) sm.beta[tid] = tid < n ? ld(beta + (size_t)(t0 + tid) * H + h) : 0.f;
+    const float bv = tid < n ? ld(beta + (size_t)(t0 + tid) * H + h) : 0.f;
+#pragma unroll
+    for (int u = 0; u < NK; ++u) {
+        const int e = tid + u * kThreads, r = e / DK, i = e % DK;
+        sm.kd[r][i] = kv[u];
+        sm.qd[r][i] = qv[u];
+        sm.gs[r][i] = gv[u];
+    }
+#pragma unroll
+    for (int u = 0; u < NV; ++u) {
+        const int e = tid + u * kThreads;
+        sm.vs[e / DV][e % DV] = vv[u];
+    }
+    if (tid < C) sm.beta[tid] = bv;
     __syncthreads();
     if (tid < DK) {  // decay: one thread per key channel, down the rows
         const int i = tid;
@@ -520,18 +536,27 @@ __global__ void __launch_bounds__(kThreads, 2) grad_kernel(BwdParams p) {
     const size_t idx = (size_t)slot * H + h;
     const T *dy = (const T *)p.dy, *gate = (const T *)p.gate;
 
-    // U, dU (workspace) and dO = gate (.) dy
-    for (int e = tid; e < C * DV; e += kThreads) {
-        const int r = e / DV, jj = e % DV;
-        sm.us[r][jj] = p.Ust[idx * C * DV + e];
-        sm.dus[r][jj] = p.dUst[idx * C * DV + e];
-        float d = 0.f;
-        if (r < n) {
-            const size_t o = ((size_t)(t0 + r) * H + h) * DV + jj;
-            d = ld(dy + o);
-            if (gate) d *= ld(gate + o);
+    {  // U, dU (workspace) and dO = gate (.) dy; loads first, then the stores
+        constexpr int NV = C * DV / kThreads;
+        float uv[NV], duv[NV], dov[NV];
+#pragma unroll
+        for (int u = 0; u < NV; ++u) {
+            const int e = tid + u * kThreads, r = e / DV, jj = e % DV;
+            uv[u] = p.Ust[idx * C * DV + e];
+            duv[u] = p.dUst[idx * C * DV + e];
+            dov[u] = 0.f;
+            if (r < n) {
+                const size_t o = ((size_t)(t0 + r) * H + h) * DV + jj;
+                dov[u] = gate ? ld(dy + o) * ld(gate + o) : ld(dy + o);
+            }
         }
-        sm.dos[r][jj] = d;
+#pragma unroll
+        for (int u = 0; u < NV; ++u) {
+            const int e = tid + u * kThreads, r = e / DV, jj = e % DV;
+            sm.us[r][jj] = uv[u];
+            sm.dus[r][jj] = duv[u];
+            sm.dos[r][jj] = dov[u];
+        }
     }
     // dQd = dO S^T, dW = -dU S^T, dKb = U dS'^T on split-tf32 tensor-core tiles
     // (B[j][i] = S[i][j]); warp w takes key channels 8 w NTG .. 8 (w + 1) NTG - 1;
