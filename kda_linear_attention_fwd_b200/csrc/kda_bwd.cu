@@ -29,9 +29,9 @@
 // Three launches, all fp32 arithmetic on bf16 or fp32 inputs:
 //   prep_kernel   per (chunk, head), parallel: W, Qd, Kb, U0, P, gamma_C -> workspace
 //   chain_kernel  two independent sequential passes side by side:
-//     fwd_chain   per (sequence, head, 16 state columns), chunks in order: the
+//     fwd_chain   per (sequence, head, 32 state columns), chunks in order: the
 //                 state entering each chunk and U -> workspace; dgate = dy (.) O
-//     rev_chain   per (sequence, head, 16 columns), chunks in reverse: dS' and
+//     rev_chain   per (sequence, head, 32 columns), chunks in reverse: dS' and
 //                 dU -> workspace; dL/d(initial state)
 //   grad_kernel   per (chunk, head), parallel: the other gradients from the
 //                 chunk's inputs, S, dS', U and dU; its three products with a
@@ -52,7 +52,9 @@ using sm100::cp_async_wait;
 constexpr int C = 16;          // tokens per chunk
 constexpr int kThreads = 256;  // every launch
 constexpr int kWarps = kThreads / 32;
-constexpr int NC = 16;         // state columns of one chain CTA
+constexpr int NC = 16;         // state columns of one half of a chain CTA
+constexpr int kHalves = 2;     // chain CTAs: two halves of 256 threads share the chunk operands
+constexpr int kChainThreads = kHalves * kThreads;
 
 struct BwdParams {
     const void *q, *k, *v, *g, *beta, *gate, *dy;
@@ -292,38 +294,41 @@ KDA_DEVICE void mma3(float (&d)[4], const uint32_t (&ah)[4], const uint32_t (&al
     mma_tf32(d, ah, bh0, bh1);
 }
 
-// ---- the sequential passes: one CTA per (sequence, head, NC state columns).
-// Thread t owns column j = t % 16 of the slice and rows rg R .. rg R + R - 1
-// (rg = t / 16, R = DK / 16) of the state (or of its gradient) in registers;
-// for the chunk's [C][NC] outputs it is thread (r, j) with r = rg.  Sums over
-// the key channels: the two row groups of a warp are added with one shuffle,
-// then the eight warps through shared memory.
+// ---- the sequential passes: one CTA per (sequence, head, 2 NC state
+// columns), two halves of 256 threads with NC columns each that share one copy
+// of the chunk operands.  In a half, thread t owns column j = t % 16 and rows
+// rg R .. rg R + R - 1 (rg = t / 16, R = DK / 16) of the state (or of its
+// gradient) in registers; for the chunk's [C][NC] outputs it is thread (r, j)
+// with r = rg.  Sums over the key channels: the two row groups of a warp are
+// added with one shuffle, then the eight warps of the half through shared
+// memory.
 template <int DK> struct alignas(16) ChainSm {
     struct Buf {                   // one chunk's prep block (the rows this CTA needs)
         float wqk[3 * C * DK];     // W, Qd, Kb: [C][DK] each
         float pg[C * C + DK];      // P [C][C], gamma_C [DK]
-        float u0[C * NC];          // forward pass: U0 columns of this CTA
+        float u0[C * kHalves * NC];  // forward pass: U0 columns of this CTA, [C][2 NC]
         KDA_DEVICE const float *w() const { return wqk; }
         KDA_DEVICE const float *qd() const { return wqk + C * DK; }
         KDA_DEVICE const float *kb() const { return wqk + 2 * C * DK; }
         KDA_DEVICE const float *pm() const { return pg; }
         KDA_DEVICE const float *gc() const { return pg + C * C; }
     } buf[2];
-    float red[kWarps][C][32];      // partial sums per warp
-    float xs[2][C][NC];            // reverse pass: dO of the chunk (by iteration parity)
-    float us[C][NC];               // U (forward) or dU (reverse) of the chunk
+    float red[kHalves][kWarps][C][32];  // partial sums per warp
+    float xs[kHalves][2][C][NC];        // reverse pass: dO of the chunk (by iteration parity)
+    float us[kHalves][C][NC];           // U (forward) or dU (reverse) of the chunk
 };
 
 // cp.async of chunk prep block `blk` into `b` (one group).
 template <int DK, int DV>
 KDA_DEVICE void fetch_prep(typename ChainSm<DK>::Buf &b, const float *blk, int j0, bool with_u0) {
     using B = Blk<DK, DV>;
+    constexpr int NW = kHalves * NC;  // columns of the CTA
     const int tid = threadIdx.x;
-    for (int e = tid; e < 3 * C * DK / 4; e += kThreads) cp_async16(b.wqk + 4 * e, blk + B::W + 4 * e, true);
-    for (int e = tid; e < (C * C + DK) / 4; e += kThreads) cp_async16(b.pg + 4 * e, blk + B::P + 4 * e, true);
-    if (with_u0 && tid < C * NC / 4) {
-        const int r = tid / (NC / 4), c4 = tid % (NC / 4);
-        cp_async16(b.u0 + r * NC + 4 * c4, blk + B::U0 + r * DV + j0 + 4 * c4, true);
+    for (int e = tid; e < 3 * C * DK / 4; e += kChainThreads) cp_async16(b.wqk + 4 * e, blk + B::W + 4 * e, true);
+    for (int e = tid; e < (C * C + DK) / 4; e += kChainThreads) cp_async16(b.pg + 4 * e, blk + B::P + 4 * e, true);
+    if (with_u0 && tid < C * NW / 4) {
+        const int r = tid / (NW / 4), c4 = tid % (NW / 4);
+        cp_async16(b.u0 + r * NW + 4 * c4, blk + B::U0 + r * DV + j0 + 4 * c4, true);
     }
     cp_async_commit();
 }
@@ -360,10 +365,12 @@ template <int DK, int DV, typename T>
 KDA_DEVICE void fwd_chain(const BwdParams &p, ChainSm<DK> &sm) {
     constexpr int R = DK / 16;
     using B = Blk<DK, DV>;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int hv = threadIdx.x / kThreads, tid = threadIdx.x % kThreads, lane = tid & 31, warp = tid >> 5;
     const int j = tid & 15, rg = tid >> 4, i0 = rg * R;
     const int nh = blockIdx.x, n = nh / p.H, h = nh % p.H, H = p.H;
-    const int j0 = blockIdx.y * NC;
+    const int jc = blockIdx.y * kHalves * NC, j0 = jc + hv * NC;  // the CTA's and the half's first column
+    auto &red = sm.red[hv];
+    auto &us = sm.us[hv];
     const Seq s = seq_of(p, n);
     const T *dy = (const T *)p.dy;
     float S[R];
@@ -375,13 +382,13 @@ KDA_DEVICE void fwd_chain(const BwdParams &p, ChainSm<DK> &sm) {
         const int r = c * C + rg;
         return (p.dgate && r < s.len) ? ld(dy + ((size_t)(s.bos + r) * H + h) * DV + j0 + j) : 0.f;
     };
-    fetch_prep<DK, DV>(sm.buf[0], blk(0), j0, true);
+    fetch_prep<DK, DV>(sm.buf[0], blk(0), jc, true);
     float dyv = load_dy(0);
     for (int c = 0; c < s.nb; ++c) {
         const auto &b = sm.buf[c & 1];
         cp_async_wait<0>();
         __syncthreads();
-        if (c + 1 < s.nb) fetch_prep<DK, DV>(sm.buf[(c + 1) & 1], blk(c + 1), j0, true);
+        if (c + 1 < s.nb) fetch_prep<DK, DV>(sm.buf[(c + 1) & 1], blk(c + 1), jc, true);
         const size_t idx = (size_t)(s.slot0 + c) * H + h;
         float *Sg = p.Sst + idx * DK * DV + (size_t)i0 * DV + j0 + j;
 #pragma unroll
@@ -394,22 +401,22 @@ KDA_DEVICE void fwd_chain(const BwdParams &p, ChainSm<DK> &sm) {
             const float pu = dot_rows<R>(b.w() + r * DK + i0, S);
             const float pq = dot_rows<R>(b.qd() + r * DK + i0, S);
             const float send = hi ? pu : pq, keep = hi ? pq : pu;
-            sm.red[warp][r][lane] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+            red[warp][r][lane] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
         }
         __syncthreads();
         float u = 0.f, qs = 0.f;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) {
-            u += sm.red[w][rg][j];
-            qs += sm.red[w][rg][16 + j];
+            u += red[w][rg][j];
+            qs += red[w][rg][16 + j];
         }
-        u = b.u0[rg * NC + j] - u;
-        sm.us[rg][j] = u;
+        u = b.u0[rg * kHalves * NC + hv * NC + j] - u;
+        us[rg][j] = u;
         p.Ust[idx * C * DV + (size_t)rg * DV + j0 + j] = u;
         __syncthreads();
         float o = qs;  // O = Qd S + P U (P is zero above the diagonal)
 #pragma unroll
-        for (int r2 = 0; r2 < C; ++r2) o = fmaf(b.pm()[rg * C + r2], sm.us[r2][j], o);
+        for (int r2 = 0; r2 < C; ++r2) o = fmaf(b.pm()[rg * C + r2], us[r2][j], o);
         if (p.dgate && c * C + rg < s.len)
             p.dgate[((size_t)(s.bos + c * C + rg) * H + h) * DV + j0 + j] = dyv * o;
         if (c + 1 < s.nb) dyv = load_dy(c + 1);
@@ -418,7 +425,7 @@ KDA_DEVICE void fwd_chain(const BwdParams &p, ChainSm<DK> &sm) {
 #pragma unroll
         for (int m = 0; m < R; ++m) S[m] *= gc[m];
 #pragma unroll
-        for (int r = 0; r < C; ++r) axpy_rows<R>(b.kb() + r * DK + i0, sm.us[r][j], S);
+        for (int r = 0; r < C; ++r) axpy_rows<R>(b.kb() + r * DK + i0, us[r][j], S);
     }
 }
 
@@ -428,10 +435,12 @@ template <int DK, int DV, typename T>
 KDA_DEVICE void rev_chain(const BwdParams &p, ChainSm<DK> &sm) {
     constexpr int R = DK / 16;
     using B = Blk<DK, DV>;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int hv = threadIdx.x / kThreads, tid = threadIdx.x % kThreads, lane = tid & 31, warp = tid >> 5;
     const int j = tid & 15, rg = tid >> 4, i0 = rg * R;
     const int nh = blockIdx.x, n = nh / p.H, h = nh % p.H, H = p.H;
-    const int j0 = blockIdx.y * NC;
+    const int jc = blockIdx.y * kHalves * NC, j0 = jc + hv * NC;  // the CTA's and the half's first column
+    auto &red = sm.red[hv];
+    auto &us = sm.us[hv];
     const Seq s = seq_of(p, n);
     const T *dy = (const T *)p.dy, *gate = (const T *)p.gate;
     float dS[R];
@@ -445,15 +454,16 @@ KDA_DEVICE void rev_chain(const BwdParams &p, ChainSm<DK> &sm) {
         const float d = ld(dy + o);
         return gate ? ld(gate + o) * d : d;
     };
-    if (s.nb > 0) fetch_prep<DK, DV>(sm.buf[0], blk(s.nb - 1), j0, false);
+    auto &xs = sm.xs[hv];
+    if (s.nb > 0) fetch_prep<DK, DV>(sm.buf[0], blk(s.nb - 1), jc, false);
     float dov = s.nb > 0 ? load_do(s.nb - 1) : 0.f;
     for (int it = 0; it < s.nb; ++it) {
         const int c = s.nb - 1 - it;
         const auto &b = sm.buf[it & 1];
         cp_async_wait<0>();
         __syncthreads();
-        if (c > 0) fetch_prep<DK, DV>(sm.buf[(it + 1) & 1], blk(c - 1), j0, false);
-        sm.xs[it & 1][rg][j] = dov;
+        if (c > 0) fetch_prep<DK, DV>(sm.buf[(it + 1) & 1], blk(c - 1), jc, false);
+        xs[it & 1][rg][j] = dov;
         const size_t idx = (size_t)(s.slot0 + c) * H + h;
         float *dSg = p.dSst + idx * DK * DV + (size_t)i0 * DV + j0 + j;
 #pragma unroll
@@ -467,15 +477,15 @@ KDA_DEVICE void rev_chain(const BwdParams &p, ChainSm<DK> &sm) {
 #pragma unroll
         for (int m = 0; m < C / 2; ++m) {
             const float send = hi ? pk[m] : pk[m + 8], keep = hi ? pk[m + 8] : pk[m];
-            sm.red[warp][m][lane] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+            red[warp][m][lane] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
         }
         __syncthreads();
         float du = 0.f;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) du += sm.red[w][rg & 7][(rg >> 3) * 16 + j];
+        for (int w = 0; w < kWarps; ++w) du += red[w][rg & 7][(rg >> 3) * 16 + j];
 #pragma unroll
-        for (int r2 = 0; r2 < C; ++r2) du = fmaf(b.pm()[r2 * C + rg], sm.xs[it & 1][r2][j], du);  // P^T dO
-        sm.us[rg][j] = du;
+        for (int r2 = 0; r2 < C; ++r2) du = fmaf(b.pm()[r2 * C + rg], xs[it & 1][r2][j], du);  // P^T dO
+        us[rg][j] = du;
         p.dUst[idx * C * DV + (size_t)rg * DV + j0 + j] = du;
         if (c > 0) dov = load_do(c - 1);
         __syncthreads();
@@ -485,8 +495,8 @@ KDA_DEVICE void rev_chain(const BwdParams &p, ChainSm<DK> &sm) {
         for (int m = 0; m < R; ++m) dS[m] *= gc[m];
 #pragma unroll
         for (int r = 0; r < C; ++r) {
-            axpy_rows<R>(b.qd() + r * DK + i0, sm.xs[it & 1][r][j], dS);
-            axpy_rows<R>(b.w() + r * DK + i0, -sm.us[r][j], dS);
+            axpy_rows<R>(b.qd() + r * DK + i0, xs[it & 1][r][j], dS);
+            axpy_rows<R>(b.w() + r * DK + i0, -us[r][j], dS);
         }
     }
     if (p.ds0) {
@@ -499,7 +509,7 @@ KDA_DEVICE void rev_chain(const BwdParams &p, ChainSm<DK> &sm) {
 // dO, not the forward states), so one launch runs both: blockIdx.z = 0 the
 // forward pass, 1 the reverse pass.
 template <int DK, int DV, typename T>
-__global__ void __launch_bounds__(kThreads) chain_kernel(BwdParams p) {
+__global__ void __launch_bounds__(kChainThreads, 2) chain_kernel(BwdParams p) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     auto &sm = *reinterpret_cast<ChainSm<DK> *>(smem_raw);
     if (blockIdx.z == 0) fwd_chain<DK, DV, T>(p, sm);
@@ -762,13 +772,13 @@ template <typename K> cudaError_t set_smem(K kernel, size_t bytes) {
 template <int DK, int DV, typename T>
 cudaError_t launch_bwd_t(const BwdParams &p, long slots, cudaStream_t st) {
     static_assert(C * C == kThreads, "prep_kernel writes P with one thread per entry");
-    const dim3 per_chunk((unsigned)slots, (unsigned)p.H), per_seq((unsigned)(p.N * p.H), DV / NC, 2);
+    const dim3 per_chunk((unsigned)slots, (unsigned)p.H), per_seq((unsigned)(p.N * p.H), DV / (kHalves * NC), 2);
     cudaError_t e;
     if ((e = set_smem(prep_kernel<DK, DV, T>, sizeof(PrepSm<DK, DV>))) != cudaSuccess) return e;
     if ((e = set_smem(chain_kernel<DK, DV, T>, sizeof(ChainSm<DK>))) != cudaSuccess) return e;
     if ((e = set_smem(grad_kernel<DK, DV, T>, sizeof(GradSm<DK, DV>))) != cudaSuccess) return e;
     if (slots > 0) prep_kernel<DK, DV, T><<<per_chunk, kThreads, sizeof(PrepSm<DK, DV>), st>>>(p);
-    chain_kernel<DK, DV, T><<<per_seq, kThreads, sizeof(ChainSm<DK>), st>>>(p);
+    chain_kernel<DK, DV, T><<<per_seq, kChainThreads, sizeof(ChainSm<DK>), st>>>(p);
     if (slots > 0) grad_kernel<DK, DV, T><<<per_chunk, kThreads, sizeof(GradSm<DK, DV>), st>>>(p);
     return cudaGetLastError();
 }
