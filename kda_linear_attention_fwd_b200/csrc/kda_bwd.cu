@@ -50,7 +50,7 @@ using sm100::cp_async_commit;
 using sm100::cp_async_wait;
 
 constexpr int C = 16;          // tokens per chunk
-constexpr int kThreads = 256;  // every launch
+constexpr int kThreads = 256;  // prep and grad CTAs, and each half of a chain CTA
 constexpr int kWarps = kThreads / 32;
 constexpr int NC = 16;         // state columns of one half of a chain CTA
 constexpr int kHalves = 2;     // chain CTAs: two halves of 256 threads share the chunk operands
