@@ -522,8 +522,10 @@ template <int DK, int DV> struct alignas(16) GradSm {
     static constexpr int NB = kThreads / DK;   // threads per key channel
     static constexpr int LV = DV + 4;
     PrepSm<DK, DV> pr;                         // its vs holds dV once V is used
-    float us[C][LV], dus[C][LV], dos[C][LV];   // U, dU, dO
-    float dqd[C][LK], dw[C][LK], dkb[C][LK];
+    static constexpr int LM = PrepSm<DK, DV>::LM;
+    float us[C][LM];                           // U, then dKi
+    float dus[C][LV], dos[C][LV];              // dU, dO
+    float dqd[C][LK], dw[C][LK], dkb[C][LK];   // dw: dW, then dKd
     float dP[C][C], dT[C][C], M[C][C], dLs[C][C], dA[C][C];
     float dgc[DK];                             // dgamma_C
     float bs[NB][DK], ks[NB][DK];              // per row block: sum of dG, colsum of dKb (.) Kb
@@ -705,27 +707,87 @@ __global__ void __launch_bounds__(kThreads, 2) grad_kernel(BwdParams p) {
         const int r = e / DV, jj = e % DV;
         if (r < n) p.dv[((size_t)(t0 + r) * H + h) * DV + jj] = pr.vs[r][jj];
     }
-    {  // dKd = T^T dW + dA Ki, dKi = dA^T Kd + dP^T Qd, dQd += dP Ki for rows
-       // r0 .. r0 + RPT - 1 of channel i; then dq, dk, dg
+    {  // dKd = T^T dW + dA Ki, dKi = dA^T Kd + dP^T Qd, dQd += dP Ki on split-tf32 tiles
+       // (M = the 16 rows, K = 16, N = key channels); warp w takes channels 8 w NTG ..
+       // 8 (w + 1) NTG - 1 and writes its results over its own columns: dKd over dW,
+       // dKi over U (used up), dQd in place
+        constexpr int NTG = DK / 8 / (kThreads / 32);
+        const int lane = tid & 31, warp = tid >> 5, g = lane >> 2, t = lane & 3;
+        // A fragment of k-tile kt of a 16 x 16 matrix given by an element function:
+        // a0 = (g, 8kt + t), a1 = (g + 8, 8kt + t), a2 = (g, 8kt + t + 4), a3 = (g + 8, 8kt + t + 4)
+        auto a_frag = [&](auto elem, int kt, uint32_t (&ah)[4], uint32_t (&al)[4]) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) split_tf32(elem(g + 8 * (e & 1), 8 * kt + t + 4 * (e >> 1)), ah[e], al[e]);
+        };
+        auto tT = [&](int r, int q) { return pr.Tm[q][r]; };
+        auto dA = [&](int r, int q) { return sm.dA[r][q]; };
+        auto dAT = [&](int r, int q) { return sm.dA[q][r]; };
+        auto dPT = [&](int r, int q) { return sm.dP[q][r]; };
+        auto dPm = [&](int r, int q) { return sm.dP[r][q]; };
+        float dkd[NTG][4], dki[NTG][4], dqd[NTG][4];
+#pragma unroll
+        for (int nt = 0; nt < NTG; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                dkd[nt][e] = dki[nt][e] = 0.f;
+                dqd[nt][e] = sm.dqd[g + 8 * (e >> 1)][8 * (warp * NTG + nt) + 2 * t + (e & 1)];
+            }
+        // B[q][i] = X[q][i]: b0 = X[8kt + t][8nt + g], b1 = X[8kt + t + 4][8nt + g]
+#pragma unroll
+        for (int kt = 0; kt < 2; ++kt) {
+            uint32_t ah[4], al[4];
+            const int q0 = 8 * kt + t;
+            a_frag(tT, kt, ah, al);
+#pragma unroll
+            for (int nt = 0; nt < NTG; ++nt) {
+                const int i = 8 * (warp * NTG + nt) + g;
+                mma3(dkd[nt], ah, al, sm.dw[q0][i], sm.dw[q0 + 4][i]);
+            }
+            a_frag(dA, kt, ah, al);
+#pragma unroll
+            for (int nt = 0; nt < NTG; ++nt) {
+                const int i = 8 * (warp * NTG + nt) + g;
+                mma3(dkd[nt], ah, al, pr.ki[q0][i], pr.ki[q0 + 4][i]);
+            }
+            a_frag(dAT, kt, ah, al);
+#pragma unroll
+            for (int nt = 0; nt < NTG; ++nt) {
+                const int i = 8 * (warp * NTG + nt) + g;
+                mma3(dki[nt], ah, al, pr.kd[q0][i], pr.kd[q0 + 4][i]);
+            }
+            a_frag(dPT, kt, ah, al);
+#pragma unroll
+            for (int nt = 0; nt < NTG; ++nt) {
+                const int i = 8 * (warp * NTG + nt) + g;
+                mma3(dki[nt], ah, al, pr.qd[q0][i], pr.qd[q0 + 4][i]);
+            }
+            a_frag(dPm, kt, ah, al);
+#pragma unroll
+            for (int nt = 0; nt < NTG; ++nt) {
+                const int i = 8 * (warp * NTG + nt) + g;
+                mma3(dqd[nt], ah, al, pr.ki[q0][i], pr.ki[q0 + 4][i]);
+            }
+        }
+        __syncwarp();  // this warp's reads of its dW columns are done
+#pragma unroll
+        for (int nt = 0; nt < NTG; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int r = g + 8 * (e >> 1), i = 8 * (warp * NTG + nt) + 2 * t + (e & 1);
+                sm.dw[r][i] = dkd[nt][e];
+                sm.us[r][i] = dki[nt][e];
+                sm.dqd[r][i] = dqd[nt][e];
+            }
+    }
+    __syncthreads();
+    {  // dq, dk, dg for rows r0 .. r0 + RPT - 1 of channel i
         const int i = tid % DK, rb = tid / DK, r0 = rb * RPT;
         float dkd[RPT], dki[RPT], dqd[RPT];
 #pragma unroll
         for (int rr = 0; rr < RPT; ++rr) {
-            dkd[rr] = dki[rr] = 0.f;
+            dkd[rr] = sm.dw[r0 + rr][i];
+            dki[rr] = sm.us[r0 + rr][i];
             dqd[rr] = sm.dqd[r0 + rr][i];
-        }
-#pragma unroll 4
-        for (int q = 0; q < C; ++q) {
-            const float dwq = sm.dw[q][i], kiq = pr.ki[q][i], kdq = pr.kd[q][i], qdq = pr.qd[q][i];
-#pragma unroll
-            for (int rr = 0; rr < RPT; ++rr) {  // r is the same across a warp: broadcast reads
-                const int r = r0 + rr;
-                dkd[rr] = fmaf(pr.Tm[q][r], dwq, dkd[rr]);  // T^T dW
-                dkd[rr] = fmaf(sm.dA[r][q], kiq, dkd[rr]);  // dA Ki
-                dki[rr] = fmaf(sm.dA[q][r], kdq, dki[rr]);  // dA^T Kd
-                dki[rr] = fmaf(sm.dP[q][r], qdq, dki[rr]);  // dP^T Qd
-                dqd[rr] = fmaf(sm.dP[r][q], kiq, dqd[rr]);  // dP Ki
-            }
         }
         float dG[RPT], bsum = 0.f, ksum = 0.f;
 #pragma unroll
