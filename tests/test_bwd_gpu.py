@@ -1,9 +1,11 @@
 """The backward (kda_bwd) on the GPU, through the C ABI, against the fp64
 backward oracle (oracle/backward.py) on identical inputs.
 
-Tolerance: the kernel runs the recurrence and its reverse in fp32 on the
-dtype-rounded inputs, and its gradients are fp32 outputs (no output rounding),
-so each gradient gets the forward's fp32 bar scaled by its own magnitude:
+Tolerance: the kernels take the chunk form of the gradient to fp32 accuracy on
+the dtype-rounded inputs (CUDA-core fp32, and tensor-core products whose
+operands are split into two tf32 parts, leaving out terms below 2^-20
+relative), and the gradients are fp32 outputs (no output rounding), so each
+gradient gets the forward's fp32 bar scaled by its own magnitude:
 max |err| <= 1e-4 * max(1, max |ref|).  A gradient entry sums O(dk + dv)
 products per token and, through dS, contributions from the later tokens that
 decay by exp(g) per step; fp32 rounding of those sums (relative error of
@@ -54,8 +56,8 @@ def _oracle(inp, dy, dsf, scale, gate=True):
 @pytest.mark.parametrize("dtype,dk,dv", [("bf16", 128, 128), ("bf16", 64, 128),
                                           ("f32", 64, 64), ("f32", 128, 64)])
 def test_bwd_matches_oracle(cuda_lib, dtype, dk, dv):
-    """Varlen with an empty, a partial-block and multi-block sequences (16-token
-    checkpoint blocks), initial state, final-state gradient and a gate."""
+    """Varlen with an empty, a one-partial-chunk and multi-chunk sequences
+    (16-token chunks), initial state, final-state gradient and a gate."""
     w = W.custom(dtype=dtype, H=2, dk=dk, dv=dv, lengths=(0, 5, 64, 130, 300),
                  init_state=True, seed=91)
     inp = W.pack_prefill(w, device="cuda")
