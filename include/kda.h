@@ -316,8 +316,10 @@ int kda_state_compose(const float *transitions, const float *zero_states, int32_
  * Recurrent") differentiated by the chain rule: per-chunk operands in
  * parallel, a forward pass over the chunks storing the state entering each,
  * a reverse pass carrying dL/dS, then the per-chunk gradients in parallel
- * (three launches on `stream`; the two passes over the chunks share one).  fp32 arithmetic; every output element is
- * written once, so results are deterministic.
+ * (three launches on `stream`; the two passes over the chunks share one).
+ * fp32 accuracy (products with a whole state on split-tf32 tensor-core
+ * tiles); every output element is written once, so results are
+ * deterministic.
  *
  * kda_bwd_workspace_size: bytes of workspace kda_bwd needs (0 for
  *   unsupported sizes).  With ch = (total_tokens / 16 + num_seqs) * H chunk
