@@ -54,9 +54,9 @@ def peaks():
 # point, the plan and scan, the chunk kernels and their headers).  When those
 # differ from the hash (a kernel on the path changed since the capture) the
 # figure is stale and `traffic` is reported as null.
-PREFILL_SOURCES = ("kda_api.cu", "kda_args.h", "kda_plan.cu", "kda_prefill_c32.cu", "kda_prefill_mma.cu",
-                   "kda_prefill_simt.cu", "kda_prefill_tc.cu", "kda_common.cuh", "kda_prefill.cuh",
-                   "kda_sm100.cuh")
+PREFILL_SOURCES = ("kda_api.cu", "kda_args.h", "kda_chain.cu", "kda_plan.cu", "kda_prefill_c32.cu",
+                   "kda_prefill_mma.cu", "kda_prefill_simt.cu", "kda_prefill_tc.cu", "kda_common.cuh",
+                   "kda_prefill.cuh", "kda_sm100.cuh")
 
 
 def source_hash():

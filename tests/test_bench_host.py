@@ -15,10 +15,12 @@ def test_prefill_sources_exist():
     csrc = os.path.join(ROOT, "kda_linear_attention_fwd_b200", "csrc")
     for name in bench.PREFILL_SOURCES:
         assert os.path.exists(os.path.join(csrc, name)), name
-    # every prefill kernel file is covered
+    # every prefill kernel file is covered, and the plan, fold and entry points
     for name in os.listdir(csrc):
         if name.startswith("kda_prefill") or name.endswith(".cuh"):
             assert name in bench.PREFILL_SOURCES, name
+    for name in ("kda_api.cu", "kda_args.h", "kda_chain.cu", "kda_plan.cu"):
+        assert name in bench.PREFILL_SOURCES, name
 
 
 def test_traffic_is_null_when_stale(tmp_path, monkeypatch):
