@@ -105,3 +105,23 @@ def test_bwd_sampled_heads_full_size(cuda_lib):
         for name in NAMES:
             act = np32(got[name][n, h]) if name == "ds0" else np32(got[name][a:b, h])
             assert_grad_close(act, r[name], f"{name} (n={n}, h={h})")
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_bwd_decay_at_the_floor(cuda_lib, dtype):
+    """Every channel at the minimum retention in every token: the chunk form's
+    decay factors exp(-G) reach about 6e34 inside a 16-token chunk, the widest
+    range its fp32 products see; the gradients still match the oracle."""
+    import math
+    w = W.custom(dtype=dtype, H=2, dk=128, dv=128, lengths=(77, 130), init_state=True, seed=97)
+    inp = W.pack_prefill(w, device="cuda")
+    inp["g"] = torch.full_like(inp["g"], math.log(0.0067))
+    dy, dsf = _grads_in(inp, dtype, seed=98)
+    got = kda.bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["gate"], dy,
+                  inp["cu_seqlens"], scale=0.5, initial_state=inp["initial_state"],
+                  d_final_state=dsf, cu_seqlens_host=inp["cu_seqlens"].tolist())
+    torch.cuda.synchronize()
+    ref = _oracle(inp, dy, dsf, 0.5)
+    for name in NAMES:
+        assert_grad_close(np32(got[name]), ref[name], name)
