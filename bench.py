@@ -59,19 +59,23 @@ PREFILL_SOURCES = ("kda_api.cu", "kda_args.h", "kda_chain.cu", "kda_plan.cu", "k
                    "kda_prefill.cuh", "kda_sm100.cuh")
 
 
-def source_hash():
+BACKWARD_SOURCES = ("kda_bwd.cu", "kda_common.cuh", "kda_sm100.cuh")
+
+
+def source_hash(sources=PREFILL_SOURCES):
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "kda_linear_attention_fwd_b200", "csrc")
-    for name in PREFILL_SOURCES:
+    for name in sources:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 
-def measured_traffic(workload):
+def measured_traffic(workload, sources=PREFILL_SOURCES):
     """(bytes per launch of the dominant kernel, kernel name, source) or
-    (None, None, reason)."""
+    (None, None, reason); `workload` keys profiles/traffic.json, whose entry
+    holds the hash of `sources` it was captured from."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None, None, "no committed capture"
@@ -79,7 +83,7 @@ def measured_traffic(workload):
         d = json.load(f).get(workload)
     if not d:
         return None, None, "no capture for this workload"
-    if d.get("source_hash") != source_hash():
+    if d.get("source_hash") != source_hash(sources):
         return None, d.get("kernel"), "stale: kernel sources changed since the capture"
     return float(d["bytes_per_launch"]), d.get("kernel"), d.get("source", "profiles/traffic.json")
 
@@ -515,11 +519,13 @@ def main():
         bbytes = (Tb * wb.H * ((3 * wb.dk + 3 * wb.dv + 1) * e + 4 * (3 * wb.dk + 2 * wb.dv + 1))
                   + 2 * Nb * wb.H * wb.dk * wb.dv * 4)
         bgbs = bbytes / (bms / 1e3) / 1e9
+        btraffic, _, btraffic_src = measured_traffic("backward_prefill_bf16", BACKWARD_SOURCES)
         bwdm = {"value": ws * Tb / (bms / 1e3), "unit": "tokens/s", "ms_per_call": bms,
                 "workload": "prefill_bf16 backward: 2 x 4096 tokens, H=16, dk=dv=128, bf16 in, "
                             "fp32 gradients, final-state gradient given",
                 "roofline": {"bound": "hbm", "achieved": bgbs, "peak": hbm, "unit": "GB/s",
-                             "frac": bgbs / hbm, "traffic": None,
+                             "frac": bgbs / hbm, "traffic": btraffic,
+                             "traffic_source": btraffic_src,
                              "kernel": "kda_bwd call (per-chunk operands, the forward and "
                                        "reverse chains in one launch, per-chunk gradients)",
                              "peak_source": f"{pk_kind} hbm_gbs"},
